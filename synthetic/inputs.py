@@ -1,0 +1,226 @@
+"""Seeded synthetic decode-step inputs.
+
+Every tensor is drawn from its own counter-keyed PCG64 stream
+(``SeedSequence(seed, spawn_key=(tag, i, j))``), so any (batch, kv-head)
+slice can be regenerated on its own and two runs with the same seed produce
+identical bytes.  bf16 tensors are returned as their raw uint16 bit patterns
+(round-to-nearest-even from float32 draws), which both the CUDA path (as
+``torch.bfloat16``) and the CPU oracle (widened to float64) consume exactly.
+
+Workload shapes follow the five decode configurations this library is
+measured on: a tiny single-head-group step, a Qwen3-8B-shaped 32k step with
+planted "hot" blocks, a Qwen3-14B-shaped ragged batch with block size 128, a
+64k sparsity sweep and a 256-step threshold decode loop.  The pages measure
+on reasoning benchmarks (AIME, MATH-500, GPQA); these seeded N(0,1) tensors
+stand in for a model's activations on them.
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+from typing import Dict, List, Optional, Sequence, Tuple
+
+import numpy as np
+
+# stream tags
+_T_Q, _T_K, _T_V, _T_WQ, _T_WK, _T_LEN, _T_HOT, _T_PAGES = range(8)
+
+BF16_NAN_BITS = 0x7FC0
+
+
+def _rng(seed: int, *key: int) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence(seed, spawn_key=tuple(key))))
+
+
+def bf16_bits_from_f32(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to bf16 (nearest, ties to even); return uint16 bits."""
+    b = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    b = (b + 0x7FFF + ((b >> 16) & 1)) >> 16
+    return b.astype(np.uint16)
+
+
+def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    """Widen bf16 bit patterns to float32 (exact)."""
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+@dataclass(frozen=True)
+class DecodeConfig:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    head_dim: int
+    gate_dim: int
+    block: int
+    length: int = 0                       # fixed context length (tokens, incl. the current one)
+    length_range: Tuple[int, int] = (0, 0)  # ragged: uniform per sequence, never a multiple of block
+    mode: str = "topk"                    # "topk" | "threshold"
+    budget: int = 0                       # token budget (top-k)
+    tau: float = 0.0                      # score threshold (threshold mode)
+    hot_blocks: int = 0                   # planted q-aligned blocks per (b, kv head)
+    steps: int = 1                        # decode steps (one appended token each)
+    rope_base: float = 1e6
+    seed: int = 0
+
+    @property
+    def g(self) -> int:
+        return self.Hq // self.Hkv
+
+    @property
+    def topk_blocks(self) -> int:
+        return -(-self.budget // self.block)
+
+
+CONFIGS: Dict[int, DecodeConfig] = {
+    1: DecodeConfig("tiny-decode-step", B=1, Hq=4, Hkv=1, head_dim=64, gate_dim=64, block=64,
+                    length=2048, mode="topk", budget=512, seed=1001),
+    2: DecodeConfig("qwen3-8b-32k-step", B=8, Hq=32, Hkv=8, head_dim=128, gate_dim=128, block=64,
+                    length=32768, mode="topk", budget=4096, hot_blocks=8, seed=1002),
+    3: DecodeConfig("qwen3-14b-ragged-step", B=16, Hq=40, Hkv=8, head_dim=128, gate_dim=128,
+                    block=128, length_range=(8000, 32000), mode="topk", budget=4096, seed=1003),
+    4: DecodeConfig("sparsity-sweep-64k", B=4, Hq=32, Hkv=8, head_dim=128, gate_dim=128, block=64,
+                    length=65536, mode="topk", budget=6554, seed=1004),
+    5: DecodeConfig("decode-loop-256-threshold", B=32, Hq=32, Hkv=8, head_dim=128, gate_dim=128,
+                    block=64, length=16384, mode="threshold", tau=2.0 / 256.0, hot_blocks=8,
+                    steps=256, seed=1005),
+}
+
+SWEEP_SPARSITIES = (0.50, 0.75, 0.90, 0.95)
+
+
+def sweep_budget(length: int, sparsity: float) -> int:
+    """Token budget that keeps (1 - sparsity) of a `length`-token context."""
+    return int(math.ceil((1.0 - sparsity) * length - 1e-9))
+
+
+def config(cid: int, **overrides) -> DecodeConfig:
+    base = CONFIGS[cid]
+    if not overrides:
+        return base
+    d = dict(base.__dict__)
+    d.update(overrides)
+    return DecodeConfig(**d)
+
+
+@dataclass
+class DecodeInputs:
+    cfg: DecodeConfig
+    seqlens: np.ndarray            # int32 [B]  current lengths (incl. the current token)
+    final_lens: np.ndarray         # int32 [B]  lengths after all decode steps
+    q: np.ndarray                  # uint16 [B, Hq, d]    (step 0 query; also q_nope)
+    k: np.ndarray                  # uint16 [B, Hkv, Lcap, d]  (also k_nope)
+    v: np.ndarray                  # uint16 [B, Hkv, Lcap, d]
+    w_q: np.ndarray                # uint16 [Hkv, d_gate, g*d]
+    w_k: np.ndarray                # uint16 [Hkv, d_gate, 3*d]
+    hot: Dict[Tuple[int, int], List[int]] = field(default_factory=dict)
+
+    @property
+    def lcap(self) -> int:
+        return self.k.shape[2]
+
+    @property
+    def max_blocks(self) -> int:
+        return -(-self.lcap // self.cfg.block)
+
+
+def _lengths(cfg: DecodeConfig) -> np.ndarray:
+    if cfg.length_range != (0, 0):
+        lo, hi = cfg.length_range
+        rng = _rng(cfg.seed, _T_LEN)
+        out = []
+        for _ in range(cfg.B):
+            while True:
+                L = int(rng.integers(lo, hi + 1))
+                if L % cfg.block != 0:
+                    break
+            out.append(L)
+        return np.asarray(out, dtype=np.int32)
+    return np.full(cfg.B, cfg.length, dtype=np.int32)
+
+
+def make_step_query(cfg: DecodeConfig, step: int) -> np.ndarray:
+    """Query (bf16 bits, [B, Hq, d]) of decode step `step` (step 0 = the initial query)."""
+    q = np.empty((cfg.B, cfg.Hq, cfg.head_dim), dtype=np.uint16)
+    for b in range(cfg.B):
+        r = _rng(cfg.seed, _T_Q, step, b)
+        q[b] = bf16_bits_from_f32(r.standard_normal((cfg.Hq, cfg.head_dim), dtype=np.float32))
+    return q
+
+
+def make_inputs(cfg: DecodeConfig, *, tail: str = "random",
+                lengths: Optional[Sequence[int]] = None) -> DecodeInputs:
+    """Draw one decode problem.
+
+    tail="nan" fills cache rows past each sequence's final length with bf16
+    NaN, so any read of a masked token poisons the result.
+    """
+    B, Hq, Hkv, d, dg, blk = cfg.B, cfg.Hq, cfg.Hkv, cfg.head_dim, cfg.gate_dim, cfg.block
+    g = cfg.g
+    seqlens = np.asarray(lengths, dtype=np.int32) if lengths is not None else _lengths(cfg)
+    final = seqlens + (cfg.steps - 1 if cfg.steps > 1 else 0)
+    lcap = int(-(-int(final.max()) // blk) * blk) if final.max() > 0 else blk
+
+    q = make_step_query(cfg, 0)
+    q32 = bf16_bits_to_f32(q)
+
+    w_q = np.empty((Hkv, dg, g * d), dtype=np.uint16)
+    w_k = np.empty((Hkv, dg, 3 * d), dtype=np.uint16)
+    for h in range(Hkv):
+        w_q[h] = bf16_bits_from_f32(_rng(cfg.seed, _T_WQ, h).standard_normal((dg, g * d), dtype=np.float32)
+                                    / np.float32(math.sqrt(g * d)))
+        w_k[h] = bf16_bits_from_f32(_rng(cfg.seed, _T_WK, h).standard_normal((dg, 3 * d), dtype=np.float32)
+                                    / np.float32(math.sqrt(3 * d)))
+
+    k = np.empty((B, Hkv, lcap, d), dtype=np.uint16)
+    v = np.empty((B, Hkv, lcap, d), dtype=np.uint16)
+    hot: Dict[Tuple[int, int], List[int]] = {}
+    for b in range(B):
+        for h in range(Hkv):
+            kf = _rng(cfg.seed, _T_K, b, h).standard_normal((lcap, d), dtype=np.float32)
+            vf = _rng(cfg.seed, _T_V, b, h).standard_normal((lcap, d), dtype=np.float32)
+            nfull0 = int(seqlens[b]) // blk
+            if cfg.hot_blocks and nfull0 > 0:
+                qs = q32[b, h * g:(h + 1) * g].astype(np.float64).sum(axis=0)
+                qhat = (qs / np.linalg.norm(qs)).astype(np.float32)
+                chosen = sorted(int(x) for x in _rng(cfg.seed, _T_HOT, b, h).choice(
+                    nfull0, size=min(cfg.hot_blocks, nfull0), replace=False))
+                hot[(b, h)] = chosen
+                for n in chosen:
+                    kf[n * blk:(n + 1) * blk] += np.float32(3.0) * qhat
+            k[b, h] = bf16_bits_from_f32(kf)
+            v[b, h] = bf16_bits_from_f32(vf)
+            if tail == "nan":
+                k[b, h, int(final[b]):] = BF16_NAN_BITS
+                v[b, h, int(final[b]):] = BF16_NAN_BITS
+    return DecodeInputs(cfg=cfg, seqlens=seqlens, final_lens=final.astype(np.int32), q=q, k=k, v=v,
+                        w_q=w_q, w_k=w_k, hot=hot)
+
+
+def scale_gate_weights(w_q: np.ndarray, c: Sequence[float]) -> np.ndarray:
+    """Multiply W_q[h] by c[h] (a per-head logit temperature) and re-round to bf16."""
+    w = bf16_bits_to_f32(w_q).copy()
+    for h, ch in enumerate(c):
+        w[h] *= np.float32(ch)
+    return bf16_bits_from_f32(w)
+
+
+def paged_view(x: np.ndarray, block: int, seed: int, spare_pages: int = 3):
+    """Scatter a contiguous [B, Hkv, Lcap, d] cache into a shuffled page pool.
+
+    Returns (pool [P, Hkv, block, d], block_table int32 [B, Lcap // block]).
+    Page ids are a seeded permutation, so logical neighbours are not physical
+    neighbours.  Unused pool pages hold bf16 NaN.
+    """
+    B, Hkv, lcap, d = x.shape
+    assert lcap % block == 0
+    npb = lcap // block
+    P = B * npb + spare_pages
+    perm = _rng(seed, _T_PAGES).permutation(P)[: B * npb].astype(np.int32)
+    table = perm.reshape(B, npb)
+    pool = np.full((P, Hkv, block, d), BF16_NAN_BITS, dtype=np.uint16)
+    for b in range(B):
+        for n in range(npb):
+            pool[table[b, n]] = x[b, :, n * block:(n + 1) * block, :]
+    return pool, table
