@@ -1,0 +1,24 @@
+"""SeerAttention-R gated block-sparse GQA decode for NVIDIA B200 (sm_100a).
+
+The compute lives in libseer.so (C ABI: include/seer.h); the `seer` module is
+its Python binding.  Any public name resolves through `seer`, which loads the
+library and raises ImportError when it has not been built -- there is no
+fallback path.  (The lazy lookup lets `python -m <package>.build` run before
+the library exists.)
+"""
+
+_PUBLIC = (
+    "DEVERR_BLOCK_INDEX", "DEVERR_COUNT", "DEVERR_PAGE_INDEX", "DEVERR_TIMEOUT", "EXPORTED", "KV_CONTIGUOUS",
+    "KV_PAGED", "LIB_PATH", "SELECT_THRESHOLD", "SELECT_TOPK", "SELECT_TOPP", "DecodeStep", "Dims", "KVCache",
+    "KVDesc", "SeerError", "Shape", "alloc_workspace", "gate_score", "kcomp_update", "select_blocks",
+    "sparse_decode", "sparse_decode_auto_split", "sparse_decode_workspace_bytes", "version",
+)
+
+__all__ = list(_PUBLIC)
+
+
+def __getattr__(name):
+    if name in _PUBLIC:
+        from . import seer
+        return getattr(seer, name)
+    raise AttributeError(name)

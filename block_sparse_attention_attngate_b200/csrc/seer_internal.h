@@ -1,0 +1,115 @@
+// Internal launch interface between the C ABI layer (seer_api.cu) and the
+// kernel translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+
+namespace seer {
+
+// Raise a kernel's dynamic shared-memory limit once per device (a host-side
+// attribute call, kept out of CUDA-graph capture after the first use).
+template <typename Kernel>
+cudaError_t ensure_smem_limit(Kernel kern, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = uint64_t(1) << (dev & 63);
+  if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
+
+constexpr int kMaxGroup = 8;        // query heads per KV head
+constexpr int kMaxBlocksRow = 8192; // max_blocks limit (selection keeps a row in shared memory)
+
+// Where a K/V tile lives, for kernels that read it with plain loads.
+struct KvPlain {
+  const uint16_t* data;
+  int64_t stride_b, stride_h, stride_t;   // elements
+  const int32_t* block_table;             // paged only
+  int32_t max_pages;
+  int64_t num_pages;
+  int64_t num_tokens;                     // contiguous only: token capacity
+  int32_t paged;
+};
+
+// ---------------------------------------------------------------- kcomp update
+struct KcompParams {
+  KvPlain k;
+  const int32_t* seqlens;
+  const int32_t* valid;
+  int32_t* valid_out;
+  const uint16_t* w_k;     // [Hkv, DG, 3D]
+  uint16_t* kcomp;         // [B, Hkv, NB, DG]
+  int32_t B, Hkv, NB;
+  float rope_base;
+  int32_t* err;
+};
+cudaError_t launch_kcomp_update(const KcompParams& p, int D, int BLK, int DG, int grid_x,
+                                cudaStream_t s);
+
+// ---------------------------------------------------------------- gate score
+struct GateParams {
+  const uint16_t* q;       // [B, Hq, D]
+  const uint16_t* w_q;     // [Hkv, DG, g*D]
+  const uint16_t* kcomp;   // [B, Hkv, NB, DG]
+  const int32_t* seqlens;
+  float* logits;           // [B, Hkv, NB]
+  float* q_gate;           // [B, Hkv, DG] or null
+  int32_t B, Hq, Hkv, g, NB, BLK;
+  float rope_base;
+};
+cudaError_t launch_gate_score(const GateParams& p, int D, int DG, cudaStream_t s);
+
+// ---------------------------------------------------------------- select
+struct SelectParams {
+  const float* logits;     // [B, Hkv, NB]
+  const int32_t* seqlens;
+  int32_t* idx;            // [B, Hkv, cap]
+  int32_t* cnt;            // [B, Hkv]
+  int32_t B, Hkv, NB, BLK, cap;
+  int32_t mode;            // 0 top-k, 1 threshold, 2 top-p
+  int32_t kblocks;         // top-k
+  double tau;              // threshold / top-p mass
+};
+cudaError_t launch_select(const SelectParams& p, cudaStream_t s);
+
+// ---------------------------------------------------------------- sparse decode
+struct DecodeParams {
+  const uint16_t* q;        // [B, Hq, D]
+  const int32_t* idx;       // [B, Hkv, cap]
+  const int32_t* cnt;       // [B, Hkv]
+  const int32_t* seqlens;   // [B]
+  const int32_t* k_table;   // paged block tables (may be equal)
+  const int32_t* v_table;
+  int32_t k_maxp, v_maxp;
+  int64_t k_pages, v_pages;
+  int32_t k_paged, v_paged;
+  int32_t k_perm[3], v_perm[3];   // TMA dim (1..3) that holds token / head / batch-or-page
+  int32_t B, Hq, Hkv, g;
+  int32_t cap, ns, per_split;
+  float scale_log2;         // softmax scale * log2(e)
+  float* o_part;            // [B, Hq, ns, D]
+  float* lse_part;          // [B, Hq, ns]
+  int32_t* counters;        // [B, Hkv]
+  uint16_t* out;            // [B, Hq, D] bf16
+  float* lse_out;           // [B, Hq] or null
+  int32_t* err;
+};
+struct DecodeConfig {
+  int stages;
+  int warps;       // consumer warps
+  size_t smem;
+};
+DecodeConfig decode_config(int D, int BLK);
+cudaError_t launch_sparse_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
+                                 int D, int BLK, cudaStream_t s);
+int decode_ctas_per_sm(int D, int BLK);
+
+}  // namespace seer

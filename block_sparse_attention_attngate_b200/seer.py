@@ -1,0 +1,272 @@
+"""Thin Python binding of libseer (include/seer.h).
+
+Argument marshalling only: every step of the decode path runs in the CUDA
+kernels behind the C ABI.  Tensors are torch CUDA tensors; torch provides
+device memory and the current stream, nothing else.  If libseer.so is missing
+this module raises at import time -- there is no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libseer.so")
+
+SEER_OK, SEER_ERR_INVALID_ARG, SEER_ERR_UNSUPPORTED, SEER_ERR_CAPACITY, SEER_ERR_CUDA = range(5)
+STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CAPACITY", 4: "CUDA"}
+KV_CONTIGUOUS, KV_PAGED = 0, 1
+SELECT_TOPK, SELECT_THRESHOLD, SELECT_TOPP = 0, 1, 2
+DEVERR_BLOCK_INDEX, DEVERR_PAGE_INDEX, DEVERR_COUNT, DEVERR_TIMEOUT = 1, 2, 4, 8
+
+EXPORTED = (
+    "seer_kcomp_update", "seer_gate_score", "seer_select_blocks", "seer_sparse_decode_auto_split",
+    "seer_sparse_decode_workspace_bytes", "seer_sparse_decode", "seer_last_error", "seer_version",
+)
+
+
+class SeerError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"libseer {STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("gate_dim", ctypes.c_int32), ("block_size", ctypes.c_int32),
+                ("max_blocks", ctypes.c_int32), ("rope_base", ctypes.c_float), ("softmax_scale", ctypes.c_float)]
+
+
+class KVDesc(ctypes.Structure):
+    _fields_ = [("layout", ctypes.c_int32), ("data", ctypes.c_void_p), ("stride_b", ctypes.c_int64),
+                ("stride_h", ctypes.c_int64), ("stride_t", ctypes.c_int64), ("num_tokens", ctypes.c_int64),
+                ("num_pages", ctypes.c_int64), ("block_table", ctypes.c_void_p),
+                ("max_pages_per_seq", ctypes.c_int32)]
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with `python -m block_sparse_attention_attngate_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I32, I64, F32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    DP, KP = ctypes.POINTER(Dims), ctypes.POINTER(KVDesc)
+    sig = {
+        "seer_kcomp_update": (I32, [DP, KP, P, P, P, P, P]),
+        "seer_gate_score": (I32, [DP, P, P, P, P, P, P, P]),
+        "seer_select_blocks": (I32, [DP, P, P, I32, I32, F32, P, P, I32, P]),
+        "seer_sparse_decode_auto_split": (I32, [DP, I32]),
+        "seer_sparse_decode_workspace_bytes": (SZ, [DP, I32, I32]),
+        "seer_sparse_decode": (I32, [DP, P, KP, KP, P, P, P, I32, I32, P, SZ, P, P, P, P]),
+        "seer_last_error": (ctypes.c_char_p, []),
+        "seer_version": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = load_library()
+
+
+def version() -> str:
+    return _lib.seer_version().decode()
+
+
+def _check(status: int):
+    if status != SEER_OK:
+        raise SeerError(status, _lib.seer_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, dtype: torch.dtype, name: str, contiguous: bool = True):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+@dataclass
+class Shape:
+    """Problem shape of one attention layer (mirrors seer_dims_t)."""
+    batch: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    gate_dim: int
+    block_size: int
+    max_blocks: int
+    rope_base: float = 1e6
+    softmax_scale: float = 0.0
+
+    def c(self) -> Dims:
+        return Dims(self.batch, self.num_q_heads, self.num_kv_heads, self.head_dim, self.gate_dim,
+                    self.block_size, self.max_blocks, self.rope_base, self.softmax_scale)
+
+    @property
+    def group(self) -> int:
+        return self.num_q_heads // self.num_kv_heads
+
+
+class KVCache:
+    """A bf16 K or V cache as the library sees it (contiguous or paged)."""
+
+    def __init__(self, desc: KVDesc, keep):
+        self.desc = desc
+        self._keep = keep
+
+    @classmethod
+    def contiguous(cls, t: torch.Tensor) -> "KVCache":
+        """t: [B, Hkv, T, d] view (any strides with unit-stride head_dim)."""
+        _need(t, torch.bfloat16, "kv cache", contiguous=False)
+        if t.dim() != 4 or t.stride(3) != 1:
+            raise ValueError("contiguous KV cache must be a 4-D [B, Hkv, T, d] view with unit-stride d")
+        d = KVDesc(KV_CONTIGUOUS, t.data_ptr(), t.stride(0), t.stride(1), t.stride(2), t.shape[2], 0, None, 0)
+        return cls(d, (t,))
+
+    @classmethod
+    def paged(cls, pool: torch.Tensor, block_table: torch.Tensor) -> "KVCache":
+        """pool: [P, Hkv, block, d]; block_table: int32 [B, max_pages_per_seq]."""
+        _need(pool, torch.bfloat16, "page pool", contiguous=False)
+        _need(block_table, torch.int32, "block_table")
+        if pool.dim() != 4 or pool.stride(3) != 1:
+            raise ValueError("page pool must be a 4-D [P, Hkv, block, d] view with unit-stride d")
+        d = KVDesc(KV_PAGED, pool.data_ptr(), pool.stride(0), pool.stride(1), pool.stride(2), 0, pool.shape[0],
+                   block_table.data_ptr(), block_table.shape[1])
+        return cls(d, (pool, block_table))
+
+
+def kcomp_update(shape: Shape, k_nope: KVCache, seqlens: torch.Tensor, valid_blocks: torch.Tensor,
+                 w_k: torch.Tensor, kcomp: torch.Tensor, stream=None):
+    _need(seqlens, torch.int32, "seqlens")
+    _need(valid_blocks, torch.int32, "valid_blocks")
+    _need(w_k, torch.bfloat16, "w_k")
+    _need(kcomp, torch.bfloat16, "kcomp")
+    dims = shape.c()
+    _check(_lib.seer_kcomp_update(ctypes.byref(dims), ctypes.byref(k_nope.desc), _ptr(seqlens),
+                                  _ptr(valid_blocks), _ptr(w_k), _ptr(kcomp), _stream(stream)))
+
+
+def gate_score(shape: Shape, q_nope: torch.Tensor, w_q: torch.Tensor, kcomp: torch.Tensor, seqlens: torch.Tensor,
+               logits: torch.Tensor, q_gate: Optional[torch.Tensor] = None, stream=None):
+    _need(q_nope, torch.bfloat16, "q_nope")
+    _need(w_q, torch.bfloat16, "w_q")
+    _need(kcomp, torch.bfloat16, "kcomp")
+    _need(seqlens, torch.int32, "seqlens")
+    _need(logits, torch.float32, "logits")
+    if q_gate is not None:
+        _need(q_gate, torch.float32, "q_gate")
+    dims = shape.c()
+    _check(_lib.seer_gate_score(ctypes.byref(dims), _ptr(q_nope), _ptr(w_q), _ptr(kcomp), _ptr(seqlens),
+                                _ptr(logits), _ptr(q_gate), _stream(stream)))
+
+
+def select_blocks(shape: Shape, logits: torch.Tensor, seqlens: torch.Tensor, mode: int, block_idx: torch.Tensor,
+                  block_cnt: torch.Tensor, token_budget: int = 0, tau: float = 0.0, stream=None):
+    _need(logits, torch.float32, "logits")
+    _need(seqlens, torch.int32, "seqlens")
+    _need(block_idx, torch.int32, "block_idx")
+    _need(block_cnt, torch.int32, "block_cnt")
+    dims = shape.c()
+    _check(_lib.seer_select_blocks(ctypes.byref(dims), _ptr(logits), _ptr(seqlens), int(mode), int(token_budget),
+                                   float(tau), _ptr(block_idx), _ptr(block_cnt), block_idx.shape[-1],
+                                   _stream(stream)))
+
+
+def sparse_decode_auto_split(shape: Shape, capacity: int) -> int:
+    dims = shape.c()
+    return int(_lib.seer_sparse_decode_auto_split(ctypes.byref(dims), int(capacity)))
+
+
+def sparse_decode_workspace_bytes(shape: Shape, capacity: int, num_split: int = 0) -> int:
+    dims = shape.c()
+    return int(_lib.seer_sparse_decode_workspace_bytes(ctypes.byref(dims), int(capacity), int(num_split)))
+
+
+def alloc_workspace(shape: Shape, capacity: int, num_split: int = 0, device=None) -> torch.Tensor:
+    """Zero-filled workspace (the arrival counters must start at zero)."""
+    n = sparse_decode_workspace_bytes(shape, capacity, num_split)
+    return torch.zeros(max(n, 16), dtype=torch.uint8, device=device or "cuda")
+
+
+def sparse_decode(shape: Shape, q: torch.Tensor, k: KVCache, v: KVCache, block_idx: torch.Tensor,
+                  block_cnt: torch.Tensor, seqlens: torch.Tensor, out: torch.Tensor, workspace: Optional[torch.Tensor],
+                  num_split: int = 0, lse: Optional[torch.Tensor] = None, err: Optional[torch.Tensor] = None,
+                  stream=None):
+    _need(q, torch.bfloat16, "q")
+    _need(block_idx, torch.int32, "block_idx")
+    _need(block_cnt, torch.int32, "block_cnt")
+    _need(seqlens, torch.int32, "seqlens")
+    _need(out, torch.bfloat16, "out")
+    if lse is not None:
+        _need(lse, torch.float32, "lse")
+    if err is not None:
+        _need(err, torch.int32, "err")
+    dims = shape.c()
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.seer_sparse_decode(ctypes.byref(dims), _ptr(q), ctypes.byref(k.desc), ctypes.byref(v.desc),
+                                   _ptr(block_idx), _ptr(block_cnt), _ptr(seqlens), block_idx.shape[-1],
+                                   int(num_split), _ptr(workspace), ws_bytes, _ptr(out), _ptr(lse), _ptr(err),
+                                   _stream(stream)))
+
+
+class DecodeStep:
+    """One layer's per-step pipeline: kcomp_update -> gate_score -> select_blocks -> sparse_decode.
+
+    Owns the step's scratch tensors (logits, index lists, workspace, output) so a
+    decode loop (or a CUDA graph capturing `run`) reuses them every step.
+    """
+
+    def __init__(self, shape: Shape, k: KVCache, v: KVCache, w_q: torch.Tensor, w_k: torch.Tensor,
+                 kcomp: torch.Tensor, valid_blocks: torch.Tensor, mode: int = SELECT_TOPK, token_budget: int = 0,
+                 tau: float = 0.0, capacity: Optional[int] = None, num_split: int = 0, k_nope: Optional[KVCache] = None,
+                 device=None):
+        dev = device or w_q.device
+        self.shape, self.k, self.v, self.w_q, self.w_k = shape, k, v, w_q, w_k
+        self.k_nope = k_nope or k
+        self.kcomp, self.valid_blocks = kcomp, valid_blocks
+        self.mode, self.token_budget, self.tau = mode, token_budget, tau
+        if capacity is None:
+            if mode == SELECT_TOPK:
+                capacity = min(shape.max_blocks, -(-token_budget // shape.block_size) + 1)
+            else:
+                capacity = shape.max_blocks
+        self.capacity = capacity
+        B, Hq, Hkv = shape.batch, shape.num_q_heads, shape.num_kv_heads
+        self.logits = torch.empty(B, Hkv, shape.max_blocks, dtype=torch.float32, device=dev)
+        self.block_idx = torch.empty(B, Hkv, capacity, dtype=torch.int32, device=dev)
+        self.block_cnt = torch.empty(B, Hkv, dtype=torch.int32, device=dev)
+        self.num_split = num_split if num_split > 0 else sparse_decode_auto_split(shape, capacity)
+        self.workspace = alloc_workspace(shape, capacity, self.num_split, dev)
+        self.out = torch.empty(B, Hq, shape.head_dim, dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def run(self, q: torch.Tensor, seqlens: torch.Tensor, q_nope: Optional[torch.Tensor] = None, stream=None):
+        s = self.shape
+        kcomp_update(s, self.k_nope, seqlens, self.valid_blocks, self.w_k, self.kcomp, stream)
+        gate_score(s, q if q_nope is None else q_nope, self.w_q, self.kcomp, seqlens, self.logits, None, stream)
+        select_blocks(s, self.logits, seqlens, self.mode, self.block_idx, self.block_cnt, self.token_budget,
+                      self.tau, stream)
+        sparse_decode(s, q, self.k, self.v, self.block_idx, self.block_cnt, seqlens, self.out, self.workspace,
+                      self.num_split, self.lse, self.err, stream)
+        return self.out
+
+    KERNELS_PER_STEP = 5   # kcomp update + commit, gate, select, decode

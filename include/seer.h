@@ -1,0 +1,221 @@
+/*
+ * seer.h -- C ABI of libseer: SeerAttention-R's gated block-sparse GQA decode
+ * step on NVIDIA B200 (sm_100a).
+ *
+ * Sources, cited by page and section:
+ *   [CP] "SeerAttention-R: Sparse Attention Adaptation for Long Reasoning"
+ *        (chapterpal.com summary): Knowl 1-2 (AttnGate), Knowl 5 (K
+ *        Compression Cache, token budget and threshold), Knowl 6 (block-sparse
+ *        flash decoding on a (batch, heads_kv, num_split) grid), Knowl 14
+ *        (PagedAttention support).
+ *   [PN] "Sparse Attention Adaptation for Long Reasoning" (papernotes.org
+ *        notes): key designs 1, 2 and 4.
+ *
+ * One decode step of one attention layer is
+ *     seer_kcomp_update -> seer_gate_score -> seer_select_blocks -> seer_sparse_decode
+ *
+ * Conventions shared by every call
+ *   - The caller owns all memory.  The library never allocates or frees.
+ *   - Every pointer argument named "device" is a CUDA device pointer on the
+ *     current device; arguments of type seer_dims_t* / seer_kv_t* are HOST
+ *     pointers read during the call only.
+ *   - Every call only enqueues kernels on `stream` (a cudaStream_t, NULL =
+ *     legacy default stream) and returns without synchronising the host.
+ *   - Sequence lengths L_b (`seqlens`) count the tokens in the cache,
+ *     including the token being decoded.  nfull_b = floor(L_b / b) full
+ *     blocks; block nfull_b is partial when L_b mod b != 0.
+ *   - bf16 tensors are IEEE bfloat16.  Query head i belongs to KV head
+ *     floor(i / g), g = Hq / Hkv.
+ *   - Device pointers must be 16-byte aligned.
+ *   - Supported shapes: head_dim in {64, 128}; block_size in {64, 128};
+ *     gate_dim in {64, 128}; 1 <= g <= 8; max_blocks <= 8192.  Anything else
+ *     returns SEER_ERR_UNSUPPORTED before any work is enqueued.
+ *   - On a non-OK status nothing has been enqueued (argument errors) or the
+ *     launch failed (SEER_ERR_CUDA); seer_last_error() gives the reason.
+ *   - Anomalies that only the device can see (a block index outside
+ *     [0, ceil(L_b/b)), a page id outside the pool, a count above the
+ *     capacity, a pipeline wait that timed out) never trap: the kernel skips
+ *     the offending work and ORs a SEER_DEVERR_* bit into *err_word when the
+ *     call was given one.
+ */
+#ifndef SEER_H
+#define SEER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SEER_OK = 0,
+  SEER_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned pointer or stride */
+  SEER_ERR_UNSUPPORTED = 2, /* shape outside the supported set above */
+  SEER_ERR_CAPACITY = 3,    /* index tensor width too small for the selection mode */
+  SEER_ERR_CUDA = 4         /* a CUDA runtime/driver call failed */
+} seer_status;
+
+/* Bits ORed into the optional device error word. */
+#define SEER_DEVERR_BLOCK_INDEX 1  /* selected block index outside [0, ceil(L/b)) */
+#define SEER_DEVERR_PAGE_INDEX 2   /* block_table entry outside [0, num_pages) */
+#define SEER_DEVERR_COUNT 4        /* block count above capacity */
+#define SEER_DEVERR_TIMEOUT 8      /* a pipeline wait exceeded its bound */
+
+typedef enum { SEER_KV_CONTIGUOUS = 0, SEER_KV_PAGED = 1 } seer_kv_layout;
+
+/*
+ * A K or V cache (bf16).  head_dim elements of one token are contiguous.
+ *   SEER_KV_CONTIGUOUS: element (b, h, t, c) at data + b*stride_b + h*stride_h + t*stride_t + c,
+ *     t < num_tokens (the cache's token capacity).
+ *   SEER_KV_PAGED (PagedAttention-style [CP Knowl 14], page size == block_size):
+ *     token t of sequence b lives in page p = block_table[b*max_pages_per_seq + t/block_size]
+ *     at data + p*stride_b + h*stride_h + (t % block_size)*stride_t + c, p < num_pages.
+ * Strides are in elements; stride_t, stride_h and stride_b must be multiples of 8
+ * (16 bytes) for the TMA tile loads.
+ */
+typedef struct {
+  int32_t layout;             /* seer_kv_layout */
+  const void* data;           /* device, bf16 */
+  int64_t stride_b;           /* contiguous: per sequence; paged: per page */
+  int64_t stride_h;           /* per KV head */
+  int64_t stride_t;           /* per token */
+  int64_t num_tokens;         /* contiguous: token capacity per (b, h); paged: ignored */
+  int64_t num_pages;          /* paged: pages in the pool; contiguous: ignored */
+  const int32_t* block_table; /* paged: device int32 [B, max_pages_per_seq]; contiguous: NULL */
+  int32_t max_pages_per_seq;  /* paged: row length of block_table */
+} seer_kv_t;
+
+/* Problem shape shared by all calls of one layer. */
+typedef struct {
+  int32_t batch;        /* B */
+  int32_t num_q_heads;  /* Hq */
+  int32_t num_kv_heads; /* Hkv (Hq must be a multiple) */
+  int32_t head_dim;     /* d */
+  int32_t gate_dim;     /* d_gate: AttnGate hidden size per KV head [CP Knowl 1] */
+  int32_t block_size;   /* b: sparse block = pooling kernel/stride = page size */
+  int32_t max_blocks;   /* row length of kcomp and logits; must cover ceil(L_b/b) for every b */
+  float rope_base;      /* RoPE base inside the gate (e.g. 1e6) */
+  float softmax_scale;  /* attention scale; 0 selects 1/sqrt(head_dim) */
+} seer_dims_t;
+
+/*
+ * seer_kcomp_update -- K Compression Cache maintenance [CP Knowl 5; PN design 2, 4].
+ *
+ * For every sequence b and KV head h and every block n with
+ * valid_blocks[b] <= n < floor(seqlens[b] / b):
+ *   p = [max | min | avg] over the b pre-RoPE keys of block n (per channel, 3d values)
+ *   kcomp[b, h, n, :] = bf16( RoPE_{n*b}( W_k[h] . p ) )      (RoPE rotate-half, theta_i = base^(-2i/d_gate))
+ * then valid_blocks[b] = floor(seqlens[b] / b).  Entries below valid_blocks[b] are not
+ * touched, so calling this every decode step recomputes a block exactly once, when it
+ * fills; valid_blocks = 0 rebuilds the whole cache (prefill).
+ *
+ *   k_nope        pre-RoPE key cache (see seer_kv_t); may alias the attention K cache
+ *   seqlens       device int32 [B]
+ *   valid_blocks  device int32 [B], read then written
+ *   w_k           device bf16 [Hkv, d_gate, 3*d]  (no bias)
+ *   kcomp         device bf16 [B, Hkv, max_blocks, d_gate]
+ * Enqueues two kernels (update, then the valid_blocks write).
+ */
+seer_status seer_kcomp_update(const seer_dims_t* dims, const seer_kv_t* k_nope,
+                              const int32_t* seqlens, int32_t* valid_blocks, const void* w_k,
+                              void* kcomp, void* stream);
+
+/*
+ * seer_gate_score -- AttnGate block logits [CP Knowl 1-2; PN design 1].
+ *
+ *   Q_gate[b, h] = RoPE_{L_b - 1}( W_q[h] . concat_j q_nope[b, h*g + j, :] )   (fp32, not rounded)
+ *   logits[b, h, n] = <Q_gate[b, h], kcomp[b, h, n]> / sqrt(d_gate)   for n < floor(L_b / b)
+ *   logits[b, h, n] = -inf                                             for floor(L_b/b) <= n < max_blocks
+ * softmax over n of the logits is the gate score S.
+ *
+ *   q_nope      device bf16 [B, Hq, d]  (pre-RoPE query of the current token)
+ *   w_q         device bf16 [Hkv, d_gate, g*d]  (one projection per KV head, no bias)
+ *   kcomp       device bf16 [B, Hkv, max_blocks, d_gate]
+ *   seqlens     device int32 [B]
+ *   logits      device fp32 [B, Hkv, max_blocks]  (written)
+ *   q_gate_out  device fp32 [B, Hkv, d_gate] or NULL
+ */
+seer_status seer_gate_score(const seer_dims_t* dims, const void* q_nope, const void* w_q,
+                            const void* kcomp, const int32_t* seqlens, float* logits,
+                            float* q_gate_out, void* stream);
+
+#define SEER_SELECT_TOPK 0
+#define SEER_SELECT_THRESHOLD 1
+#define SEER_SELECT_TOPP 2
+
+/*
+ * seer_select_blocks -- logits -> block index lists [CP Knowl 5, Knowl 14].
+ *
+ * Per (b, h), over the nfull = floor(L_b/b) full blocks:
+ *   SEER_SELECT_TOPK:      k = ceil(token_budget / b); the min(k, nfull) blocks with the largest
+ *                          logits, ties to the lower block index.  Capacity >= k + 1.
+ *   SEER_SELECT_THRESHOLD: S = softmax(logits[0:nfull]); blocks with S > tau (strict).
+ *                          Capacity >= max_blocks.  S and the comparison are evaluated in fp64.
+ *   SEER_SELECT_TOPP:      fewest blocks, in descending S order (ties to the lower index),
+ *                          whose S-sum reaches tau (used as p).  Capacity >= max_blocks.
+ * In every mode the partial block nfull is appended when L_b mod b != 0.
+ * Output rows list the chosen indices ascending, then -1 up to `capacity`.
+ *
+ *   logits     device fp32 [B, Hkv, max_blocks]
+ *   seqlens    device int32 [B]
+ *   block_idx  device int32 [B, Hkv, capacity]  (written)
+ *   block_cnt  device int32 [B, Hkv]            (written)
+ */
+seer_status seer_select_blocks(const seer_dims_t* dims, const float* logits,
+                               const int32_t* seqlens, int32_t mode, int32_t token_budget,
+                               float tau, int32_t* block_idx, int32_t* block_cnt,
+                               int32_t capacity, void* stream);
+
+/* Split count seer_sparse_decode uses when num_split == 0 (host heuristic, no device reads). */
+int32_t seer_sparse_decode_auto_split(const seer_dims_t* dims, int32_t capacity);
+
+/*
+ * Workspace bytes seer_sparse_decode needs for `num_split` (0 = auto) splits: per-split partial
+ * outputs and LSEs plus one arrival counter per (b, h).  The counters must be zero before the
+ * first call (e.g. allocate zero-filled); every completed call leaves them zero again.
+ */
+size_t seer_sparse_decode_workspace_bytes(const seer_dims_t* dims, int32_t capacity,
+                                          int32_t num_split);
+
+/*
+ * seer_sparse_decode -- block-sparse flash decoding + split LSE combine [CP Knowl 6; PN design 4].
+ *
+ * For each query head i of KV head h (GQA group shares the list [PN design 1]):
+ *   T = union over the first block_cnt[b, h] entries n of block_idx[b, h, :] of tokens
+ *       [n*b, min((n+1)*b, L_b))
+ *   out[b, i] = sum_{t in T} softmax_t(scale * q[b,i] . K[b,h,t]) V[b,h,t]
+ *   lse_out[b, i] = log sum_{t in T} exp(scale * q[b,i] . K[b,h,t])   (-inf, out = 0 when T is empty)
+ * The list is split along num_split slices of ceil(capacity / num_split) positions (the split
+ * size comes from the index tensor width, max_selected_blocks, not from the sequence length);
+ * grid (num_split, Hkv, B); the last CTA of each (b, h) merges the partial results.
+ *
+ *   q          device bf16 [B, Hq, d]  (post-RoPE query, as the model uses it)
+ *   k, v       K and V caches (see seer_kv_t)
+ *   block_idx  device int32 [B, Hkv, capacity]; block_cnt device int32 [B, Hkv]
+ *   seqlens    device int32 [B]
+ *   num_split  0 = seer_sparse_decode_auto_split(); must match the workspace size
+ *   workspace  device, >= seer_sparse_decode_workspace_bytes(dims, capacity, num_split) bytes
+ *   out        device bf16 [B, Hq, d]
+ *   lse_out    device fp32 [B, Hq] or NULL
+ *   err_word   device int32 or NULL (SEER_DEVERR_* bits ORed in)
+ * Calls on the same workspace must not overlap on the GPU.
+ */
+seer_status seer_sparse_decode(const seer_dims_t* dims, const void* q, const seer_kv_t* k,
+                               const seer_kv_t* v, const int32_t* block_idx,
+                               const int32_t* block_cnt, const int32_t* seqlens,
+                               int32_t capacity, int32_t num_split, void* workspace,
+                               size_t workspace_bytes, void* out, float* lse_out,
+                               int32_t* err_word, void* stream);
+
+/* Thread-local text describing the last non-OK status returned on this thread. */
+const char* seer_last_error(void);
+
+/* Library version string. */
+const char* seer_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SEER_H */

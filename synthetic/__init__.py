@@ -12,7 +12,9 @@ from .inputs import (  # noqa: F401
     bf16_bits_from_f32,
     bf16_bits_to_f32,
     config,
+    make_block_lists,
     make_inputs,
+    make_logits,
     make_step_query,
     paged_view,
     scale_gate_weights,

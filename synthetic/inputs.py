@@ -83,7 +83,7 @@ CONFIGS: Dict[int, DecodeConfig] = {
     4: DecodeConfig("sparsity-sweep-64k", B=4, Hq=32, Hkv=8, head_dim=128, gate_dim=128, block=64,
                     length=65536, mode="topk", budget=6554, seed=1004),
     5: DecodeConfig("decode-loop-256-threshold", B=32, Hq=32, Hkv=8, head_dim=128, gate_dim=128,
-                    block=64, length=16384, mode="threshold", tau=2.0 / 256.0, hot_blocks=8,
+                    block=64, length=16384, mode="threshold", tau=1.0 / 512.0, hot_blocks=8,
                     steps=256, seed=1005),
 }
 
@@ -224,3 +224,37 @@ def paged_view(x: np.ndarray, block: int, seed: int, spare_pages: int = 3):
         for n in range(npb):
             pool[table[b, n]] = x[b, :, n * block:(n + 1) * block, :]
     return pool, table
+
+
+_T_LOGITS, _T_LISTS = 8, 9
+
+
+def make_logits(seed: int, B: int, Hkv: int, nb: int, kind: str = "normal") -> np.ndarray:
+    """float32 [B, Hkv, nb] score rows: N(0, 2^2) draws, or small integers (many exact ties)."""
+    r = _rng(seed, _T_LOGITS)
+    if kind == "ties":
+        return r.integers(-3, 4, size=(B, Hkv, nb)).astype(np.float32)
+    return (r.standard_normal((B, Hkv, nb)) * 2.0).astype(np.float32)
+
+
+def make_block_lists(seed: int, seqlens: Sequence[int], Hkv: int, block: int, capacity: int,
+                     density: float = 0.3, force_partial: bool = True):
+    """Random ascending block lists: idx int32 [B, Hkv, capacity] (-1 padded), cnt int32 [B, Hkv].
+
+    Each full block is kept with probability `density` (at most capacity - 1 of
+    them); the partial last block is appended when the length leaves one.
+    """
+    r = _rng(seed, _T_LISTS)
+    B = len(seqlens)
+    idx = np.full((B, Hkv, capacity), -1, dtype=np.int32)
+    cnt = np.zeros((B, Hkv), dtype=np.int32)
+    for b in range(B):
+        L = int(seqlens[b])
+        nfull = L // block
+        for h in range(Hkv):
+            keep = [n for n in range(nfull) if r.random() < density][: capacity - 1]
+            if force_partial and L % block:
+                keep.append(nfull)
+            idx[b, h, :len(keep)] = keep
+            cnt[b, h] = len(keep)
+    return idx, cnt

@@ -1,0 +1,147 @@
+"""Shared helpers of the GPU parity tests: upload seeded inputs, run the oracle
+per (batch, kv head), and compare with the tolerances the parity contract fixes.
+
+Tolerances (restated from the parity contract of the decode path):
+  * gate logits: |gpu - oracle| <= 1e-3 * max(|oracle|, rms(oracle row)) per (b, h)
+  * block indices: identical (threshold mode: a difference is allowed only
+    for a block whose oracle score lies within 1e-6 relative of tau)
+  * attention output: max-abs <= 1e-2 and relative L2 <= 5e-3 against the
+    float64 oracle on the same block lists
+  * kcomp: within one bf16 ulp of the oracle
+"""
+
+from __future__ import annotations
+
+import math
+from typing import Dict, List, Sequence, Tuple
+
+import numpy as np
+import torch
+
+from oracle import seer_oracle as O
+from synthetic import DecodeInputs
+
+LOGIT_RTOL = 1e-3
+OUT_MAX_ABS = 1e-2
+OUT_REL_L2 = 5e-3
+LSE_ABS = 2e-3
+THRESH_REL = 1e-6
+
+
+def to_dev_bf16(bits: np.ndarray, device="cuda") -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(device).view(torch.bfloat16)
+
+
+def bf16_bits(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def f64(bits) -> np.ndarray:
+    return O.bf16_to_f64(bits)
+
+
+class OracleBH:
+    """Oracle results of one (b, kv-head) of a DecodeInputs problem (computed lazily, cached)."""
+
+    def __init__(self, inp: DecodeInputs, b: int, h: int):
+        self.inp, self.b, self.h = inp, b, h
+        c = inp.cfg
+        self.g, self.blk = c.g, c.block
+        self._k = None
+        self._v = None
+        self._kc = None
+
+    @property
+    def k(self):
+        if self._k is None:
+            self._k = f64(self.inp.k[self.b, self.h])
+        return self._k
+
+    @property
+    def v(self):
+        if self._v is None:
+            self._v = f64(self.inp.v[self.b, self.h])
+        return self._v
+
+    def kcomp(self, length: int) -> np.ndarray:
+        """Cache built incrementally up to `length` (entries of full blocks only)."""
+        nb = self.inp.max_blocks
+        if self._kc is None:
+            self._kc = (np.zeros((nb, self.inp.cfg.gate_dim)), 0)
+        kc, valid = self._kc
+        valid = O.kcomp_update(self.k, length, valid, f64(self.inp.w_k[self.h]), kc, self.blk, self.inp.cfg.rope_base)
+        self._kc = (kc, valid)
+        return kc
+
+    def q_group(self, q_bits: np.ndarray) -> np.ndarray:
+        return f64(q_bits[self.b, self.h * self.g:(self.h + 1) * self.g])
+
+    def step(self, length: int, q_bits: np.ndarray, mode: str, k_blocks: int = 0, tau: float = 0.0,
+             w_q_bits: np.ndarray = None):
+        wq = f64((self.inp.w_q if w_q_bits is None else w_q_bits)[self.h])
+        return O.decode_step_bh(self.q_group(q_bits), self.k, self.v, wq, self.kcomp(length), length, self.blk,
+                                self.inp.cfg.rope_base, mode, k_blocks=k_blocks, tau=tau)
+
+    def attention(self, length: int, q_bits: np.ndarray, blocks: Sequence[int]):
+        d = self.inp.cfg.head_dim
+        return O.sparse_decode(self.q_group(q_bits), self.k, self.v, list(blocks), length, self.blk, 1 / math.sqrt(d))
+
+
+def check_logits(gpu: np.ndarray, ref: np.ndarray, what: str = ""):
+    ref = np.asarray(ref, np.float64)
+    gpu = np.asarray(gpu, np.float64)
+    assert gpu.shape == ref.shape, what
+    if ref.size == 0:
+        return 0.0
+    rms = math.sqrt(float(np.mean(ref ** 2)))
+    bound = LOGIT_RTOL * np.maximum(np.abs(ref), rms)
+    err = np.abs(gpu - ref)
+    bad = err > bound
+    assert not bad.any(), f"{what}: {bad.sum()} logits off, worst {float(err.max()):.3e} (rms {rms:.3e})"
+    return float((err / np.maximum(np.abs(ref), rms)).max())
+
+
+def check_attention(gpu_o: np.ndarray, ref_o: np.ndarray, what: str = ""):
+    gpu_o = np.asarray(gpu_o, np.float64)
+    ref_o = np.asarray(ref_o, np.float64)
+    assert np.all(np.isfinite(gpu_o)), f"{what}: non-finite output"
+    max_abs = float(np.abs(gpu_o - ref_o).max()) if ref_o.size else 0.0
+    denom = float(np.linalg.norm(ref_o))
+    rel = float(np.linalg.norm(gpu_o - ref_o) / denom) if denom > 0 else float(np.linalg.norm(gpu_o))
+    assert max_abs <= OUT_MAX_ABS, f"{what}: max-abs {max_abs:.3e} > {OUT_MAX_ABS}"
+    assert rel <= OUT_REL_L2, f"{what}: rel-L2 {rel:.3e} > {OUT_REL_L2}"
+    return max_abs, rel
+
+
+def check_lse(gpu_l: np.ndarray, ref_l: np.ndarray, what: str = ""):
+    gpu_l = np.asarray(gpu_l, np.float64)
+    ref_l = np.asarray(ref_l, np.float64)
+    fin = np.isfinite(ref_l)
+    assert np.array_equal(fin, np.isfinite(gpu_l)), f"{what}: lse finiteness differs"
+    if fin.any():
+        err = float(np.abs(gpu_l[fin] - ref_l[fin]).max())
+        assert err <= LSE_ABS, f"{what}: lse err {err:.3e}"
+
+
+def bf16_ulp_diff(a_bits: np.ndarray, b_bits: np.ndarray) -> np.ndarray:
+    """Distance in bf16 ulps between two arrays of bf16 bit patterns (same sign assumed near zero)."""
+    def ordered(x):
+        x = x.astype(np.int32)
+        return np.where(x & 0x8000, -(x & 0x7FFF), x)
+    return np.abs(ordered(a_bits) - ordered(b_bits))
+
+
+def gpu_list(idx_row: np.ndarray, cnt: int) -> List[int]:
+    return [int(x) for x in idx_row[:cnt]]
+
+
+def check_selection(gpu: List[int], ref: List[int], scores: np.ndarray = None, tau: float = None, what=""):
+    """Exact match; in threshold mode a block may differ only when its score is within 1e-6 of tau."""
+    if gpu == ref:
+        return 0
+    assert scores is not None and tau is not None, f"{what}: selection differs: gpu {gpu} vs oracle {ref}"
+    diff = set(gpu) ^ set(ref)
+    for n in diff:
+        assert n < len(scores) and abs(scores[n] - tau) <= THRESH_REL * tau, \
+            f"{what}: block {n} differs (score {scores[n] if n < len(scores) else None}, tau {tau})"
+    return len(diff)
