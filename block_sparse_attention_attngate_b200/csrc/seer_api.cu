@@ -259,6 +259,11 @@ size_t ws_layout(const seer_dims_t* d, int32_t ns, size_t* off_lse, size_t* off_
 
 }  // namespace
 
+int seer::set_last_error(int status, const char* msg) {
+  g_err = msg ? msg : "";
+  return status;
+}
+
 extern "C" {
 
 const char* seer_last_error(void) { return g_err.c_str(); }

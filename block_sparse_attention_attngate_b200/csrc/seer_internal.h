@@ -112,4 +112,7 @@ cudaError_t launch_sparse_decode(const CUtensorMap& tk, const CUtensorMap& tv, c
                                  int D, int BLK, cudaStream_t s);
 int decode_ctas_per_sm(int D, int BLK);
 
+// Record `msg` as the text seer_last_error() returns on this thread; returns `status`.
+int set_last_error(int status, const char* msg);
+
 }  // namespace seer

@@ -27,7 +27,8 @@ DEVERR_BLOCK_INDEX, DEVERR_PAGE_INDEX, DEVERR_COUNT, DEVERR_TIMEOUT = 1, 2, 4, 8
 
 EXPORTED = (
     "seer_kcomp_update", "seer_gate_score", "seer_select_blocks", "seer_sparse_decode_auto_split",
-    "seer_sparse_decode_workspace_bytes", "seer_sparse_decode", "seer_last_error", "seer_version",
+    "seer_sparse_decode_workspace_bytes", "seer_sparse_decode", "seer_sparse_decode_noalloc", "seer_last_error",
+    "seer_version",
 )
 
 
@@ -63,6 +64,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "seer_sparse_decode_auto_split": (I32, [DP, I32]),
         "seer_sparse_decode_workspace_bytes": (SZ, [DP, I32, I32]),
         "seer_sparse_decode": (I32, [DP, P, KP, KP, P, P, P, I32, I32, P, SZ, P, P, P, P]),
+        "seer_sparse_decode_noalloc": (I32, [DP, P, KP, KP, P, P, P, I32, I32, P, P, P, P]),
         "seer_last_error": (ctypes.c_char_p, []),
         "seer_version": (ctypes.c_char_p, []),
     }
@@ -225,6 +227,25 @@ def sparse_decode(shape: Shape, q: torch.Tensor, k: KVCache, v: KVCache, block_i
                                    _ptr(block_idx), _ptr(block_cnt), _ptr(seqlens), block_idx.shape[-1],
                                    int(num_split), _ptr(workspace), ws_bytes, _ptr(out), _ptr(lse), _ptr(err),
                                    _stream(stream)))
+
+
+def sparse_decode_noalloc(shape: Shape, q: torch.Tensor, k: KVCache, v: KVCache, block_idx: torch.Tensor,
+                          block_cnt: torch.Tensor, seqlens: torch.Tensor, out: torch.Tensor, num_split: int = 0,
+                          lse: Optional[torch.Tensor] = None, err: Optional[torch.Tensor] = None, stream=None):
+    """sparse_decode without a workspace argument, for callers that cannot allocate device memory.
+
+    The library's fixed 8 MiB scratch array takes the workspace's place: calls on one device
+    must not overlap on the GPU, and the first call on a device must come before any capture.
+    """
+    _need(q, torch.bfloat16, "q")
+    _need(block_idx, torch.int32, "block_idx")
+    _need(block_cnt, torch.int32, "block_cnt")
+    _need(seqlens, torch.int32, "seqlens")
+    _need(out, torch.bfloat16, "out")
+    dims = shape.c()
+    _check(_lib.seer_sparse_decode_noalloc(ctypes.byref(dims), _ptr(q), ctypes.byref(k.desc), ctypes.byref(v.desc),
+                                           _ptr(block_idx), _ptr(block_cnt), _ptr(seqlens), block_idx.shape[-1],
+                                           int(num_split), _ptr(out), _ptr(lse), _ptr(err), _stream(stream)))
 
 
 class DecodeStep:

@@ -208,6 +208,30 @@ seer_status seer_sparse_decode(const seer_dims_t* dims, const void* q, const see
                                size_t workspace_bytes, void* out, float* lse_out,
                                int32_t* err_word, void* stream);
 
+/*
+ * seer_sparse_decode_noalloc -- seer_sparse_decode for callers that cannot allocate.
+ *
+ * The pages have no counterpart to this call; it is an interface convenience.  Callers that
+ * must not call cudaMalloc -- an engine that reserved all free device memory for its KV pool
+ * before serving, a plugin whose host owns every allocation, a hot loop that cannot afford
+ * cudaMalloc's implicit device synchronisation -- pass only inputs and outputs here.  The
+ * split partials and arrival counters live in a fixed 8 MiB scratch array inside the library
+ * image (held by every GPU that loads the library until the process exits).
+ *
+ * Arguments and results are those of seer_sparse_decode without workspace/workspace_bytes.
+ * Returns SEER_ERR_CAPACITY when the chosen split count needs more scratch than 8 MiB
+ * (seer_sparse_decode_workspace_bytes > 8388608); nothing is enqueued then.
+ * The first call on a device looks up the scratch's device address (cudaGetSymbolAddress) with
+ * that device current; make that first call before any stream capture.  Each call clears the
+ * arrival counters with an async memset on `stream`.  All calls on a device share the scratch:
+ * calls that overlap on the GPU race and must be serialised by the caller.  Allocates nothing.
+ */
+seer_status seer_sparse_decode_noalloc(const seer_dims_t* dims, const void* q, const seer_kv_t* k,
+                                       const seer_kv_t* v, const int32_t* block_idx,
+                                       const int32_t* block_cnt, const int32_t* seqlens,
+                                       int32_t capacity, int32_t num_split, void* out,
+                                       float* lse_out, int32_t* err_word, void* stream);
+
 /* Thread-local text describing the last non-OK status returned on this thread. */
 const char* seer_last_error(void);
 
