@@ -8,8 +8,9 @@ d_gate=128, context 32768, block 64, token budget 4096 (64 of 512 blocks),
 
 A step is one pass of the whole hot path on one batch: K Compression Cache
 update (a no-op check unless a block fills) -> AttnGate logits -> top-k
-selection -> block-sparse flash decode with the fused split combine.  Each
-step is a CUDA-graph replay of those five kernel launches.  Inputs rotate
+selection (these three fused in one launch, seer_decode_plan) -> block-sparse
+flash decode with the split combine.  Each step is a CUDA-graph replay of
+those two kernel launches.  Inputs rotate
 over replicas whose combined selected K/V (3 x 134 MB) exceeds the 126 MB
 L2, so no step reads the previous step's blocks from L2.
 
@@ -54,6 +55,8 @@ def parse():
     ap.add_argument("--budget", type=int, default=0, help="override the token budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample", type=int, default=16, help="(b, h) pairs in the oracle sample")
+    ap.add_argument("--only", default="all", choices=["all", "decode"],
+                    help="decode: run just the sparse-decode launches (a small target for profilers)")
     return ap.parse_args()
 
 
@@ -246,7 +249,7 @@ def run_seer(args):
         v = v0 if r == 0 else v0.clone()
         q = q0.clone()
         kc = torch.zeros(B, Hkv, NB, dg, dtype=torch.bfloat16, device=dev)
-        valid = torch.zeros(B, dtype=torch.int32, device=dev)
+        valid = torch.zeros(B, Hkv, dtype=torch.int32, device=dev)
         step = S.DecodeStep(shape, S.KVCache.contiguous(k), S.KVCache.contiguous(v), w_q, w_k, kc, valid,
                             mode=S.SELECT_TOPK, token_budget=cfg.budget, num_split=args.num_split)
         S.kcomp_update(shape, S.KVCache.contiguous(k), seqlens, valid, w_k, kc)   # prefill build (untimed)
@@ -256,6 +259,18 @@ def run_seer(args):
 
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
+    if args.only == "decode":
+        with torch.cuda.stream(stream):
+            for rp in reps:
+                rp["step"].run(rp["q"], seqlens, stream=stream)     # builds the block lists
+            for i in range(args.warmup + args.steps):
+                st = reps[i % R]["step"]
+                S.sparse_decode(shape, reps[i % R]["q"], st.k, st.v, st.block_idx, st.block_cnt, seqlens, st.out,
+                                st.workspace, st.num_split, st.lse, st.err, stream=stream)
+        stream.synchronize()
+        if rank == 0:
+            print(json.dumps({"only": "decode", "launches": args.warmup + args.steps, "replicas": R}), flush=True)
+        return 0
     # warm once eagerly (first-call set-up happens outside capture), then capture one graph per replica
     with torch.cuda.stream(stream):
         for rp in reps:
@@ -328,13 +343,20 @@ def run_seer(args):
         st = reps[i % R]["step"]
         S.kcomp_update(shape, st.k_nope, seqlens, st.valid_blocks, w_k, st.kcomp, stream=stream)
 
+    def run_plan(i):
+        st = reps[i % R]["step"]
+        S.decode_plan(shape, seqlens, st.kcomp, reps[i % R]["q"], w_q, S.SELECT_TOPK, st.block_idx, st.block_cnt,
+                      cfg.budget, 0.0, k_nope=st.k_nope, valid_blocks=st.valid_blocks, w_k=w_k, logits=st.logits,
+                      stream=stream)
+
     decode_us = part(run_decode)
+    plan_us = part(run_plan)
     gate_us = part(run_gate)
     select_us = part(run_select)
     kcomp_noop_us = part(run_kcomp_noop)
 
     # kcomp fill step: one new block per (b, h) (the step where a block fills)
-    fill_valid = torch.full((args.warmup + args.steps + 1, B), NB - 1, dtype=torch.int32, device=dev)
+    fill_valid = torch.full((args.warmup + args.steps + 1, B, Hkv), NB - 1, dtype=torch.int32, device=dev)
     fill_row = [0]
 
     def run_kcomp_fill(i):
@@ -348,7 +370,7 @@ def run_seer(args):
     # ---------------- dense path: every block of every (b, h), same kernel
     dense_idx = torch.arange(NB, dtype=torch.int32, device=dev).expand(B, Hkv, NB).contiguous()
     dense_cnt = torch.full((B, Hkv), NB, dtype=torch.int32, device=dev)
-    dense_ns = S.sparse_decode_auto_split(shape, NB)
+    dense_ns = args.num_split
     dense_ws = S.alloc_workspace(shape, NB, dense_ns, dev)
     dense_out = torch.empty(B, Hq, d, dtype=torch.bfloat16, device=dev)
 
@@ -407,8 +429,9 @@ def run_seer(args):
                    "sparsity": 1.0 - float(cnt_h.mean()) / NB, "num_split": st0.num_split,
                    "l2": f"inputs rotate over {R} replicas ({R * nbytes['selected_kv'] / 1e6:.0f} MB selected K/V "
                          f"per rotation > 126 MB L2)", "parallelism": f"dp{world} (independent batches)"},
-        "parts_us": {"kcomp_update_noop": kcomp_noop_us, "kcomp_update_fill": kcomp_fill_us, "gate_score": gate_us,
-                     "select_blocks": select_us, "sparse_decode": decode_us},
+        "parts_us": {"decode_plan": plan_us, "sparse_decode": decode_us,
+                     "unfused": {"kcomp_update_noop": kcomp_noop_us, "kcomp_update_fill": kcomp_fill_us,
+                                 "gate_score": gate_us, "select_blocks": select_us}},
         "dense_path_us": dense_us, "speedup_vs_dense": dense_us / decode_us,
         "bytes": {"decode_algorithmic": nbytes["decode"], "step_algorithmic": nbytes["step"]},
         "step_gbs": step_gbs,

@@ -1,0 +1,105 @@
+// The per-step planning half of the decode in one launch: K Compression Cache
+// update, AttnGate logits and block selection for each (b, h), run by one
+// 4-CTA thread-block cluster per (b, h).
+//
+//   1. new full blocks of (b, h) (if any) -> cache rows      (kcomp_device.cuh)
+//   2. Q_gate shared through distributed shared memory, each CTA scores its
+//      1/4 of the cache rows, writing the logits into rank 0's row  (gate_device.cuh)
+//   3. rank 0 selects the blocks from that row: one warp with the row in
+//      registers for rows <= 1024 blocks, the whole CTA otherwise (select_device.cuh)
+// Equivalent to seer_kcomp_update + seer_gate_score + seer_select_blocks, with
+// two kernel boundaries and the logits' round trip through global memory
+// removed; the sources of each step are cited in its header.
+#include <cooperative_groups.h>
+
+#include "gate_device.cuh"
+#include "kcomp_device.cuh"
+#include "select_device.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace seer {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kCL = 4;
+
+template <int D, int DG>
+union PlanSmem {
+  KcompSmem<D, DG, kThreads> k;
+  GateSmem<D, DG, kCL> g;
+};
+
+template <int D, int BLK, int DG>
+__global__ void __cluster_dims__(kCL, 1, 1) __launch_bounds__(kThreads) plan_kernel(const PlanParams p) {
+  __shared__ PlanSmem<D, DG> sm;
+  __shared__ SelectScratch sc;
+  extern __shared__ float row[];   // [NB] logits (rank 0), then selection keys / pairs
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int h = blockIdx.y, b = blockIdx.z, bh = b * p.g.Hkv + h;
+  pdl_wait();
+  pdl_trigger();
+  const int L = max(p.g.seqlens[b], 0);
+  int nfull_k = 0;
+  if (p.update_cache) {
+    nfull_k = kcomp_nfull<BLK>(p.k, L);
+    const int v0 = max(p.k.valid[bh], 0);
+    if (nfull_k > v0) {   // the same decision in every CTA of the cluster
+      kcomp_update_share<D, BLK, DG, kThreads>(p.k, b, h, v0, nfull_k, rank, kCL, sm.k);
+      __threadfence();    // the new rows are read by the other CTAs of the cluster below
+      cluster.sync();
+    }
+  }
+  gate_cluster<D, DG, kCL, kThreads>(p.g, b, h, rank, cluster, sm.g, cluster.map_shared_rank(row, 0));
+  cluster.sync();   // rank 0's row is complete; every CTA has read the fill count
+  if (rank != 0) return;
+  const int nfull = min(L / p.s.BLK, p.s.NB);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(row + ((p.s.NB + 1) & ~1));
+  uint64_t* pairs = reinterpret_cast<uint64_t*>(keys + ((p.s.NB + 1) & ~1));
+  int32_t* out = p.s.idx + (size_t)bh * p.s.cap;
+  int total;
+  if (p.s.NB <= kWarpSelectMax && p.s.mode != 2) {
+    if (threadIdx.x >= 32) return;
+    total = select_row_warp<kWarpSelectMax / 32>(row, nfull, (L % p.s.BLK) != 0, p.s.mode, p.s.kblocks, p.s.tau, out,
+                                                 p.s.cap);
+  } else {
+    total = select_row<kThreads>(row, nfull, (L % p.s.BLK) != 0, p.s.mode, p.s.kblocks, p.s.tau, keys, pairs, sc, out,
+                                 p.s.cap);
+  }
+  if (threadIdx.x == 0) {
+    p.s.cnt[bh] = total;
+    if (p.update_cache) p.k.valid_out[bh] = nfull_k;
+  }
+}
+
+template <int D, int BLK, int DG>
+cudaError_t launch_t(const PlanParams& p, cudaStream_t s) {
+  auto kern = plan_kernel<D, BLK, DG>;
+  static std::atomic<uint64_t> attr_done{0};
+  const size_t row_bytes = (size_t)((kMaxBlocksRow + 1) & ~1) * 4;
+  cudaError_t e = ensure_smem_limit(kern, (int)(row_bytes + select_smem_bytes(kMaxBlocksRow, 2)), attr_done);
+  if (e != cudaSuccess) return e;
+  const size_t smem = (size_t)((p.s.NB + 1) & ~1) * 4 + select_smem_bytes(p.s.NB, p.s.mode);
+  dim3 grid(kCL, p.g.Hkv, p.g.B);
+  return launch_pdl(kern, grid, dim3(kThreads), smem, s, p);
+}
+
+}  // namespace
+
+cudaError_t launch_plan(const PlanParams& p, int D, int BLK, int DG, cudaStream_t s) {
+#define SEER_P(d, blk, dg) \
+  if (D == d && BLK == blk && DG == dg) return launch_t<d, blk, dg>(p, s);
+  SEER_P(64, 64, 64)
+  SEER_P(64, 64, 128)
+  SEER_P(64, 128, 64)
+  SEER_P(64, 128, 128)
+  SEER_P(128, 64, 64)
+  SEER_P(128, 64, 128)
+  SEER_P(128, 128, 64)
+  SEER_P(128, 128, 128)
+#undef SEER_P
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace seer

@@ -4,7 +4,9 @@
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <string.h>
 
+#include <algorithm>
 #include <mutex>
 #include <string>
 
@@ -223,6 +225,33 @@ seer_status tensor_map(const seer_dims_t* d, const seer_kv_t* kv, const char* na
   return SEER_OK;
 }
 
+void rope_thetas(const seer_dims_t* d, double* theta) {
+  const int half = d->gate_dim / 2;
+  for (int i = 0; i < half; ++i) theta[i] = pow((double)d->rope_base, -2.0 * i / d->gate_dim);
+}
+
+seer_status select_args(const seer_dims_t* dims, int32_t mode, int32_t token_budget, float tau, int32_t capacity,
+                        int32_t* kblocks) {
+  if (mode != SEER_SELECT_TOPK && mode != SEER_SELECT_THRESHOLD && mode != SEER_SELECT_TOPP)
+    return fail(SEER_ERR_INVALID_ARG, "unknown selection mode %d", mode);
+  if (capacity < 1) return fail(SEER_ERR_INVALID_ARG, "capacity must be >= 1");
+  *kblocks = 0;
+  if (mode == SEER_SELECT_TOPK) {
+    if (token_budget < 0) return fail(SEER_ERR_INVALID_ARG, "token_budget must be >= 0");
+    int32_t k = (int32_t)(((int64_t)token_budget + dims->block_size - 1) / dims->block_size);
+    if (k > dims->max_blocks) k = dims->max_blocks;
+    if (capacity < k + 1 && capacity < dims->max_blocks)
+      return fail(SEER_ERR_CAPACITY, "capacity %d < k+1 = %d (top-k plus the partial block)", capacity, k + 1);
+    *kblocks = k;
+  } else {
+    if (!isfinite(tau)) return fail(SEER_ERR_INVALID_ARG, "tau must be finite");
+    if (capacity < dims->max_blocks)
+      return fail(SEER_ERR_CAPACITY, "capacity %d < max_blocks %d (threshold / top-p may select every block)",
+                  capacity, dims->max_blocks);
+  }
+  return SEER_OK;
+}
+
 seer::KvPlain plain(const seer_kv_t* kv) {
   seer::KvPlain k;
   k.data = static_cast<const uint16_t*>(kv->data);
@@ -247,14 +276,24 @@ int32_t auto_split(const seer_dims_t* d, int32_t capacity, DevFacts* df) {
   return (int32_t)(ns < 1 ? 1 : ns);
 }
 
-size_t ws_layout(const seer_dims_t* d, int32_t ns, size_t* off_lse, size_t* off_o) {
+// CTAs of the balanced (num_split == 0) schedule: one per SM slot.
+int flat_grid(const seer_dims_t* d, DevFacts* df) { return df->sms * decode_occ(df, d->head_dim, d->block_size); }
+
+// Workspace: split-arrival counters [B*Hkv] int32 (zero before the first call, left zero) |
+// lse partials [slots][g] | o partials [slots][g][d].  Balanced schedule: 2 partial slots per
+// CTA (a CTA's first and last segment are the only ones that can belong to a (b, h) split
+// across CTAs).  Grid schedule: num_split slots per (b, h).
+size_t ws_layout(const seer_dims_t* d, int32_t ns, int flat_ctas, size_t* off_lse, size_t* off_o) {
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
-  const size_t cnt = up((size_t)d->batch * d->num_kv_heads * 4);
-  const size_t lse = up((size_t)d->batch * d->num_q_heads * ns * 4);
-  const size_t o = (size_t)d->batch * d->num_q_heads * ns * d->head_dim * 4;
-  *off_lse = cnt;
-  *off_o = cnt + lse;
-  return ns <= 1 ? 0 : cnt + lse + o;
+  const size_t g = (size_t)(d->num_q_heads / d->num_kv_heads);
+  const size_t bh = (size_t)d->batch * d->num_kv_heads;
+  const size_t slots = ns == 0 ? 2 * (size_t)flat_ctas : bh * ns;
+  const size_t rec = up(bh * 4);
+  const size_t lse = up(slots * g * 4);
+  const size_t o = slots * g * d->head_dim * 4;
+  *off_lse = rec;
+  *off_o = rec + lse;
+  return ns == 1 ? 0 : rec + lse + o;
 }
 
 }  // namespace
@@ -281,6 +320,7 @@ seer_status seer_kcomp_update(const seer_dims_t* dims, const seer_kv_t* k_nope, 
   DevFacts* df;
   if ((st = device_facts(&dev, &df)) != SEER_OK) return st;
   seer::KcompParams p;
+  rope_thetas(dims, p.theta);
   p.k = plain(k_nope);
   p.seqlens = seqlens;
   p.valid = valid_blocks;
@@ -311,6 +351,7 @@ seer_status seer_gate_score(const seer_dims_t* dims, const void* q_nope, const v
       (q_gate_out && !aligned16(q_gate_out)))
     return fail(SEER_ERR_INVALID_ARG, "pointer not 16-byte aligned");
   seer::GateParams p;
+  rope_thetas(dims, p.theta);
   p.q = static_cast<const uint16_t*>(q_nope);
   p.w_q = static_cast<const uint16_t*>(w_q);
   p.kcomp = static_cast<const uint16_t*>(kcomp);
@@ -335,22 +376,8 @@ seer_status seer_select_blocks(const seer_dims_t* dims, const float* logits, con
   seer_status st = check_dims(dims);
   if (st != SEER_OK) return st;
   if (!logits || !seqlens || !block_idx || !block_cnt) return fail(SEER_ERR_INVALID_ARG, "NULL pointer argument");
-  if (mode != SEER_SELECT_TOPK && mode != SEER_SELECT_THRESHOLD && mode != SEER_SELECT_TOPP)
-    return fail(SEER_ERR_INVALID_ARG, "unknown selection mode %d", mode);
-  if (capacity < 1) return fail(SEER_ERR_INVALID_ARG, "capacity must be >= 1");
   int32_t kblocks = 0;
-  if (mode == SEER_SELECT_TOPK) {
-    if (token_budget < 0) return fail(SEER_ERR_INVALID_ARG, "token_budget must be >= 0");
-    kblocks = (int32_t)(((int64_t)token_budget + dims->block_size - 1) / dims->block_size);
-    if (kblocks > dims->max_blocks) kblocks = dims->max_blocks;
-    if (capacity < kblocks + 1 && capacity < dims->max_blocks)
-      return fail(SEER_ERR_CAPACITY, "capacity %d < k+1 = %d (top-k plus the partial block)", capacity, kblocks + 1);
-  } else {
-    if (!isfinite(tau)) return fail(SEER_ERR_INVALID_ARG, "tau must be finite");
-    if (capacity < dims->max_blocks)
-      return fail(SEER_ERR_CAPACITY, "capacity %d < max_blocks %d (threshold / top-p may select every block)",
-                  capacity, dims->max_blocks);
-  }
+  if ((st = select_args(dims, mode, token_budget, tau, capacity, &kblocks)) != SEER_OK) return st;
   seer::SelectParams p;
   p.logits = logits;
   p.seqlens = seqlens;
@@ -369,6 +396,71 @@ seer_status seer_select_blocks(const seer_dims_t* dims, const float* logits, con
   return SEER_OK;
 }
 
+seer_status seer_decode_plan(const seer_dims_t* dims, const seer_kv_t* k_nope, const int32_t* seqlens,
+                             int32_t* valid_blocks, const void* w_k, void* kcomp, const void* q_nope,
+                             const void* w_q, float* logits_out, float* q_gate_out, int32_t mode,
+                             int32_t token_budget, float tau, int32_t* block_idx, int32_t* block_cnt,
+                             int32_t capacity, void* stream) {
+  seer_status st = check_dims(dims);
+  if (st != SEER_OK) return st;
+  if (!seqlens || !kcomp || !q_nope || !w_q || !block_idx || !block_cnt)
+    return fail(SEER_ERR_INVALID_ARG, "NULL pointer argument");
+  if (!aligned16(kcomp) || !aligned16(q_nope) || !aligned16(w_q) || (logits_out && !aligned16(logits_out)) ||
+      (q_gate_out && !aligned16(q_gate_out)))
+    return fail(SEER_ERR_INVALID_ARG, "pointer not 16-byte aligned");
+  const bool update = valid_blocks != nullptr;
+  if (update) {
+    if ((st = check_kv(dims, k_nope, "k_nope")) != SEER_OK) return st;
+    if (!w_k || !aligned16(w_k)) return fail(SEER_ERR_INVALID_ARG, "w_k is NULL or not 16-byte aligned");
+  }
+  int32_t kblocks = 0;
+  if ((st = select_args(dims, mode, token_budget, tau, capacity, &kblocks)) != SEER_OK) return st;
+  seer::PlanParams p;
+  p.update_cache = update;
+  rope_thetas(dims, p.k.theta);
+  if (update) p.k.k = plain(k_nope);
+  else memset(&p.k.k, 0, sizeof(p.k.k));
+  p.k.seqlens = seqlens;
+  p.k.valid = valid_blocks;
+  p.k.valid_out = valid_blocks;
+  p.k.w_k = static_cast<const uint16_t*>(w_k);
+  p.k.kcomp = static_cast<uint16_t*>(kcomp);
+  p.k.B = dims->batch;
+  p.k.Hkv = dims->num_kv_heads;
+  p.k.NB = dims->max_blocks;
+  p.k.rope_base = dims->rope_base;
+  p.k.err = nullptr;
+  rope_thetas(dims, p.g.theta);
+  p.g.q = static_cast<const uint16_t*>(q_nope);
+  p.g.w_q = static_cast<const uint16_t*>(w_q);
+  p.g.kcomp = static_cast<const uint16_t*>(kcomp);
+  p.g.seqlens = seqlens;
+  p.g.logits = logits_out;
+  p.g.q_gate = q_gate_out;
+  p.g.B = dims->batch;
+  p.g.Hq = dims->num_q_heads;
+  p.g.Hkv = dims->num_kv_heads;
+  p.g.g = dims->num_q_heads / dims->num_kv_heads;
+  p.g.NB = dims->max_blocks;
+  p.g.BLK = dims->block_size;
+  p.g.rope_base = dims->rope_base;
+  p.s.logits = nullptr;
+  p.s.seqlens = seqlens;
+  p.s.idx = block_idx;
+  p.s.cnt = block_cnt;
+  p.s.B = dims->batch;
+  p.s.Hkv = dims->num_kv_heads;
+  p.s.NB = dims->max_blocks;
+  p.s.BLK = dims->block_size;
+  p.s.cap = capacity;
+  p.s.mode = mode;
+  p.s.kblocks = kblocks;
+  p.s.tau = (double)tau;
+  cudaError_t e = seer::launch_plan(p, dims->head_dim, dims->block_size, dims->gate_dim, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "decode_plan launch");
+  return SEER_OK;
+}
+
 int32_t seer_sparse_decode_auto_split(const seer_dims_t* dims, int32_t capacity) {
   if (check_dims(dims) != SEER_OK || capacity < 1) return 1;
   int dev;
@@ -378,11 +470,17 @@ int32_t seer_sparse_decode_auto_split(const seer_dims_t* dims, int32_t capacity)
 }
 
 size_t seer_sparse_decode_workspace_bytes(const seer_dims_t* dims, int32_t capacity, int32_t num_split) {
-  if (check_dims(dims) != SEER_OK || capacity < 1) return 0;
-  int32_t ns = num_split;
-  if (ns <= 0) ns = seer_sparse_decode_auto_split(dims, capacity);
+  if (check_dims(dims) != SEER_OK || capacity < 1 || num_split < 0) return 0;
+  const int32_t ns = num_split > capacity ? capacity : num_split;
+  int ctas = 0;
+  if (ns == 0) {
+    int dev;
+    DevFacts* df;
+    if (device_facts(&dev, &df) != SEER_OK) return 0;
+    ctas = flat_grid(dims, df);
+  }
   size_t a, b;
-  return ws_layout(dims, ns, &a, &b);
+  return ws_layout(dims, ns, ctas, &a, &b);
 }
 
 seer_status seer_sparse_decode(const seer_dims_t* dims, const void* q, const seer_kv_t* k, const seer_kv_t* v,
@@ -400,9 +498,14 @@ seer_status seer_sparse_decode(const seer_dims_t* dims, const void* q, const see
   int dev;
   DevFacts* df;
   if ((st = device_facts(&dev, &df)) != SEER_OK) return st;
-  const int32_t ns = num_split == 0 ? auto_split(dims, capacity, df) : (num_split > capacity ? capacity : num_split);
+  if (dims->batch > seer::kMaxDecodeB) return fail(SEER_ERR_UNSUPPORTED, "batch %d > %d", dims->batch, seer::kMaxDecodeB);
+  int32_t ns = num_split > capacity ? capacity : num_split;
+  if (ns == 0 && dims->batch * dims->num_kv_heads > seer::kMaxDecodeBH)
+    return fail(SEER_ERR_UNSUPPORTED, "balanced schedule needs batch*num_kv_heads <= %d; pass num_split >= 1",
+                seer::kMaxDecodeBH);
+  const int ctas = ns == 0 ? flat_grid(dims, df) : 0;
   size_t off_lse, off_o;
-  const size_t need = ws_layout(dims, ns, &off_lse, &off_o);
+  const size_t need = ws_layout(dims, ns, ctas, &off_lse, &off_o);
   if (need > 0) {
     if (!workspace) return fail(SEER_ERR_INVALID_ARG, "workspace is NULL (num_split %d needs %zu bytes)", ns, need);
     if (workspace_bytes < need)
@@ -430,8 +533,9 @@ seer_status seer_sparse_decode(const seer_dims_t* dims, const void* q, const see
   p.Hkv = dims->num_kv_heads;
   p.g = dims->num_q_heads / dims->num_kv_heads;
   p.cap = capacity;
+  p.flat = ns == 0;
   p.ns = ns;
-  p.per_split = (capacity + ns - 1) / ns;
+  p.per_split = ns ? (capacity + ns - 1) / ns : capacity;
   const float scale = dims->softmax_scale > 0.f ? dims->softmax_scale : 1.0f / sqrtf((float)dims->head_dim);
   p.scale_log2 = scale * 1.4426950408889634f;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -441,7 +545,7 @@ seer_status seer_sparse_decode(const seer_dims_t* dims, const void* q, const see
   p.out = static_cast<uint16_t*>(out);
   p.lse_out = lse_out;
   p.err = err_word;
-  cudaError_t e = seer::launch_sparse_decode(tk, tv, p, dims->head_dim, dims->block_size,
+  cudaError_t e = seer::launch_sparse_decode(tk, tv, p, dims->head_dim, dims->block_size, ctas,
                                              static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "sparse_decode launch");
   return SEER_OK;

@@ -22,6 +22,14 @@ __device__ __forceinline__ void report(int32_t* err, int32_t bit) {
   if (err) atomicOr(err, bit);
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// Kernels are launched with programmatic stream serialization: the next kernel
+// in the stream may start while this one runs.  Every kernel waits for its
+// predecessors to complete (and their writes to be visible) before it reads
+// any global input, then lets its own successor launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -66,10 +74,48 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
+// Bounded barrier among the `count` warps that arrive on `bar` (one elected
+// lane per warp).  `phase` counts completed uses; returns false on timeout.
+__device__ __forceinline__ bool warps_sync(uint64_t* bar, uint32_t& phase) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+  const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, phase & 1));
+  ++phase;
+  return ok;
+}
+
+// Atomic add with acquire-release semantics at GPU scope (publishes this thread's
+// and, cumulatively, everything it has observed; acquires everything published before).
+__device__ __forceinline__ int atomic_add_acq_rel_gpu(int* addr, int v) {
+  int old;
+  asm volatile("atom.add.acq_rel.gpu.s32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v) : "memory");
+  return old;
+}
+
+// ---------------------------------------------------------------- RoPE angles
+// cos / sin of a large angle (position * theta, up to ~1e5 rad): reduce modulo
+// 2*pi in fp64 (2*pi split in two doubles, so the reduction error stays near
+// 1e-16 * angle / (2*pi)), then evaluate in fp32 on |r| <= pi.
+__device__ __forceinline__ void rope_cos_sin(double angle, float& c, float& s) {
+  constexpr double kTwoPiHi = 6.283185307179586;
+  constexpr double kTwoPiLo = 2.4492935982947064e-16;
+  const double k = rint(angle * (1.0 / kTwoPiHi));
+  const double r = fma(-k, kTwoPiLo, fma(-k, kTwoPiHi, angle));
+  sincosf((float)r, &s, &c);
+}
+
 // ---------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// Contiguous bulk copy global -> shared (16-byte aligned, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
 }
 
 // 4-D tiled bulk tensor load global -> shared, completion counted on `bar`.

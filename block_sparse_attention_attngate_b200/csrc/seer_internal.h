@@ -10,6 +10,24 @@
 
 namespace seer {
 
+// Launch `kern` on `s` with programmatic stream serialization (see pdl_wait /
+// pdl_trigger in seer_device.cuh).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
+
 // Raise a kernel's dynamic shared-memory limit once per device (a host-side
 // attribute call, kept out of CUDA-graph capture after the first use).
 template <typename Kernel>
@@ -27,6 +45,8 @@ cudaError_t ensure_smem_limit(Kernel kern, int bytes, std::atomic<uint64_t>& don
 
 constexpr int kMaxGroup = 8;        // query heads per KV head
 constexpr int kMaxBlocksRow = 8192; // max_blocks limit (selection keeps a row in shared memory)
+constexpr int kMaxDecodeB = 4096;   // decode keeps the sequence lengths in shared memory
+constexpr int kMaxDecodeBH = 4096;  // balanced decode keeps the list-length prefix in shared memory
 
 // Where a K/V tile lives, for kernels that read it with plain loads.
 struct KvPlain {
@@ -40,7 +60,10 @@ struct KvPlain {
 };
 
 // ---------------------------------------------------------------- kcomp update
+constexpr int kMaxHalfGate = 64;    // d_gate / 2 rotation frequencies
+
 struct KcompParams {
+  double theta[kMaxHalfGate];   // base^(-2i/d_gate), computed on the host in fp64
   KvPlain k;
   const int32_t* seqlens;
   const int32_t* valid;
@@ -56,6 +79,7 @@ cudaError_t launch_kcomp_update(const KcompParams& p, int D, int BLK, int DG, in
 
 // ---------------------------------------------------------------- gate score
 struct GateParams {
+  double theta[kMaxHalfGate];   // base^(-2i/d_gate), computed on the host in fp64
   const uint16_t* q;       // [B, Hq, D]
   const uint16_t* w_q;     // [Hkv, DG, g*D]
   const uint16_t* kcomp;   // [B, Hkv, NB, DG]
@@ -80,6 +104,15 @@ struct SelectParams {
 };
 cudaError_t launch_select(const SelectParams& p, cudaStream_t s);
 
+// ---------------------------------------------------------------- fused plan (cache update + gate + select)
+struct PlanParams {
+  KcompParams k;
+  GateParams g;
+  SelectParams s;
+  int32_t update_cache;   // run the cache update first
+};
+cudaError_t launch_plan(const PlanParams& p, int D, int BLK, int DG, cudaStream_t s);
+
 // ---------------------------------------------------------------- sparse decode
 struct DecodeParams {
   const uint16_t* q;        // [B, Hq, D]
@@ -93,23 +126,18 @@ struct DecodeParams {
   int32_t k_paged, v_paged;
   int32_t k_perm[3], v_perm[3];   // TMA dim (1..3) that holds token / head / batch-or-page
   int32_t B, Hq, Hkv, g;
+  int32_t flat;             // 1: balanced ranges over a persistent grid; 0: (split, kv head, batch) grid
   int32_t cap, ns, per_split;
   float scale_log2;         // softmax scale * log2(e)
   float* o_part;            // [B, Hq, ns, D]
   float* lse_part;          // [B, Hq, ns]
-  int32_t* counters;        // [B, Hkv]
+  int32_t* counters;        // [B, Hkv] split-arrival counters (zero between calls)
   uint16_t* out;            // [B, Hq, D] bf16
   float* lse_out;           // [B, Hq] or null
   int32_t* err;
 };
-struct DecodeConfig {
-  int stages;
-  int warps;       // consumer warps
-  size_t smem;
-};
-DecodeConfig decode_config(int D, int BLK);
 cudaError_t launch_sparse_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
-                                 int D, int BLK, cudaStream_t s);
+                                 int D, int BLK, int grid_flat, cudaStream_t s);
 int decode_ctas_per_sm(int D, int BLK);
 
 // Record `msg` as the text seer_last_error() returns on this thread; returns `status`.

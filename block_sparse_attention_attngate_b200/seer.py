@@ -17,7 +17,8 @@ from typing import Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libseer.so")
+# SEER_LIBRARY selects another build of the library (e.g. a variant with different tile choices)
+LIB_PATH = os.environ.get("SEER_LIBRARY") or os.path.join(_HERE, "libseer.so")
 
 SEER_OK, SEER_ERR_INVALID_ARG, SEER_ERR_UNSUPPORTED, SEER_ERR_CAPACITY, SEER_ERR_CUDA = range(5)
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CAPACITY", 4: "CUDA"}
@@ -26,7 +27,7 @@ SELECT_TOPK, SELECT_THRESHOLD, SELECT_TOPP = 0, 1, 2
 DEVERR_BLOCK_INDEX, DEVERR_PAGE_INDEX, DEVERR_COUNT, DEVERR_TIMEOUT = 1, 2, 4, 8
 
 EXPORTED = (
-    "seer_kcomp_update", "seer_gate_score", "seer_select_blocks", "seer_sparse_decode_auto_split",
+    "seer_kcomp_update", "seer_gate_score", "seer_select_blocks", "seer_decode_plan", "seer_sparse_decode_auto_split",
     "seer_sparse_decode_workspace_bytes", "seer_sparse_decode", "seer_sparse_decode_noalloc", "seer_last_error",
     "seer_version",
 )
@@ -61,6 +62,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "seer_kcomp_update": (I32, [DP, KP, P, P, P, P, P]),
         "seer_gate_score": (I32, [DP, P, P, P, P, P, P, P]),
         "seer_select_blocks": (I32, [DP, P, P, I32, I32, F32, P, P, I32, P]),
+        "seer_decode_plan": (I32, [DP, KP, P, P, P, P, P, P, P, P, I32, I32, F32, P, P, I32, P]),
         "seer_sparse_decode_auto_split": (I32, [DP, I32]),
         "seer_sparse_decode_workspace_bytes": (SZ, [DP, I32, I32]),
         "seer_sparse_decode": (I32, [DP, P, KP, KP, P, P, P, I32, I32, P, SZ, P, P, P, P]),
@@ -192,6 +194,34 @@ def select_blocks(shape: Shape, logits: torch.Tensor, seqlens: torch.Tensor, mod
                                    _stream(stream)))
 
 
+def decode_plan(shape: Shape, seqlens: torch.Tensor, kcomp: torch.Tensor, q_nope: torch.Tensor, w_q: torch.Tensor,
+                mode: int, block_idx: torch.Tensor, block_cnt: torch.Tensor, token_budget: int = 0, tau: float = 0.0,
+                k_nope: Optional[KVCache] = None, valid_blocks: Optional[torch.Tensor] = None,
+                w_k: Optional[torch.Tensor] = None, logits: Optional[torch.Tensor] = None,
+                q_gate: Optional[torch.Tensor] = None, stream=None):
+    """kcomp_update (when valid_blocks is given) + gate_score + select_blocks in one launch."""
+    _need(seqlens, torch.int32, "seqlens")
+    _need(kcomp, torch.bfloat16, "kcomp")
+    _need(q_nope, torch.bfloat16, "q_nope")
+    _need(w_q, torch.bfloat16, "w_q")
+    _need(block_idx, torch.int32, "block_idx")
+    _need(block_cnt, torch.int32, "block_cnt")
+    if valid_blocks is not None:
+        _need(valid_blocks, torch.int32, "valid_blocks")
+        _need(w_k, torch.bfloat16, "w_k")
+        if k_nope is None:
+            raise ValueError("k_nope is required with valid_blocks")
+    if logits is not None:
+        _need(logits, torch.float32, "logits")
+    if q_gate is not None:
+        _need(q_gate, torch.float32, "q_gate")
+    dims = shape.c()
+    kv = ctypes.byref(k_nope.desc) if k_nope is not None else None
+    _check(_lib.seer_decode_plan(ctypes.byref(dims), kv, _ptr(seqlens), _ptr(valid_blocks), _ptr(w_k), _ptr(kcomp),
+                                 _ptr(q_nope), _ptr(w_q), _ptr(logits), _ptr(q_gate), int(mode), int(token_budget),
+                                 float(tau), _ptr(block_idx), _ptr(block_cnt), block_idx.shape[-1], _stream(stream)))
+
+
 def sparse_decode_auto_split(shape: Shape, capacity: int) -> int:
     dims = shape.c()
     return int(_lib.seer_sparse_decode_auto_split(ctypes.byref(dims), int(capacity)))
@@ -274,20 +304,29 @@ class DecodeStep:
         self.logits = torch.empty(B, Hkv, shape.max_blocks, dtype=torch.float32, device=dev)
         self.block_idx = torch.empty(B, Hkv, capacity, dtype=torch.int32, device=dev)
         self.block_cnt = torch.empty(B, Hkv, dtype=torch.int32, device=dev)
-        self.num_split = num_split if num_split > 0 else sparse_decode_auto_split(shape, capacity)
+        self.num_split = num_split    # 0 = the balanced schedule
         self.workspace = alloc_workspace(shape, capacity, self.num_split, dev)
         self.out = torch.empty(B, Hq, shape.head_dim, dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
 
-    def run(self, q: torch.Tensor, seqlens: torch.Tensor, q_nope: Optional[torch.Tensor] = None, stream=None):
+    def run(self, q: torch.Tensor, seqlens: torch.Tensor, q_nope: Optional[torch.Tensor] = None, stream=None,
+            fused: bool = True):
+        """One decode step.  fused=True plans with seer_decode_plan (one launch); fused=False makes
+        the three separate calls (kcomp_update, gate_score, select_blocks) instead."""
         s = self.shape
-        kcomp_update(s, self.k_nope, seqlens, self.valid_blocks, self.w_k, self.kcomp, stream)
-        gate_score(s, q if q_nope is None else q_nope, self.w_q, self.kcomp, seqlens, self.logits, None, stream)
-        select_blocks(s, self.logits, seqlens, self.mode, self.block_idx, self.block_cnt, self.token_budget,
-                      self.tau, stream)
+        qn = q if q_nope is None else q_nope
+        if fused:
+            decode_plan(s, seqlens, self.kcomp, qn, self.w_q, self.mode, self.block_idx, self.block_cnt,
+                        self.token_budget, self.tau, k_nope=self.k_nope, valid_blocks=self.valid_blocks, w_k=self.w_k,
+                        logits=self.logits, stream=stream)
+        else:
+            kcomp_update(s, self.k_nope, seqlens, self.valid_blocks, self.w_k, self.kcomp, stream)
+            gate_score(s, qn, self.w_q, self.kcomp, seqlens, self.logits, None, stream)
+            select_blocks(s, self.logits, seqlens, self.mode, self.block_idx, self.block_cnt, self.token_budget,
+                          self.tau, stream)
         sparse_decode(s, q, self.k, self.v, self.block_idx, self.block_cnt, seqlens, self.out, self.workspace,
                       self.num_split, self.lse, self.err, stream)
         return self.out
 
-    KERNELS_PER_STEP = 5   # kcomp update + commit, gate, select, decode
+    KERNELS_PER_STEP = 2   # plan, decode

@@ -13,6 +13,8 @@
  *
  * One decode step of one attention layer is
  *     seer_kcomp_update -> seer_gate_score -> seer_select_blocks -> seer_sparse_decode
+ * or, with the first three fused into one launch,
+ *     seer_decode_plan -> seer_sparse_decode
  *
  * Conventions shared by every call
  *   - The caller owns all memory.  The library never allocates or frees.
@@ -103,19 +105,19 @@ typedef struct {
  * seer_kcomp_update -- K Compression Cache maintenance [CP Knowl 5; PN design 2, 4].
  *
  * For every sequence b and KV head h and every block n with
- * valid_blocks[b] <= n < floor(seqlens[b] / b):
+ * valid_blocks[b, h] <= n < floor(seqlens[b] / b):
  *   p = [max | min | avg] over the b pre-RoPE keys of block n (per channel, 3d values)
  *   kcomp[b, h, n, :] = bf16( RoPE_{n*b}( W_k[h] . p ) )      (RoPE rotate-half, theta_i = base^(-2i/d_gate))
- * then valid_blocks[b] = floor(seqlens[b] / b).  Entries below valid_blocks[b] are not
+ * then valid_blocks[b, h] = floor(seqlens[b] / b).  Entries below valid_blocks[b, h] are not
  * touched, so calling this every decode step recomputes a block exactly once, when it
  * fills; valid_blocks = 0 rebuilds the whole cache (prefill).
  *
  *   k_nope        pre-RoPE key cache (see seer_kv_t); may alias the attention K cache
  *   seqlens       device int32 [B]
- *   valid_blocks  device int32 [B], read then written
+ *   valid_blocks  device int32 [B, Hkv] (cache fill count per sequence and KV head), read then written
  *   w_k           device bf16 [Hkv, d_gate, 3*d]  (no bias)
  *   kcomp         device bf16 [B, Hkv, max_blocks, d_gate]
- * Enqueues two kernels (update, then the valid_blocks write).
+ * One launch: a cluster of 8 CTAs per (b, h) shares its new blocks.
  */
 seer_status seer_kcomp_update(const seer_dims_t* dims, const seer_kv_t* k_nope,
                               const int32_t* seqlens, int32_t* valid_blocks, const void* w_k,
@@ -167,13 +169,34 @@ seer_status seer_select_blocks(const seer_dims_t* dims, const float* logits,
                                float tau, int32_t* block_idx, int32_t* block_cnt,
                                int32_t capacity, void* stream);
 
-/* Split count seer_sparse_decode uses when num_split == 0 (host heuristic, no device reads). */
+/*
+ * seer_decode_plan -- seer_kcomp_update + seer_gate_score + seer_select_blocks in one launch.
+ *
+ * Same arguments and results as the three calls made in that order, with these differences:
+ *   valid_blocks  NULL skips the cache update (the cache must then be current already)
+ *   logits_out    device fp32 [B, Hkv, max_blocks] or NULL (the logits stay on chip)
+ * One cluster of 4 CTAs per (b, h): the cache rows of newly full blocks, the gate logits
+ * (shared through distributed shared memory) and the selection never leave the cluster.
+ */
+seer_status seer_decode_plan(const seer_dims_t* dims, const seer_kv_t* k_nope, const int32_t* seqlens,
+                             int32_t* valid_blocks, const void* w_k, void* kcomp, const void* q_nope,
+                             const void* w_q, float* logits_out, float* q_gate_out, int32_t mode,
+                             int32_t token_budget, float tau, int32_t* block_idx, int32_t* block_cnt,
+                             int32_t capacity, void* stream);
+
+/*
+ * A split count for the pages' (num_split, Hkv, B) grid that fills one wave of the SMs (host
+ * heuristic, no device reads).  seer_sparse_decode uses its own balanced schedule when given
+ * num_split == 0; pass this value to get the grid schedule instead.
+ */
 int32_t seer_sparse_decode_auto_split(const seer_dims_t* dims, int32_t capacity);
 
 /*
- * Workspace bytes seer_sparse_decode needs for `num_split` (0 = auto) splits: per-split partial
- * outputs and LSEs plus one arrival counter per (b, h).  The counters must be zero before the
- * first call (e.g. allocate zero-filled); every completed call leaves them zero again.
+ * Workspace bytes seer_sparse_decode needs for `num_split`: one arrival counter per (b, h) plus
+ * fp32 partial outputs and LSEs -- 2 slots per CTA of the balanced schedule (num_split == 0),
+ * num_split slots per (b, h) for the grid schedule, none for num_split == 1.  The counters must
+ * be zero before the first call (e.g. allocate zero-filled); every completed call leaves them
+ * zero again.
  */
 size_t seer_sparse_decode_workspace_bytes(const seer_dims_t* dims, int32_t capacity,
                                           int32_t num_split);
@@ -186,15 +209,19 @@ size_t seer_sparse_decode_workspace_bytes(const seer_dims_t* dims, int32_t capac
  *       [n*b, min((n+1)*b, L_b))
  *   out[b, i] = sum_{t in T} softmax_t(scale * q[b,i] . K[b,h,t]) V[b,h,t]
  *   lse_out[b, i] = log sum_{t in T} exp(scale * q[b,i] . K[b,h,t])   (-inf, out = 0 when T is empty)
- * The list is split along num_split slices of ceil(capacity / num_split) positions (the split
- * size comes from the index tensor width, max_selected_blocks, not from the sequence length);
- * grid (num_split, Hkv, B); the last CTA of each (b, h) merges the partial results.
+ * Schedules:
+ *   num_split >= 1: the pages' grid (num_split, Hkv, B); each list is split into slices of
+ *     ceil(capacity / num_split) positions (the split size comes from the index tensor width,
+ *     max_selected_blocks, not from the sequence length).
+ *   num_split == 0: balanced -- the concatenation of all lists is cut into equal contiguous
+ *     ranges, one per CTA of a grid with one CTA per SM slot.
+ * In both, a (b, h) computed by several CTAs is merged (LSE combine) by the last of them.
  *
  *   q          device bf16 [B, Hq, d]  (post-RoPE query, as the model uses it)
  *   k, v       K and V caches (see seer_kv_t)
  *   block_idx  device int32 [B, Hkv, capacity]; block_cnt device int32 [B, Hkv]
  *   seqlens    device int32 [B]
- *   num_split  0 = seer_sparse_decode_auto_split(); must match the workspace size
+ *   num_split  0 = balanced schedule, >= 1 = grid schedule; must match the workspace size
  *   workspace  device, >= seer_sparse_decode_workspace_bytes(dims, capacity, num_split) bytes
  *   out        device bf16 [B, Hq, d]
  *   lse_out    device fp32 [B, Hq] or NULL

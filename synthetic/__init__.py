@@ -7,6 +7,7 @@ RoPE, scoring, selection or attention).
 
 from .inputs import (  # noqa: F401
     CONFIGS,
+    SWEEP_SPARSITIES,
     DecodeConfig,
     DecodeInputs,
     bf16_bits_from_f32,
@@ -18,4 +19,5 @@ from .inputs import (  # noqa: F401
     make_step_query,
     paged_view,
     scale_gate_weights,
+    sweep_budget,
 )
