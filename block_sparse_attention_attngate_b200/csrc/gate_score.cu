@@ -8,7 +8,10 @@ namespace seer {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kCL = 4;
+#ifndef SEER_GATE_CLUSTER
+#define SEER_GATE_CLUSTER 4   // CTAs per (b, h) cluster
+#endif
+constexpr int kCL = SEER_GATE_CLUSTER;
 
 template <int D, int DG>
 __global__ void __cluster_dims__(kCL, 1, 1) __launch_bounds__(kThreads) gate_score_kernel(const GateParams p) {

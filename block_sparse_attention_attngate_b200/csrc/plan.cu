@@ -5,8 +5,8 @@
 //   1. new full blocks of (b, h) (if any) -> cache rows      (kcomp_device.cuh)
 //   2. Q_gate shared through distributed shared memory, each CTA scores its
 //      1/4 of the cache rows, writing the logits into rank 0's row  (gate_device.cuh)
-//   3. rank 0 selects the blocks from that row: one warp with the row in
-//      registers for rows <= 1024 blocks, the whole CTA otherwise (select_device.cuh)
+//   3. rank 0 selects the blocks from that row, keys in registers for rows of
+//      up to 2048 blocks, in shared memory beyond that or for top-p (select_device.cuh)
 // Equivalent to seer_kcomp_update + seer_gate_score + seer_select_blocks, with
 // two kernel boundaries and the logits' round trip through global memory
 // removed; the sources of each step are cited in its header.
@@ -22,7 +22,10 @@ namespace seer {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kCL = 4;
+#ifndef SEER_GATE_CLUSTER
+#define SEER_GATE_CLUSTER 4   // CTAs per (b, h) cluster
+#endif
+constexpr int kCL = SEER_GATE_CLUSTER;
 
 template <int D, int DG>
 union PlanSmem {
@@ -33,7 +36,12 @@ union PlanSmem {
 template <int D, int BLK, int DG>
 __global__ void __cluster_dims__(kCL, 1, 1) __launch_bounds__(kThreads) plan_kernel(const PlanParams p) {
   __shared__ PlanSmem<D, DG> sm;
-  __shared__ SelectScratch sc;
+  __shared__ union {
+    SelectScratch sc;
+    SelectRegsScratch sr;
+  } ss;
+  SelectScratch& sc = ss.sc;
+  SelectRegsScratch& sr = ss.sr;
   extern __shared__ float row[];   // [NB] logits (rank 0), then selection keys / pairs
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = (int)cluster.block_rank();
@@ -58,14 +66,16 @@ __global__ void __cluster_dims__(kCL, 1, 1) __launch_bounds__(kThreads) plan_ker
   uint32_t* keys = reinterpret_cast<uint32_t*>(row + ((p.s.NB + 1) & ~1));
   uint64_t* pairs = reinterpret_cast<uint64_t*>(keys + ((p.s.NB + 1) & ~1));
   int32_t* out = p.s.idx + (size_t)bh * p.s.cap;
+  const bool partial = (L % p.s.BLK) != 0;
   int total;
-  if (p.s.NB <= kWarpSelectMax && p.s.mode != 2) {
-    if (threadIdx.x >= 32) return;
-    total = select_row_warp<kWarpSelectMax / 32>(row, nfull, (L % p.s.BLK) != 0, p.s.mode, p.s.kblocks, p.s.tau, out,
-                                                 p.s.cap);
+  if (p.s.mode != 2 && p.s.NB <= 2 * kThreads) {
+    total = select_row_regs<kThreads, 2>(row, nfull, partial, p.s.mode, p.s.kblocks, p.s.tau, sr, out, p.s.cap);
+  } else if (p.s.mode != 2 && p.s.NB <= 4 * kThreads) {
+    total = select_row_regs<kThreads, 4>(row, nfull, partial, p.s.mode, p.s.kblocks, p.s.tau, sr, out, p.s.cap);
+  } else if (p.s.mode != 2 && p.s.NB <= 8 * kThreads) {
+    total = select_row_regs<kThreads, 8>(row, nfull, partial, p.s.mode, p.s.kblocks, p.s.tau, sr, out, p.s.cap);
   } else {
-    total = select_row<kThreads>(row, nfull, (L % p.s.BLK) != 0, p.s.mode, p.s.kblocks, p.s.tau, keys, pairs, sc, out,
-                                 p.s.cap);
+    total = select_row<kThreads>(row, nfull, partial, p.s.mode, p.s.kblocks, p.s.tau, keys, pairs, sc, out, p.s.cap);
   }
   if (threadIdx.x == 0) {
     p.s.cnt[bh] = total;

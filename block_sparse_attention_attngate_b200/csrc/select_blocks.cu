@@ -1,5 +1,6 @@
-// Standalone block selection: one CTA per (b, h) runs select_row (select_device.cuh)
-// on its row of gate logits.
+// Standalone block selection: one CTA per (b, h) selects from its row of gate
+// logits (select_device.cuh): select_row_regs for top-k and threshold rows of up
+// to 2048 blocks, select_row otherwise.
 //
 // "SeerAttention-R: Sparse Attention Adaptation for Long Reasoning"
 // (chapterpal.com summary), Knowl 5 (token budget top-k, threshold, forced
@@ -29,36 +30,36 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const SelectParams p) 
   if (threadIdx.x == 0) p.cnt[b * p.Hkv + h] = total;
 }
 
-// rows of at most kWarpSelectMax blocks (top-k, threshold): one warp per (b, h)
-constexpr int kRowsPerCta = 4;
-__global__ void __launch_bounds__(32 * kRowsPerCta) select_warp_kernel(const SelectParams p) {
-  const int row_id = blockIdx.x * kRowsPerCta + (threadIdx.x >> 5);
+// top-k and threshold rows of up to 8 * kRegsThreads blocks: keys in registers
+constexpr int kRegsThreads = 256;
+template <int E>
+__global__ void __launch_bounds__(kRegsThreads) select_regs_kernel(const SelectParams p) {
+  __shared__ SelectRegsScratch sr;
+  const int h = blockIdx.x, b = blockIdx.y;
   pdl_wait();
   pdl_trigger();
-  if (row_id >= p.B * p.Hkv) return;
-  const int b = row_id / p.Hkv;
   const int L = max(p.seqlens[b], 0);
   const int nfull = min(L / p.BLK, p.NB);
-  const float* row = p.logits + (size_t)row_id * p.NB;
-  int32_t* out = p.idx + (size_t)row_id * p.cap;
-  const int total = select_row_warp<kWarpSelectMax / 32>(row, nfull, (L % p.BLK) != 0, p.mode, p.kblocks, p.tau, out,
-                                                         p.cap);
-  if ((threadIdx.x & 31) == 0) p.cnt[row_id] = total;
+  const float* row = p.logits + ((size_t)b * p.Hkv + h) * p.NB;
+  int32_t* out = p.idx + ((size_t)b * p.Hkv + h) * p.cap;
+  const int total = select_row_regs<kRegsThreads, E>(row, nfull, (L % p.BLK) != 0, p.mode, p.kblocks, p.tau, sr,
+                                                     out, p.cap);
+  if (threadIdx.x == 0) p.cnt[b * p.Hkv + h] = total;
 }
 
 }  // namespace
 
 cudaError_t launch_select(const SelectParams& p, cudaStream_t s) {
-  if (p.NB <= kWarpSelectMax && p.mode != 2) {
-    const int rows = p.B * p.Hkv;
-    return launch_pdl(select_warp_kernel, dim3((rows + kRowsPerCta - 1) / kRowsPerCta), dim3(32 * kRowsPerCta), 0, s,
-                      p);
+  const dim3 grid(p.Hkv, p.B);
+  if (p.mode != 2) {
+    if (p.NB <= 2 * kRegsThreads) return launch_pdl(select_regs_kernel<2>, grid, dim3(kRegsThreads), 0, s, p);
+    if (p.NB <= 4 * kRegsThreads) return launch_pdl(select_regs_kernel<4>, grid, dim3(kRegsThreads), 0, s, p);
+    if (p.NB <= 8 * kRegsThreads) return launch_pdl(select_regs_kernel<8>, grid, dim3(kRegsThreads), 0, s, p);
   }
   const size_t smem = select_smem_bytes(p.NB, p.mode);
   static std::atomic<uint64_t> attr_done{0};
   cudaError_t e = ensure_smem_limit(select_kernel, (int)select_smem_bytes(kMaxBlocksRow, 2), attr_done);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.Hkv, p.B);
   return launch_pdl(select_kernel, grid, dim3(kThreads), smem, s, p);
 }
 

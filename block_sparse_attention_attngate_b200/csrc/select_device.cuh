@@ -287,30 +287,39 @@ __device__ int select_row(const float* row, int nfull, bool partial, int mode, i
   return total;
 }
 
-// ---------------------------------------------------------------- one-warp selection
-// Top-k and threshold for rows of at most 32 * KPL blocks, by one warp with the
-// keys in registers (index n = i * 32 + lane): no shared memory, no CTA barrier.
-// Top-k: the k-th largest key T is found bit by bit from the top (count of keys
-// >= candidate, warp-reduced); keys > T are kept, then the lowest-index keys == T
-// until k.  Threshold: S = exp(x - max) / sum in fp64.  Output ascending via
-// ballot prefix counts.  Same results as select_row for these modes.
-constexpr int kWarpSelectMax = 1024;
+// ---------------------------------------------------------------- register-resident selection
+// Top-k and threshold for rows of at most NT * E blocks, by the whole CTA with
+// each thread holding E consecutive indices (n = tid * E + e) as keys in
+// registers.  Top-k: 4-pass 8-bit radix select of the k-th largest key T (one
+// shared atomic per key of the live bucket, bucket search by warp 0, two
+// barriers a pass, early exit when a whole bucket is taken); threshold: max and
+// sum of exp in fp64 by block reductions.  One block-wide scan of the packed
+// (keys > T, keys == T) counts then places every kept index, so the output is
+// ascending and ties at T go to the lowest indices: the same result as
+// select_row for these modes.
+struct SelectRegsScratch {
+  int hist[2][256];
+  int ws[64];
+  double wsd[32];
+  int pick[3];
+};
 
-template <int KPL>
-__device__ int select_row_warp(const float* row, int nfull, bool partial, int mode, int kblocks, double tau,
-                               int32_t* out, int cap) {
-  const int lane = threadIdx.x & 31;
-  const unsigned lt = (1u << lane) - 1u;
-  uint32_t key[KPL];
-  float val[KPL];
+template <int NT, int E>
+__device__ int select_row_regs(const float* row, int nfull, bool partial, int mode, int kblocks, double tau,
+                               SelectRegsScratch& sc, int32_t* out, int cap) {
+  static_assert(NT >= 256 && NT % 32 == 0, "one thread per radix bucket");
+  const int tid = threadIdx.x;
+  const int n0 = tid * E;
+  uint32_t key[E];
+  float val[E];
 #pragma unroll
-  for (int i = 0; i < KPL; ++i) {
-    const int n = i * 32 + lane;
-    val[i] = n < nfull ? row[n] : 0.f;
-    key[i] = n < nfull ? order_key(val[i]) : 0u;   // real keys are never 0
+  for (int e = 0; e < E; ++e) {
+    const int n = n0 + e;
+    val[e] = n < nfull ? row[n] : 0.f;
+    key[e] = n < nfull ? order_key(val[e]) : 0u;   // real keys are never 0
   }
   uint32_t T = 0;
-  int need = 0;     // ties at T to keep (top-k)
+  int rem = 0;          // ties at T to keep (top-k)
   bool all = false;
   double mref = 0.0, ssum = 1.0;
   if (mode == 0) {
@@ -320,61 +329,113 @@ __device__ int select_row_warp(const float* row, int nfull, bool partial, int mo
     } else if (k <= 0) {
       T = 0xffffffffu;
     } else {
-      for (int bit = 31; bit >= 0; --bit) {
-        const uint32_t cand = T | (1u << bit);
-        int c = 0;
-#pragma unroll
-        for (int i = 0; i < KPL; ++i) c += key[i] >= cand;
-        if (__reduce_add_sync(0xffffffffu, (unsigned)c) >= (unsigned)k) T = cand;
+      if (tid < 256) {
+        sc.hist[0][tid] = 0;
+        sc.hist[1][tid] = 0;
       }
-      int gt = 0;
+      __syncthreads();
+      uint32_t prefix = 0, pmask = 0;
+      int want = k;
+      bool whole = false;
+      int cur = 0;
+      for (int pass = 3; pass >= 0 && !whole; --pass, cur ^= 1) {
+        const int shift = pass * 8;
 #pragma unroll
-      for (int i = 0; i < KPL; ++i) gt += key[i] > T;
-      need = k - (int)__reduce_add_sync(0xffffffffu, (unsigned)gt);
+        for (int e = 0; e < E; ++e)
+          if (n0 + e < nfull && (key[e] & pmask) == prefix) atomicAdd(&sc.hist[cur][(key[e] >> shift) & 255u], 1);
+        __syncthreads();
+        if (tid < 32) {
+          // lane l owns digits 255-8l .. 248-8l (descending); a lane scan gives the counts above
+          int c[8], tot = 0;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            c[j] = sc.hist[cur][255 - (8 * tid + j)];
+            tot += c[j];
+          }
+          int incl = tot;
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (tid >= off) incl += y;
+          }
+          int above = incl - tot;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (above < want && above + c[j] >= want) {
+              sc.pick[0] = 255 - (8 * tid + j);
+              sc.pick[1] = want - above;
+              sc.pick[2] = c[j];
+            }
+            above += c[j];
+          }
+        } else {
+          // clear the other histogram for the next pass (threads 32 .. NT-1 cover the 256 buckets)
+          for (int i = tid - 32; i < 256; i += NT - 32) sc.hist[cur ^ 1][i] = 0;
+        }
+        __syncthreads();
+        prefix |= (uint32_t)sc.pick[0] << shift;
+        pmask |= 255u << shift;
+        want = sc.pick[1];
+        whole = sc.pick[2] == want && prefix > 0;   // the whole bucket is taken: its lower bound settles it
+      }
+      if (whole) {
+        T = prefix - 1;
+        rem = 0;
+      } else {
+        T = prefix;
+        rem = want;
+      }
     }
   } else {
     float mx = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < KPL; ++i)
-      if (i * 32 + lane < nfull) mx = fmaxf(mx, val[i]);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    for (int e = 0; e < E; ++e)
+      if (n0 + e < nfull) mx = fmaxf(mx, val[e]);
+    mx = block_reduce<NT, float>(mx, reinterpret_cast<float*>(sc.ws), true);
     mref = (double)mx;
-    double sm = 0.0;
+    double s = 0.0;
 #pragma unroll
-    for (int i = 0; i < KPL; ++i)
-      if (i * 32 + lane < nfull) sm += exp((double)val[i] - mref);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, off);
-    ssum = sm;
+    for (int e = 0; e < E; ++e)
+      if (n0 + e < nfull) s += exp((double)val[e] - mref);
+    ssum = block_reduce<NT, double>(s, sc.wsd, false);
   }
-  int run = 0, ties = 0;
+  // packed counts: kept-for-sure (high 16 bits) and ties at T (low 16 bits); E * NT < 65536
+  bool sel[E];
+  int ngt = 0, neq = 0;
 #pragma unroll
-  for (int i = 0; i < KPL; ++i) {
-    const int n = i * 32 + lane;
-    const bool in = n < nfull;
-    bool sel;
+  for (int e = 0; e < E; ++e) {
+    const bool in = n0 + e < nfull;
     if (all) {
-      sel = in;
+      sel[e] = in;
     } else if (mode == 0) {
-      const bool eq = in && key[i] == T;
-      const unsigned em = __ballot_sync(0xffffffffu, eq);
-      sel = in && (key[i] > T || (eq && ties + __popc(em & lt) < need));
-      ties += __popc(em);
+      sel[e] = in && key[e] > T;
+      neq += (in && key[e] == T) ? 1 : 0;
     } else {
-      sel = in && exp((double)val[i] - mref) / ssum > tau;
+      sel[e] = in && exp((double)val[e] - mref) / ssum > tau;
     }
-    const unsigned sm2 = __ballot_sync(0xffffffffu, sel);
-    const int pos = run + __popc(sm2 & lt);
-    if (sel && pos < cap) out[pos] = n;
-    run += __popc(sm2);
+    ngt += sel[e] ? 1 : 0;
   }
+  int tot;
+  const int pre = block_excl_scan<NT>((ngt << 16) | neq, sc.ws, &tot);
+  const int eq_before = pre & 0xffff;
+  int pos = (pre >> 16) + min(eq_before, rem);
+  int eq_seen = eq_before;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    bool take = sel[e];
+    if (!take && mode == 0 && !all && n0 + e < nfull && key[e] == T) take = eq_seen++ < rem;
+    if (take) {
+      if (pos < cap) out[pos] = n0 + e;
+      ++pos;
+    }
+  }
+  int running = (tot >> 16) + min(tot & 0xffff, rem);
   if (partial) {
-    if (lane == 0 && run < cap) out[run] = nfull;
-    ++run;
+    if (tid == 0 && running < cap) out[running] = nfull;
+    ++running;
   }
-  const int total = min(run, cap);
-  for (int i = total + lane; i < cap; i += 32) out[i] = -1;
+  const int total = min(running, cap);
+  for (int i = total + tid; i < cap; i += NT) out[i] = -1;
   return total;
 }
 

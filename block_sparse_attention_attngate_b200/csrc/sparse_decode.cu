@@ -395,6 +395,7 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NW, STAGES>::kThreads)
       }
       n = ok ? blk : -1;
     };
+    const uint64_t stream_pol = l2_evict_first_policy();   // each K/V tile is read once
     int cn_, cb_, cf_, cp_, cc_, ckb, ckt, cvb, cvt;   // current chunk (this lane's position)
     resolve(lane, cn_, cb_, cf_, cp_, cc_, ckb, ckt, cvb, cvt);
     bool abort = false;
@@ -441,11 +442,11 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NW, STAGES>::kThreads)
                 tile_coords(p.k_perm, kt, h, kb, c1, c2, c3);
 #pragma unroll
                 for (int bx = 0; bx < S::kNBox; ++bx)
-                  tma_load_4d(kdst + bx * S::kBox, &tmK, &full[s], bx * 64, c1, c2, c3);
+                  tma_load_4d_hint(kdst + bx * S::kBox, &tmK, &full[s], bx * 64, c1, c2, c3, stream_pol);
                 tile_coords(p.v_perm, vt, h, vb, c1, c2, c3);
 #pragma unroll
                 for (int bx = 0; bx < S::kNBox; ++bx)
-                  tma_load_4d(vdst + bx * S::kBox, &tmV, &full[s], bx * 64, c1, c2, c3);
+                  tma_load_4d_hint(vdst + bx * S::kBox, &tmV, &full[s], bx * 64, c1, c2, c3, stream_pol);
               }
             } else {
               mbar_arrive(&full[s]);
