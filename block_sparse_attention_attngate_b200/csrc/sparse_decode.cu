@@ -14,24 +14,32 @@
 // group (g <= 8 query heads) stays a 16-row mma.sync fragment: the work per KV
 // byte is ~g multiply-adds and the bound is HBM, not the tensor pipe.
 //
-// CTA structure.  Warp NW is the producer.  It resolves list positions 32 at a
+// CTA structure.  Warp CW is the producer.  It resolves list positions 32 at a
 // time (one lane each: binary search in the shared-memory prefix of the list
 // lengths, one batched load of the block indices, fetched a chunk ahead), and
-// its lane 0 issues 128B-swizzled TMA tile loads of each block's K and V --
-// plus, at a segment's first block, a bulk copy of the group's q rows -- into
-// a STAGES-deep shared-memory ring, completion counted on mbarriers.  Warps
-// 0..NW-1 are consumers; each owns BLK/NW tokens of every block:
+// its lane 0 issues 128B-swizzled TMA tile loads of each block's K and V into
+// a STAGES-deep shared-memory ring (L2 evict-first: every tile is read once),
+// plus a bulk copy of the group's q rows into one of two segment buffers when
+// a segment starts; completion is counted on mbarriers.
+//
+// Warps 0..CW-1 are consumers, in NG groups of NWG warps.  Group k takes the
+// ring iterations it == k (mod NG), so NG blocks are in compute at once and
+// the per-block latency chain (ldmatrix -> mma -> softmax -> mma) is hidden;
+// within a group each warp owns BLK/NWG tokens of the block:
 //   S   = Q K^T        (A = Q from registers, B = K via ldmatrix)
 //   P   = exp2(S*scale*log2e - m)   (fp32 online softmax per query head)
 //   O^T += V^T P^T     (A = V via ldmatrix.trans, B = P from S's accumulator)
-// A segment is a run of consecutive positions of one (b, h) inside one CTA.
-// At its last block the consumers merge their states in shared memory (two
-// alternating merge buffers, one barrier per segment); a segment that is a
-// whole (b, h) writes bf16 out directly, any other writes an fp32 partial and
-// hands it to warp NW+1, the epilogue warp, which publishes it (fence, arrival
-// counter) and, if it was the (b, h)'s last segment to arrive, merges all of
-// its partials -- so the consumers never wait on a global round trip.
-// All waits are bounded.
+// A segment is a run of consecutive positions of one (b, h) inside one CTA;
+// the consumers derive the segments from the same prefix the producer uses.
+// At a segment's end all CW consumer warps meet once: each writes its state to
+// shared memory, per-head merge weights are formed by CW*g threads, and every
+// thread combines its outputs with CW independent multiply-adds.  A segment
+// that is a whole (b, h) writes bf16 out directly; any other writes an fp32
+// partial.  The CTA's first segment, if split, is handed to warp CW+1 (the
+// epilogue warp), which publishes it (fence, arrival counter) and, if it was
+// the (b, h)'s last piece to arrive, merges all of its partials, off the
+// consumers' path; the CTA's last segment is published and, if last to
+// arrive, merged by the consumers themselves.  All waits are bounded.
 #include "seer_device.cuh"
 #include "seer_internal.h"
 
@@ -40,38 +48,39 @@ namespace {
 
 constexpr float kLn2 = 0.6931471805599453f;
 
-constexpr int kSegFirst = 1;  // first block of a segment (the q rows ride along)
-constexpr int kSegLast = 2;   // last block of a segment
+constexpr int kSegFirst = 1;  // first block of a segment (a q copy precedes it)
 
 struct StageInfo {
   int n;       // block index, -1 = skip
-  int bh;      // b * Hkv + h
-  int flags;
-  int pre;     // flattened position of the (b, h)'s first list entry (0 in the grid schedule)
-  int cnt;     // the (b, h)'s list length (clamped to the capacity)
   int pad[3];
 };
 
-template <int D, int BLK, int NW, int STAGES>
+template <int D, int BLK, int NWG, int NG, int STAGES>
 struct DecodeShape {
   static constexpr int kTile = BLK * D * 2;   // bytes of one K (or V) tile
   static constexpr int kBox = BLK * 128;      // bytes of one 64-channel box
   static constexpr int kNBox = D / 64;
-  static constexpr int kTPW = BLK / NW;       // tokens per consumer warp per block
+  static constexpr int kTPW = BLK / NWG;      // tokens per consumer warp per block
   static constexpr int kNT = kTPW / 8;        // 8-token S tiles per warp
   static constexpr int kKS = kTPW / 16;       // 16-token PV k-steps per warp
   static constexpr int kDK = D / 16;          // QK^T k-steps == PV m-tiles
-  static constexpr int kThreads = (NW + 2) * 32;   // consumers, producer, epilogue
+  static constexpr int kCW = NWG * NG;        // consumer warps
+  static constexpr int kThreads = (kCW + 2) * 32;   // consumers, producer, epilogue
   static constexpr int kRing = STAGES * 2 * kTile;
   static constexpr int kQBytes = kMaxGroup * D * 2;
-  static constexpr int kMergeOne = NW * kMaxGroup * D * 4 + 2 * NW * kMaxGroup * 4;
-  static constexpr int kBars = (2 * STAGES + 3) * 8;
+  // merge area: Ow[CW][8][D], Mw[CW][8], Lw[CW][8], Wt[CW][8], Hs[8]
+  static constexpr int kMergeFloats = kCW * kMaxGroup * D + 3 * kCW * kMaxGroup + kMaxGroup;
+  static constexpr int kBars = (2 * STAGES + 7) * 8;   // full, empty, qfull[2], qempty[2], cbar, jbar[2]
+  static constexpr int kEpi = 256;   // partial LSEs (segment-major) / merge weights, + per-head M, sum
+  static constexpr int kSh = 32;     // shared scalars
   // fixed part; the list prefix and the sequence lengths follow (sized per launch)
-  static constexpr int kEpi = 256;   // epilogue scratch: partial LSEs (segment-major) + per-head M, sum
-  static constexpr size_t kSmemFixed = 1024 + kRing + STAGES * kQBytes + 2 * kMergeOne + kBars +
-                                       STAGES * sizeof(StageInfo) + 2 * 16 + (kEpi + 2 * kMaxGroup) * 4 + 16 * 4;
+  static constexpr size_t kSmemFixed = 1024 + kRing + 2 * kQBytes + (size_t)kMergeFloats * 4 + kBars +
+                                       STAGES * sizeof(StageInfo) + 16 + (kEpi + 2 * kMaxGroup) * 4 +
+                                       kSh * 4 + 2 * STAGES * 4;
   static_assert(kTPW % 16 == 0, "each consumer warp needs whole 16-token steps");
   static_assert(D % 64 == 0, "head_dim must be a multiple of 64");
+  static_assert(STAGES % NG == 0, "each ring stage belongs to one consumer group");
+  static_assert(kMergeFloats >= kEpi + 2 * kMaxGroup, "the merge area doubles as the final merge's scratch");
 };
 
 __device__ __forceinline__ void tile_coords(const int32_t perm[3], int t, int h, int bp, int& c1, int& c2,
@@ -90,11 +99,19 @@ __device__ __forceinline__ int clamp_cnt(const DecodeParams& p, int i) {
   return c < 0 ? 0 : (c > p.cap ? p.cap : c);
 }
 
+// floor(a / b) for 0 <= a < 2^53, 0 < b: a double quotient, then exact integer corrections
+// (a 64-bit integer division is a long software sequence; this is a few instructions)
+__device__ __forceinline__ long long floor_div(long long a, long long b) {
+  long long q = (long long)((double)a / (double)b);
+  while (q > 0 && q * b > a) --q;
+  while ((q + 1) * b <= a) ++q;
+  return q;
+}
 // Balanced schedule: CTA c of G owns flattened positions [lo(c), lo(c+1)).
-__device__ __forceinline__ long long range_lo(long long c, long long W, long long G) { return c * W / G; }
+__device__ __forceinline__ long long range_lo(long long c, long long W, long long G) { return floor_div(c * W, G); }
 // The CTA whose range holds position `pos`.
 __device__ __forceinline__ int cta_of(long long pos, long long W, long long G) {
-  return (int)(((pos + 1) * G - 1) / W);
+  return (int)floor_div((pos + 1) * G - 1, W);
 }
 // Last index i in [0, n) with pre[i] <= x (pre non-decreasing, pre[0] = 0 <= x).
 __device__ __forceinline__ int bh_of(const int* pre, int n, int x) {
@@ -118,27 +135,119 @@ __device__ __forceinline__ int split_slot(const DecodeParams& p, int bh, int k, 
   return k == 0 ? slot_first : (p.flat ? 2 * (cf + k) : bh * p.ns + k);
 }
 
-template <int D, int BLK, int NW, int STAGES>
-__global__ void __launch_bounds__(DecodeShape<D, BLK, NW, STAGES>::kThreads)
+// Merge the nseg partials (o, lse) of one (b, h) into bf16 out (and lse_out), by the NT threads
+// whose index is `t` (0 <= t < NT).  `wsc` is shared scratch of >= kEpi + 2*kMaxGroup floats;
+// `sync()` is a barrier among those NT threads.  Partials are read with L2-coherent loads.
+template <int D, int NT, int kEpi, typename Sync>
+__device__ void merge_partials(const DecodeParams& p, int bh, int nseg, int slot_first, int cf, int t, float* wsc,
+                               Sync sync) {
+  const int g = p.g;
+  const int b = bh / p.Hkv, h = bh - b * p.Hkv;
+  const size_t qh0 = (size_t)b * p.Hq + (size_t)h * g;
+  const int ng = nseg * g;
+  if (ng <= kEpi) {
+    // partial LSEs -> shared; per-head max and weight sum; weights w[k][j] = exp(lse - M) / Z
+    float* Mh = wsc + kEpi;
+    float* Zh = Mh + kMaxGroup;
+    for (int i = t; i < ng; i += NT)
+      wsc[i] = __ldcg(p.lse_part + (size_t)split_slot(p, bh, i / g, slot_first, cf) * g + (i % g));
+    sync();
+    if (t < g) {
+      float M = -INFINITY;
+      for (int k = 0; k < nseg; ++k) M = fmaxf(M, wsc[k * g + t]);
+      float Z = 0.f;
+      if (M != -INFINITY)
+        for (int k = 0; k < nseg; ++k) Z += expf(wsc[k * g + t] - M);
+      Mh[t] = M;
+      Zh[t] = Z;
+    }
+    sync();
+    for (int i = t; i < ng; i += NT) {
+      const int j = i % g;
+      const float M = Mh[j], Z = Zh[j];
+      wsc[i] = (M != -INFINITY && Z > 0.f) ? expf(wsc[i] - M) / Z : 0.f;
+    }
+    sync();
+    constexpr int EPT = (kMaxGroup * D + NT - 1) / NT;
+    float acc[EPT];
+#pragma unroll
+    for (int u = 0; u < EPT; ++u) acc[u] = 0.f;
+    for (int k = 0; k < nseg; ++k) {
+      const size_t sl = (size_t)split_slot(p, bh, k, slot_first, cf);
+#pragma unroll
+      for (int u = 0; u < EPT; ++u) {
+        const int e = u * NT + t;
+        if (e < g * D) {
+          const int j = e / D;
+          acc[u] += wsc[k * g + j] * __ldcg(p.o_part + (sl * g + j) * D + (e - j * D));
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < EPT; ++u) {
+      const int e = u * NT + t;
+      if (e < g * D) {
+        const int j = e / D, cc = e - j * D;
+        __nv_bfloat16 ob = __float2bfloat16_rn(acc[u]);
+        p.out[(qh0 + j) * D + cc] = *reinterpret_cast<uint16_t*>(&ob);
+        if (cc == 0 && p.lse_out) p.lse_out[qh0 + j] = Zh[j] > 0.f ? Mh[j] + logf(Zh[j]) : -INFINITY;
+      }
+    }
+  } else {
+    for (int e = t; e < g * D; e += NT) {
+      const int j = e / D, cc = e % D;
+      float M = -INFINITY;
+      for (int k = 0; k < nseg; ++k)
+        M = fmaxf(M, __ldcg(p.lse_part + (size_t)split_slot(p, bh, k, slot_first, cf) * g + j));
+      float num = 0.f, den = 0.f;
+      if (M != -INFINITY) {
+        for (int k = 0; k < nseg; ++k) {
+          const size_t sl = (size_t)split_slot(p, bh, k, slot_first, cf);
+          const float w = expf(__ldcg(p.lse_part + sl * g + j) - M);
+          num += w * __ldcg(p.o_part + (sl * g + j) * D + cc);
+          den += w;
+        }
+      }
+      const bool any = den > 0.f;
+      __nv_bfloat16 ob = __float2bfloat16_rn(any ? num / den : 0.f);
+      p.out[(qh0 + j) * D + cc] = *reinterpret_cast<uint16_t*>(&ob);
+      if (cc == 0 && p.lse_out) p.lse_out[qh0 + j] = any ? M + logf(den) : -INFINITY;
+    }
+  }
+}
+
+template <int D, int BLK, int NWG, int NG, int STAGES>
+__global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads, 1)
     sparse_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                          const DecodeParams p) {
-  using S = DecodeShape<D, BLK, NW, STAGES>;
+  using S = DecodeShape<D, BLK, NWG, NG, STAGES>;
+  constexpr int CW = S::kCW;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
-  uint8_t* qbuf = ring + S::kRing;
-  float* merge = reinterpret_cast<float*>(qbuf + STAGES * S::kQBytes);   // 2 x {Ow[NW][8][D], Mw[NW][8], Lw[NW][8]}
-  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(merge) + 2 * S::kMergeOne);
+  uint8_t* qseg = ring + S::kRing;                                   // [2] segment q rows
+  float* Ow = reinterpret_cast<float*>(qseg + 2 * S::kQBytes);       // [CW][8][D]
+  float* Mw = Ow + CW * kMaxGroup * D;                               // [CW][8]
+  float* Lw = Mw + CW * kMaxGroup;                                   // [CW][8]
+  float* Wt = Lw + CW * kMaxGroup;                                   // [CW][8] merge weights
+  float* Hs = Wt + CW * kMaxGroup;                                   // [8] segment LSE
+  uint64_t* full = reinterpret_cast<uint64_t*>(Ow + S::kMergeFloats);
   uint64_t* empty = full + STAGES;
-  uint64_t* cbar = empty + STAGES;   // consumer-warp barrier
-  uint64_t* jbar = cbar + 1;         // [2] split-segment hand-off to the epilogue warp
+  uint64_t* qfull = empty + STAGES;   // [2]
+  uint64_t* qempty = qfull + 2;       // [2]
+  uint64_t* cbar = qempty + 2;        // consumer-warp barrier
+  uint64_t* jbar = cbar + 1;          // split first segment handed to the epilogue warp
   StageInfo* info = reinterpret_cast<StageInfo*>(jbar + 2);
   Job* job = reinterpret_cast<Job*>(info + STAGES);
-  float* epi = reinterpret_cast<float*>(job + 2);   // [kEpi] + [2 * kMaxGroup]
-  // sh[0] abort, sh[2] W, sh[3] G_eff, sh[4] p0, sh[5] p1, sh[6] first bh, sh[7] its pre
+  float* epi = reinterpret_cast<float*>(job + 1);   // [kEpi] + [2 * kMaxGroup]
+  // sh[0] abort, sh[1] merge flag, sh[2] W, sh[3] G_eff, sh[4] p0, sh[5] p1, sh[6] first bh,
+  // sh[7] its pre, sh[9] producer done, sh[10..12] first segment {cf, nseg, slot_first},
+  // sh[13..15] last segment {cf, nseg, slot_first}, sh[16] last bh, sh[17] sh[10..15] ready
   volatile int* sh = reinterpret_cast<volatile int*>(epi + S::kEpi + 2 * kMaxGroup);
-  int* slen = const_cast<int*>(reinterpret_cast<volatile int*>(sh + 16));   // [B] sequence lengths
-  int* pre = slen + p.B;                                                       // [BH + 1] list prefix
+  volatile int* issued = sh + S::kSh;         // [STAGES] tiles issued per stage
+  volatile int* observed = issued + STAGES;   // [STAGES] full phases observed per stage
+  int* slen = const_cast<int*>(observed + STAGES);   // [B] sequence lengths
+  int* pre = slen + p.B;                              // [BH + 1] list prefix
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tid = threadIdx.x;
@@ -149,12 +258,18 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NW, STAGES>::kThreads)
     tma_prefetch_desc(&tmV);
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], NW);
+      mbar_init(&empty[s], NWG);
+      issued[s] = 0;
+      observed[s] = 0;
     }
-    mbar_init(cbar, NW);
-    mbar_init(&jbar[0], NW);
-    mbar_init(&jbar[1], NW);
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(&qfull[k], 1);
+      mbar_init(&qempty[k], CW);
+    }
+    mbar_init(cbar, CW);
+    mbar_init(jbar, CW);
     sh[0] = 0;
+    sh[9] = 0;
     fence_barrier_init();
   }
   pdl_wait();
@@ -182,7 +297,7 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NW, STAGES>::kThreads)
       const int y = __shfl_up_sync(0xffffffffu, incl, off);
       if (lane >= off) incl += y;
     }
-    int* wsum = pre + BH + 1;   // scratch for NW+1 warp totals, just past the prefix
+    int* wsum = pre + BH + 1;   // scratch for the warp totals, just past the prefix
     if (lane == 31) wsum[warp] = incl;
     __syncthreads();
     int before = 0;
@@ -206,168 +321,102 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NW, STAGES>::kThreads)
         p0 = range_lo(c, W, G);
         p1 = range_lo(c + 1, W, G);
       }
-      const int bh0 = p1 > p0 ? bh_of(pre, BH, (int)p0) : 0;
+      const int bf = p1 > p0 ? bh_of(pre, BH, (int)p0) : 0;
+      const int bl = p1 > p0 ? bh_of(pre, BH, (int)p1 - 1) : 0;
       sh[2] = W;
       sh[3] = (int)G;
       sh[4] = (int)p0;
       sh[5] = (int)p1;
-      sh[6] = bh0;
-      sh[7] = pre[bh0];
+      sh[6] = bf;
+      sh[7] = pre[bf];
+      sh[16] = bl;
+      sh[17] = 0;   // split bookkeeping below is filled in by the epilogue warp, off the critical path
     }
   } else if (tid == 0) {
     const int bh = blockIdx.z * p.Hkv + blockIdx.y;
     const int c = clamp_cnt(p, bh);
     if (p.cnt[bh] > p.cap && blockIdx.x == 0) report(p.err, SEER_DEVERR_COUNT);
     const int a = min((int)blockIdx.x * p.per_split, c), e = min(a + p.per_split, c);
+    const int nseg = (c + p.per_split - 1) / p.per_split;
     sh[2] = 0;
     sh[3] = 0;
     sh[4] = a;   // positions are local to the (b, h) in this schedule
     sh[5] = e;
     sh[6] = bh;
     sh[7] = 0;
+    sh[16] = bh;
+    sh[10] = sh[13] = 0;
+    sh[11] = sh[14] = nseg;
+    sh[12] = sh[15] = bh * p.ns;
+    sh[17] = 1;
     pre[0] = c;  // the grid schedule keeps its one list length here
   }
   __syncthreads();
   const int nit = sh[5] - sh[4];
 
-  if (warp == NW + 1) {
+  if (warp == CW + 1) {
     // ------------------------------------------------------------ epilogue warp
-    // Which of this CTA's segments belong to a (b, h) split across CTAs (or splits)?
-    bool expect[2] = {false, false};
-    if (nit > 0) {
-      if (p.flat) {
+    if (p.flat && lane == 0) {
+      // split bookkeeping of the CTA's first and last segments (a middle one is a whole (b, h)):
+      // the CTA of the first piece, the piece count and the first piece's partial slot
+      if (nit > 0) {
         const long long W = sh[2], G = sh[3];
-        const int p0 = sh[4], p1 = sh[5];
-        const int bf = sh[6];
-        const int bl = bh_of(pre, BH, p1 - 1);
-        auto split = [&](int x) { return cta_of(pre[x + 1] - 1, W, G) != cta_of(pre[x], W, G); };
-        (void)p0;
-        // the CTA's last segment is merged by the consumers themselves (it sets the kernel's tail)
-        expect[0] = bl != bf && split(bf);
+        const int bf = sh[6], bl = sh[16];
+        const int cf_f = cta_of(pre[bf], W, G), cf_l = cta_of(pre[bl], W, G);
+        sh[10] = cf_f;
+        sh[11] = cta_of(pre[bf + 1] - 1, W, G) - cf_f + 1;
+        sh[12] = 2 * cf_f + (range_lo(cf_f, W, G) != pre[bf] ? 1 : 0);
+        sh[13] = cf_l;
+        sh[14] = cta_of(pre[bl + 1] - 1, W, G) - cf_l + 1;
+        sh[15] = 2 * cf_l + (range_lo(cf_l, W, G) != pre[bl] ? 1 : 0);
       }
+      __threadfence_block();
+      sh[17] = 1;
     }
-    for (int k = 0; k < 2; ++k) {
-      if (!expect[k]) continue;
-      if (!__all_sync(0xffffffffu, mbar_wait(&jbar[k], 0))) {
+    __syncwarp();
+    // The CTA's first segment, when it is split across CTAs and is not also its last segment,
+    // is published (and merged, if it arrives last) here.
+    const bool expect = nit > 0 && p.flat && sh[16] != sh[6] && sh[11] > 1;
+    if (expect) {
+      if (!__all_sync(0xffffffffu, mbar_wait(jbar, 0))) {
         if (lane == 0) report(p.err, SEER_DEVERR_TIMEOUT);
-        break;
+        return;
       }
-      const Job jb = job[k];
+      const Job jb = job[0];
       int last = 0;
       // publish the consumers' partial (ordered before the hand-off) and learn whether this
       // segment is the (b, h)'s last to arrive; acquire the others' partials if so
       if (lane == 0) last = atomic_add_acq_rel_gpu(&p.counters[jb.bh], 1) == jb.nseg - 1;
-      if (!__shfl_sync(0xffffffffu, last, 0)) continue;
-      const int b = jb.bh / p.Hkv, h = jb.bh - b * p.Hkv;
-      const size_t qh0 = (size_t)b * p.Hq + (size_t)h * g;
-      const int ng = jb.nseg * g;
-      float* Mh = epi + S::kEpi;
-      float* Zh = Mh + kMaxGroup;
-      if (ng <= S::kEpi) {
-        // partial LSEs -> shared (one round trip), per-head max and weight sum, then each lane
-        // accumulates its outputs with one round of independent loads per segment
-        for (int i0 = 0; i0 < ng; i0 += 32) {
-          const int i = i0 + lane;
-          if (i < ng)
-            epi[i] = __ldcg(p.lse_part + (size_t)split_slot(p, jb.bh, i / g, jb.slot_first, jb.cf) * g + (i % g));
-        }
+      if (__shfl_sync(0xffffffffu, last, 0)) {
+        merge_partials<D, 32, S::kEpi>(p, jb.bh, jb.nseg, jb.slot_first, jb.cf, lane, epi,
+                                       [] { __syncwarp(); });
         __syncwarp();
-        if (lane < g) {
-          float M = -INFINITY;
-          for (int s2 = 0; s2 < jb.nseg; ++s2) M = fmaxf(M, epi[s2 * g + lane]);
-          float Z = 0.f;
-          if (M != -INFINITY)
-            for (int s2 = 0; s2 < jb.nseg; ++s2) Z += expf(epi[s2 * g + lane] - M);
-          Mh[lane] = M;
-          Zh[lane] = Z;
-        }
-        __syncwarp();
-        for (int i0 = 0; i0 < ng; i0 += 32) {
-          const int i = i0 + lane;
-          if (i < ng) {
-            const float M = Mh[i % g];
-            epi[i] = M != -INFINITY ? expf(epi[i] - M) : 0.f;
-          }
-        }
-        __syncwarp();
-        constexpr int EPT = kMaxGroup * D / 32;
-        float acc[EPT];
-#pragma unroll
-        for (int t = 0; t < EPT; ++t) acc[t] = 0.f;
-        for (int s2 = 0; s2 < jb.nseg; ++s2) {
-          const size_t sl = (size_t)split_slot(p, jb.bh, s2, jb.slot_first, jb.cf);
-#pragma unroll
-          for (int t = 0; t < EPT; ++t) {
-            const int e = t * 32 + lane;
-            if (e < g * D) {
-              const int j = e / D;
-              acc[t] += epi[s2 * g + j] * __ldcg(p.o_part + (sl * g + j) * D + (e - j * D));
-            }
-          }
-        }
-#pragma unroll
-        for (int t = 0; t < EPT; ++t) {
-          const int e = t * 32 + lane;
-          if (e < g * D) {
-            const int j = e / D, cc = e - j * D;
-            const float Z = Zh[j];
-            __nv_bfloat16 ob = __float2bfloat16_rn(Z > 0.f ? acc[t] / Z : 0.f);
-            p.out[(qh0 + j) * D + cc] = *reinterpret_cast<uint16_t*>(&ob);
-            if (cc == 0 && p.lse_out) p.lse_out[qh0 + j] = Z > 0.f ? Mh[j] + logf(Z) : -INFINITY;
-          }
-        }
-      } else {
-        for (int e = lane; e < g * D; e += 32) {
-          const int j = e / D, cc = e % D;
-          float M = -INFINITY;
-          for (int s2 = 0; s2 < jb.nseg; ++s2)
-            M = fmaxf(M, __ldcg(p.lse_part + (size_t)split_slot(p, jb.bh, s2, jb.slot_first, jb.cf) * g + j));
-          float num = 0.f, den = 0.f;
-          if (M != -INFINITY) {
-            for (int s2 = 0; s2 < jb.nseg; ++s2) {
-              const size_t sl = (size_t)split_slot(p, jb.bh, s2, jb.slot_first, jb.cf);
-              const float w = expf(__ldcg(p.lse_part + sl * g + j) - M);
-              num += w * __ldcg(p.o_part + (sl * g + j) * D + cc);
-              den += w;
-            }
-          }
-          const bool any = den > 0.f;
-          __nv_bfloat16 ob = __float2bfloat16_rn(any ? num / den : 0.f);
-          p.out[(qh0 + j) * D + cc] = *reinterpret_cast<uint16_t*>(&ob);
-          if (cc == 0 && p.lse_out) p.lse_out[qh0 + j] = any ? M + logf(den) : -INFINITY;
-        }
+        if (lane == 0) p.counters[jb.bh] = 0;
       }
-      __syncwarp();
-      if (lane == 0) p.counters[jb.bh] = 0;
     }
     return;
   }
 
-  if (warp == NW) {
+  if (warp == CW) {
     // ------------------------------------------------------------ producer warp
     const int p0 = sh[4];
     const int fixed_bh = sh[6];
     // resolve list position `it` of this CTA (one lane per position)
-    auto resolve = [&](int it, int& n, int& bh, int& flags, int& pr, int& cn, int& kb, int& kt, int& vb, int& vt) {
+    auto resolve = [&](int it, int& n, int& bh, int& first, int& kb, int& kt, int& vb, int& vt) {
       n = -1;
       bh = fixed_bh;
-      flags = 0;
-      pr = 0;
-      cn = 0;
+      first = 0;
       kb = vb = kt = vt = 0;
       if (it >= nit) return;
       int pos;
       if (p.flat) {
         const int x = p0 + it;
         bh = bh_of(pre, BH, x);
-        pr = pre[bh];
-        cn = pre[bh + 1] - pr;
-        pos = x - pr;
+        pos = x - pre[bh];
       } else {
-        cn = pre[0];
         pos = p0 + it;
       }
-      flags = ((it == 0 || pos == 0) ? kSegFirst : 0) | ((it == nit - 1 || pos == cn - 1) ? kSegLast : 0);
+      first = (it == 0 || pos == 0) ? kSegFirst : 0;
       const int b = bh / p.Hkv;
       const int nblk = (slen[b] + BLK - 1) / BLK;
       const int blk = p.idx[(size_t)bh * p.cap + pos];
@@ -396,61 +445,62 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NW, STAGES>::kThreads)
       n = ok ? blk : -1;
     };
     const uint64_t stream_pol = l2_evict_first_policy();   // each K/V tile is read once
-    int cn_, cb_, cf_, cp_, cc_, ckb, ckt, cvb, cvt;   // current chunk (this lane's position)
-    resolve(lane, cn_, cb_, cf_, cp_, cc_, ckb, ckt, cvb, cvt);
+    const uint32_t qbytes = (uint32_t)(g * D * 2);
+    int nq = 0;   // segments whose q copy was issued
+    int cn_, cb_, cf_, ckb, ckt, cvb, cvt;   // current chunk (this lane's position)
+    resolve(lane, cn_, cb_, cf_, ckb, ckt, cvb, cvt);
     bool abort = false;
     for (int chunk = 0; chunk * 32 < nit && !abort; ++chunk) {
-      int nn, nb, nf, np, nc, nkb, nkt, nvb, nvt;   // next chunk, fetched while this one issues
-      resolve((chunk + 1) * 32 + lane, nn, nb, nf, np, nc, nkb, nkt, nvb, nvt);
+      int nn, nb, nf, nkb, nkt, nvb, nvt;   // next chunk, fetched while this one issues
+      resolve((chunk + 1) * 32 + lane, nn, nb, nf, nkb, nkt, nvb, nvt);
       const int count = min(32, nit - chunk * 32);
       for (int j = 0; j < count; ++j) {
         const int it = chunk * 32 + j;
         const int n = __shfl_sync(0xffffffffu, cn_, j);
         const int bh = __shfl_sync(0xffffffffu, cb_, j);
-        const int flags = __shfl_sync(0xffffffffu, cf_, j);
-        const int prv = __shfl_sync(0xffffffffu, cp_, j);
-        const int cnv = __shfl_sync(0xffffffffu, cc_, j);
+        const int first = __shfl_sync(0xffffffffu, cf_, j);
         const int kb = __shfl_sync(0xffffffffu, ckb, j), kt = __shfl_sync(0xffffffffu, ckt, j);
         const int vb = __shfl_sync(0xffffffffu, cvb, j), vt = __shfl_sync(0xffffffffu, cvt, j);
         if (lane == 0) {
+          if (first) {
+            // the segment's q rows -> segment buffer nq & 1, once the segment two back has read it
+            const int k = nq & 1, u = nq >> 1;
+            if (u >= 1 && !mbar_wait(&qempty[k], (u - 1) & 1)) {
+              report(p.err, SEER_DEVERR_TIMEOUT);
+              sh[0] = 1;
+            }
+            if (!sh[0]) {
+              const int b = bh / p.Hkv, h = bh - b * p.Hkv;
+              mbar_arrive_expect_tx(&qfull[k], qbytes);
+              bulk_load(qseg + k * S::kQBytes, p.q + ((size_t)b * p.Hq + (size_t)h * g) * D, qbytes, &qfull[k]);
+            }
+            ++nq;
+          }
           const int s = it % STAGES;
-          if (it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) - 1) & 1)) {
+          if (!sh[0] && it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) - 1) & 1)) {
             report(p.err, SEER_DEVERR_TIMEOUT);
             sh[0] = 1;
           }
           if (!sh[0]) {
-            StageInfo& si = info[s];
-            si.n = n;
-            si.bh = bh;
-            si.flags = flags;
-            si.pre = prv;
-            si.cnt = cnv;
-            const bool first = flags & kSegFirst;
-            const uint32_t qbytes = (uint32_t)(g * D * 2);
-            const uint32_t tx = (n >= 0 ? 2u * S::kTile : 0u) + (first ? qbytes : 0u);
-            if (tx) {
-              mbar_arrive_expect_tx(&full[s], tx);
-              if (first) {
-                const int b = bh / p.Hkv, h = bh - b * p.Hkv;
-                bulk_load(qbuf + s * S::kQBytes, p.q + ((size_t)b * p.Hq + (size_t)h * g) * D, qbytes, &full[s]);
-              }
-              if (n >= 0) {
-                const int h = bh % p.Hkv;
-                uint8_t* kdst = ring + s * 2 * S::kTile;
-                uint8_t* vdst = kdst + S::kTile;
-                int c1, c2, c3;
-                tile_coords(p.k_perm, kt, h, kb, c1, c2, c3);
+            info[s].n = n;
+            if (n >= 0) {
+              mbar_arrive_expect_tx(&full[s], 2u * S::kTile);
+              const int h = bh % p.Hkv;
+              uint8_t* kdst = ring + s * 2 * S::kTile;
+              uint8_t* vdst = kdst + S::kTile;
+              int c1, c2, c3;
+              tile_coords(p.k_perm, kt, h, kb, c1, c2, c3);
 #pragma unroll
-                for (int bx = 0; bx < S::kNBox; ++bx)
-                  tma_load_4d_hint(kdst + bx * S::kBox, &tmK, &full[s], bx * 64, c1, c2, c3, stream_pol);
-                tile_coords(p.v_perm, vt, h, vb, c1, c2, c3);
+              for (int bx = 0; bx < S::kNBox; ++bx)
+                tma_load_4d_hint(kdst + bx * S::kBox, &tmK, &full[s], bx * 64, c1, c2, c3, stream_pol);
+              tile_coords(p.v_perm, vt, h, vb, c1, c2, c3);
 #pragma unroll
-                for (int bx = 0; bx < S::kNBox; ++bx)
-                  tma_load_4d_hint(vdst + bx * S::kBox, &tmV, &full[s], bx * 64, c1, c2, c3, stream_pol);
-              }
+              for (int bx = 0; bx < S::kNBox; ++bx)
+                tma_load_4d_hint(vdst + bx * S::kBox, &tmV, &full[s], bx * 64, c1, c2, c3, stream_pol);
             } else {
               mbar_arrive(&full[s]);
             }
+            issued[s] = issued[s] + 1;
           }
         }
         if (__shfl_sync(0xffffffffu, (int)sh[0], 0)) {
@@ -458,162 +508,195 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NW, STAGES>::kThreads)
           break;
         }
       }
-      cn_ = nn; cb_ = nb; cf_ = nf; cp_ = np; cc_ = nc; ckb = nkb; ckt = nkt; cvb = nvb; cvt = nvt;
+      cn_ = nn; cb_ = nb; cf_ = nf; ckb = nkb; ckt = nkt; cvb = nvb; cvt = nvt;
+    }
+    if (lane == 0) {
+      __threadfence_block();
+      sh[9] = 1;
     }
     return;
   }
 
   // -------------------------------------------------------------- consumers
+  const int cg = warp / NWG, wg = warp - cg * NWG;
   const int gq = lane >> 2, tq = lane & 3;
-  uint32_t qa[S::kDK][2];
-  float o[S::kDK][4];
-#pragma unroll
-  for (int i = 0; i < S::kDK; ++i) {
-    qa[i][0] = qa[i][1] = 0u;
-    o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-  }
-  float m_run = -INFINITY, l_run = 0.f;
   const float sl2 = p.scale_log2;
-  const int tok_base = warp * S::kTPW;
-  int L = 0;
-  int seg_start_it = 0;
-  int consumed = 0;
-  int nflush = 0;
+  const int tok_base = wg * S::kTPW;
+  const int p0 = sh[4], p1 = sh[5];
   uint32_t cphase = 0;
   bool alive = true;
+  uint32_t qa[S::kDK][2];
+  float o[S::kDK][4];
 
-  for (int it = 0; it < nit; ++it) {
-    const int s = it % STAGES;
-    // every lane observes the phase (acquire); the warp leaves together if any lane gave up
-    if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (it / STAGES) & 1))) {
+  int it0 = 0, seg = 0;
+  while (it0 < nit) {
+    // ---- this segment: [it0, it1) of (b, h) = bh
+    int bh, it1;
+    if (p.flat) {
+      bh = bh_of(pre, BH, p0 + it0);
+      it1 = min(p1, pre[bh + 1]) - p0;
+    } else {
+      bh = sh[6];
+      it1 = nit;
+    }
+    // the group's q rows (rows >= g stay zero), then release the segment buffer
+    if (!__all_sync(0xffffffffu, mbar_wait(&qfull[seg & 1], (seg >> 1) & 1))) {
       alive = false;
       break;
     }
-    consumed = it + 1;
-    const int si_n = info[s].n, si_bh = info[s].bh, si_flags = info[s].flags;
-    const int si_pre = info[s].pre, si_cnt = info[s].cnt;
-    if (si_flags & kSegFirst) {
-      // new segment: the group's q rows (rows >= g stay zero) and a fresh state
-      const uint8_t* qs = qbuf + s * S::kQBytes;
+    {
+      const uint8_t* qs = qseg + (seg & 1) * S::kQBytes;
       const bool live = gq < g;
 #pragma unroll
       for (int ks = 0; ks < S::kDK; ++ks) {
         qa[ks][0] = live ? *reinterpret_cast<const uint32_t*>(qs + (gq * D + ks * 16 + 2 * tq) * 2) : 0u;
         qa[ks][1] = live ? *reinterpret_cast<const uint32_t*>(qs + (gq * D + ks * 16 + 8 + 2 * tq) * 2) : 0u;
       }
-#pragma unroll
-      for (int i = 0; i < S::kDK; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-      m_run = -INFINITY;
-      l_run = 0.f;
-      L = slen[si_bh / p.Hkv];
-      seg_start_it = it;
-    }
-    if (si_n >= 0) {
-      const uint32_t kt = smem_u32(ring + s * 2 * S::kTile);
-      const uint32_t vt = kt + S::kTile;
-      const int valid = min(BLK, L - si_n * BLK);
-      // ---- S = Q K^T for this warp's tokens
-      float sacc[S::kNT][4];
-#pragma unroll
-      for (int j = 0; j < S::kNT; ++j) {
-        sacc[j][0] = sacc[j][1] = sacc[j][2] = sacc[j][3] = 0.f;
-        const uint32_t row = tok_base + j * 8 + (lane & 7);
-#pragma unroll
-        for (int kp = 0; kp < S::kDK / 2; ++kp) {
-          const uint32_t chunk = kp * 4 + (lane >> 3);
-          uint32_t r0, r1, r2, r3;
-          ldsm_x4(kt + (chunk >> 3) * S::kBox + sw128(row, chunk & 7), r0, r1, r2, r3);
-          mma_bf16_16816(sacc[j], qa[2 * kp][0], 0u, qa[2 * kp][1], 0u, r0, r1);
-          mma_bf16_16816(sacc[j], qa[2 * kp + 1][0], 0u, qa[2 * kp + 1][1], 0u, r2, r3);
-        }
-      }
-      // ---- online softmax (row = query head gq; this lane holds tokens 2tq, 2tq+1 of each tile)
-      float sv[S::kNT][2];
-      float mx = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < S::kNT; ++j) {
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int tok = tok_base + j * 8 + 2 * tq + e;
-          const float v = tok < valid ? sacc[j][e] * sl2 : -INFINITY;
-          sv[j][e] = v;
-          mx = fmaxf(mx, v);
-        }
-      }
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      const float m_new = fmaxf(m_run, mx);
-      const float m_use = m_new == -INFINITY ? 0.f : m_new;
-      const float alpha = exp2f(m_run - m_use);
-      m_run = m_new;
-      uint32_t pb[S::kNT];
-      float ls = 0.f;
-#pragma unroll
-      for (int j = 0; j < S::kNT; ++j) {
-        pb[j] = pack_bf16(exp2f(sv[j][0] - m_use), exp2f(sv[j][1] - m_use));
-        ls += bf16_lo(pb[j]) + bf16_hi(pb[j]);
-      }
-      l_run = l_run * alpha + ls;
-      const float a0 = __shfl_sync(0xffffffffu, alpha, (2 * tq) * 4);
-      const float a1 = __shfl_sync(0xffffffffu, alpha, (2 * tq + 1) * 4);
-#pragma unroll
-      for (int i = 0; i < S::kDK; ++i) {
-        o[i][0] *= a0;
-        o[i][1] *= a1;
-        o[i][2] *= a0;
-        o[i][3] *= a1;
-      }
-      // ---- O^T += V^T P^T
-      const bool ragged = valid < BLK;
-#pragma unroll
-      for (int kk = 0; kk < S::kKS; ++kk) {
-        const uint32_t b0 = pb[2 * kk], b1 = pb[2 * kk + 1];
-        const int k0 = tok_base + kk * 16;
-        const uint32_t mi = lane >> 3;
-        const uint32_t row = k0 + (lane & 7) + ((mi >> 1) << 3);
-        const int t_lo = k0 + 2 * tq;   // tokens of the fragment halves: t_lo, t_lo+1, t_lo+8, t_lo+9
-#pragma unroll
-        for (int i = 0; i < S::kDK; ++i) {
-          const uint32_t chunk = 2 * i + (mi & 1);
-          uint32_t v0, v1, v2, v3;
-          ldsm_x4_trans(vt + (chunk >> 3) * S::kBox + sw128(row, chunk & 7), v0, v1, v2, v3);
-          if (ragged) {
-            // rows past L may hold anything (even NaN): zero them so 0 * V stays 0
-            const uint32_t m01 = (t_lo < valid ? 0x0000ffffu : 0u) | (t_lo + 1 < valid ? 0xffff0000u : 0u);
-            const uint32_t m23 = (t_lo + 8 < valid ? 0x0000ffffu : 0u) | (t_lo + 9 < valid ? 0xffff0000u : 0u);
-            v0 &= m01;
-            v1 &= m01;
-            v2 &= m23;
-            v3 &= m23;
-          }
-          mma_bf16_16816(o[i], v0, v1, v2, v3, b0, b1);
-        }
-      }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
-    if (!(si_flags & kSegLast)) continue;
+    if (lane == 0) mbar_arrive(&qempty[seg & 1]);
+#pragma unroll
+    for (int i = 0; i < S::kDK; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;
+    const int L = slen[bh / p.Hkv];
+
+    for (int it = it0 + ((cg - it0 % NG) + NG) % NG; it < it1; it += NG) {
+      const int s = it % STAGES;
+      // every lane observes the phase (acquire); the warp leaves together if any lane gave up
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (it / STAGES) & 1))) {
+        alive = false;
+        break;
+      }
+      if (wg == 0 && lane == 0) observed[s] = observed[s] + 1;
+      const int si_n = info[s].n;
+      if (si_n >= 0) {
+        const uint32_t kt = smem_u32(ring + s * 2 * S::kTile);
+        const uint32_t vt = kt + S::kTile;
+        const int valid = min(BLK, L - si_n * BLK);
+        // ---- S = Q K^T for this warp's tokens (two accumulators per tile halve the mma chain)
+        float sacc[S::kNT][4];
+#pragma unroll
+        for (int j = 0; j < S::kNT; ++j) {
+          float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+          const uint32_t row = tok_base + j * 8 + (lane & 7);
+#pragma unroll
+          for (int kp = 0; kp < S::kDK / 2; ++kp) {
+            const uint32_t chunk = kp * 4 + (lane >> 3);
+            uint32_t r0, r1, r2, r3;
+            ldsm_x4(kt + (chunk >> 3) * S::kBox + sw128(row, chunk & 7), r0, r1, r2, r3);
+            if (kp & 1) {
+              mma_bf16_16816(sb, qa[2 * kp][0], 0u, qa[2 * kp][1], 0u, r0, r1);
+              mma_bf16_16816(sb, qa[2 * kp + 1][0], 0u, qa[2 * kp + 1][1], 0u, r2, r3);
+            } else {
+              mma_bf16_16816(sa, qa[2 * kp][0], 0u, qa[2 * kp][1], 0u, r0, r1);
+              mma_bf16_16816(sa, qa[2 * kp + 1][0], 0u, qa[2 * kp + 1][1], 0u, r2, r3);
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sacc[j][e] = sa[e] + sb[e];
+        }
+        // ---- online softmax (row = query head gq; this lane holds tokens 2tq, 2tq+1 of each tile)
+        float sv[S::kNT][2];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < S::kNT; ++j) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int tok = tok_base + j * 8 + 2 * tq + e;
+            const float v = tok < valid ? sacc[j][e] * sl2 : -INFINITY;
+            sv[j][e] = v;
+            mx = fmaxf(mx, v);
+          }
+        }
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        const float m_new = fmaxf(m_run, mx);
+        const float m_use = m_new == -INFINITY ? 0.f : m_new;
+        const float alpha = exp2f(m_run - m_use);
+        m_run = m_new;
+        uint32_t pb[S::kNT];
+        float ls = 0.f;
+#pragma unroll
+        for (int j = 0; j < S::kNT; ++j) {
+          pb[j] = pack_bf16(exp2f(sv[j][0] - m_use), exp2f(sv[j][1] - m_use));
+          ls += bf16_lo(pb[j]) + bf16_hi(pb[j]);
+        }
+        l_run = l_run * alpha + ls;
+        const float a0 = __shfl_sync(0xffffffffu, alpha, (2 * tq) * 4);
+        const float a1 = __shfl_sync(0xffffffffu, alpha, (2 * tq + 1) * 4);
+#pragma unroll
+        for (int i = 0; i < S::kDK; ++i) {
+          o[i][0] *= a0;
+          o[i][1] *= a1;
+          o[i][2] *= a0;
+          o[i][3] *= a1;
+        }
+        // ---- O^T += V^T P^T
+        const bool ragged = valid < BLK;
+#pragma unroll
+        for (int kk = 0; kk < S::kKS; ++kk) {
+          const uint32_t b0 = pb[2 * kk], b1 = pb[2 * kk + 1];
+          const int k0 = tok_base + kk * 16;
+          const uint32_t mi = lane >> 3;
+          const uint32_t row = k0 + (lane & 7) + ((mi >> 1) << 3);
+          const int t_lo = k0 + 2 * tq;   // tokens of the fragment halves: t_lo, t_lo+1, t_lo+8, t_lo+9
+#pragma unroll
+          for (int i = 0; i < S::kDK; ++i) {
+            const uint32_t chunk = 2 * i + (mi & 1);
+            uint32_t v0, v1, v2, v3;
+            ldsm_x4_trans(vt + (chunk >> 3) * S::kBox + sw128(row, chunk & 7), v0, v1, v2, v3);
+            if (ragged) {
+              // rows past L may hold anything (even NaN): zero them so 0 * V stays 0
+              const uint32_t m01 = (t_lo < valid ? 0x0000ffffu : 0u) | (t_lo + 1 < valid ? 0xffff0000u : 0u);
+              const uint32_t m23 = (t_lo + 8 < valid ? 0x0000ffffu : 0u) | (t_lo + 9 < valid ? 0xffff0000u : 0u);
+              v0 &= m01;
+              v1 &= m01;
+              v2 &= m23;
+              v3 &= m23;
+            }
+            mma_bf16_16816(o[i], v0, v1, v2, v3, b0, b1);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+    if (!__all_sync(0xffffffffu, alive)) {
+      alive = false;
+      break;
+    }
 
     // ================================================================ segment flush
-    const int bh = si_bh;
     const int b = bh / p.Hkv, h = bh - b * p.Hkv;
     const size_t qh0 = (size_t)b * p.Hq + (size_t)h * g;
-    int nseg, slot, slot_first, cf = 0;   // segments of this (b, h); this segment's partial slot; the first one's
-    if (p.flat) {
-      const long long W = sh[2], G = sh[3];
-      cf = cta_of(si_pre, W, G);
-      nseg = cta_of(si_pre + si_cnt - 1, W, G) - cf + 1;
-      slot = 2 * (int)blockIdx.x + (seg_start_it == 0 ? 0 : 1);
-      slot_first = 2 * cf + (range_lo(cf, W, G) != si_pre ? 1 : 0);
-    } else {
-      nseg = (si_cnt + p.per_split - 1) / p.per_split;
-      slot = bh * p.ns + (int)blockIdx.x;
-      slot_first = bh * p.ns;
+    const bool first_seg = it0 == 0, last_seg = it1 == nit;
+    if ((first_seg || last_seg) && !sh[17]) {
+      // the epilogue warp publishes the split bookkeeping long before the first flush; wait if not
+      const long long t0 = clock64();
+      while (!sh[17] && clock64() - t0 < kWaitLimitCycles) {
+      }
+      if (!__all_sync(0xffffffffu, sh[17] != 0)) {
+        alive = false;
+        break;
+      }
     }
-    float* Ow = merge + (nflush & 1) * (S::kMergeOne / 4);
-    float* Mw = Ow + NW * kMaxGroup * D;
-    float* Lw = Mw + NW * kMaxGroup;
-    ++nflush;
+    __threadfence_block();
+    int nseg, slot_first, cf;   // pieces of this (b, h); the first piece's slot and CTA
+    if (first_seg) {
+      cf = sh[10];
+      nseg = sh[11];
+      slot_first = sh[12];
+    } else if (last_seg) {
+      cf = sh[13];
+      nseg = sh[14];
+      slot_first = sh[15];
+    } else {
+      cf = 0;
+      nseg = 1;
+      slot_first = 0;
+    }
+    const int slot = p.flat ? 2 * (int)blockIdx.x + (first_seg ? 0 : 1) : bh * p.ns + (int)blockIdx.x;
+    // 1. each warp's state -> shared memory
     float lw = l_run;
     lw += __shfl_xor_sync(0xffffffffu, lw, 1);
     lw += __shfl_xor_sync(0xffffffffu, lw, 2);
@@ -639,36 +722,49 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NW, STAGES>::kThreads)
       alive = false;
       break;
     }
-    for (int e = tid; e < g * D; e += NW * 32) {
-      const int j = e / D, cc = e % D;
+    // 2. per-head merge weights of the CW warp states, and the segment's LSE
+    if (tid < CW * g) {
+      const int w = tid / g, j = tid - (tid / g) * g;
       float M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < NW; ++w) M = fmaxf(M, Mw[w * kMaxGroup + j]);
-      float num = 0.f, den = 0.f;
+      for (int w2 = 0; w2 < CW; ++w2) M = fmaxf(M, Mw[w2 * kMaxGroup + j]);
+      float den = 0.f;
       if (M != -INFINITY) {
 #pragma unroll
-        for (int w = 0; w < NW; ++w) {
-          const float sc = exp2f(Mw[w * kMaxGroup + j] - M);
-          num += sc * Ow[(w * kMaxGroup + j) * D + cc];
-          den += sc * Lw[w * kMaxGroup + j];
+        for (int w2 = 0; w2 < CW; ++w2) den += exp2f(Mw[w2 * kMaxGroup + j] - M) * Lw[w2 * kMaxGroup + j];
+      }
+      Wt[w * kMaxGroup + j] = den > 0.f ? exp2f(Mw[w * kMaxGroup + j] - M) / den : 0.f;
+      if (w == 0) Hs[j] = den > 0.f ? (M + log2f(den)) * kLn2 : -INFINITY;
+    }
+    if (!warps_sync(cbar, cphase)) {
+      alive = false;
+      break;
+    }
+    // 3. combine: each output element is CW independent multiply-adds
+    constexpr int EPT = (kMaxGroup * D + CW * 32 - 1) / (CW * 32);
+#pragma unroll
+    for (int u = 0; u < EPT; ++u) {
+      const int e = u * CW * 32 + tid;
+      if (e < g * D) {
+        const int j = e / D, cc = e - j * D;
+        float val = 0.f;
+#pragma unroll
+        for (int w = 0; w < CW; ++w) val += Wt[w * kMaxGroup + j] * Ow[(w * kMaxGroup + j) * D + cc];
+        if (nseg <= 1) {
+          __nv_bfloat16 ob = __float2bfloat16_rn(val);
+          p.out[(qh0 + j) * D + cc] = *reinterpret_cast<uint16_t*>(&ob);
+          if (cc == 0 && p.lse_out) p.lse_out[qh0 + j] = Hs[j];
+        } else {
+          p.o_part[((size_t)slot * g + j) * D + cc] = val;
+          if (cc == 0) p.lse_part[(size_t)slot * g + j] = Hs[j];
         }
       }
-      const bool any = den > 0.f;
-      const float oval = any ? num / den : 0.f;
-      const float lse = any ? (M + log2f(den)) * kLn2 : -INFINITY;
-      if (nseg <= 1) {
-        __nv_bfloat16 ob = __float2bfloat16_rn(oval);
-        p.out[(qh0 + j) * D + cc] = *reinterpret_cast<uint16_t*>(&ob);
-        if (cc == 0 && p.lse_out) p.lse_out[qh0 + j] = lse;
-      } else {
-        p.o_part[((size_t)slot * g + j) * D + cc] = oval;
-        if (cc == 0) p.lse_part[(size_t)slot * g + j] = lse;
-      }
     }
-    if (nseg > 1 && it != nit - 1) {   // a split first segment: the epilogue warp publishes / merges it
+    if (nseg > 1 && !last_seg) {
+      // the CTA's split first segment: the epilogue warp publishes / merges it
       if (tid == 0) job[0] = Job{bh, nseg, slot_first, cf};
       __syncwarp();
-      if (lane == 0) mbar_arrive(&jbar[0]);
+      if (lane == 0) mbar_arrive(jbar);
     } else if (nseg > 1) {
       // the CTA's last segment: publish it and, if it arrived last, merge the (b, h) right here
       if (!warps_sync(cbar, cphase)) {
@@ -681,75 +777,37 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NW, STAGES>::kThreads)
         break;
       }
       if (sh[1]) {
-        constexpr int EPC = (kMaxGroup * D + NW * 32 - 1) / (NW * 32);   // outputs per thread
-        constexpr int MAXS = 4;                                           // segments merged from registers
-        if (nseg <= MAXS) {
-          float lv[MAXS][EPC], ov[MAXS][EPC];
-#pragma unroll
-          for (int s2 = 0; s2 < MAXS; ++s2) {
-            const size_t sl = (size_t)split_slot(p, bh, s2 < nseg ? s2 : 0, slot_first, cf);
-#pragma unroll
-            for (int t = 0; t < EPC; ++t) {
-              const int e = tid + t * NW * 32;
-              const int j = e / D;
-              const bool on = s2 < nseg && e < g * D;
-              lv[s2][t] = on ? __ldcg(p.lse_part + sl * g + j) : -INFINITY;
-              ov[s2][t] = on ? __ldcg(p.o_part + (sl * g + j) * D + (e - j * D)) : 0.f;
-            }
-          }
-#pragma unroll
-          for (int t = 0; t < EPC; ++t) {
-            const int e = tid + t * NW * 32;
-            if (e >= g * D) continue;
-            const int j = e / D, cc = e - j * D;
-            float M = -INFINITY;
-#pragma unroll
-            for (int s2 = 0; s2 < MAXS; ++s2) M = fmaxf(M, lv[s2][t]);
-            float num = 0.f, den = 0.f;
-            if (M != -INFINITY) {
-#pragma unroll
-              for (int s2 = 0; s2 < MAXS; ++s2) {
-                const float w = s2 < nseg ? expf(lv[s2][t] - M) : 0.f;
-                num += w * ov[s2][t];
-                den += w;
-              }
-            }
-            const bool any = den > 0.f;
-            __nv_bfloat16 ob = __float2bfloat16_rn(any ? num / den : 0.f);
-            p.out[(qh0 + j) * D + cc] = *reinterpret_cast<uint16_t*>(&ob);
-            if (cc == 0 && p.lse_out) p.lse_out[qh0 + j] = any ? M + logf(den) : -INFINITY;
-          }
-        } else {
-          for (int e = tid; e < g * D; e += NW * 32) {
-            const int j = e / D, cc = e % D;
-            float M = -INFINITY;
-            for (int s2 = 0; s2 < nseg; ++s2)
-              M = fmaxf(M, __ldcg(p.lse_part + (size_t)split_slot(p, bh, s2, slot_first, cf) * g + j));
-            float num = 0.f, den = 0.f;
-            if (M != -INFINITY) {
-              for (int s2 = 0; s2 < nseg; ++s2) {
-                const size_t sl = (size_t)split_slot(p, bh, s2, slot_first, cf);
-                const float w = expf(__ldcg(p.lse_part + sl * g + j) - M);
-                num += w * __ldcg(p.o_part + (sl * g + j) * D + cc);
-                den += w;
-              }
-            }
-            const bool any = den > 0.f;
-            __nv_bfloat16 ob = __float2bfloat16_rn(any ? num / den : 0.f);
-            p.out[(qh0 + j) * D + cc] = *reinterpret_cast<uint16_t*>(&ob);
-            if (cc == 0 && p.lse_out) p.lse_out[qh0 + j] = any ? M + logf(den) : -INFINITY;
-          }
+        bool ok = true;
+        // scratch: the merge area (every warp has finished reading it) -- `epi` belongs to the epilogue warp
+        merge_partials<D, CW * 32, S::kEpi>(p, bh, nseg, slot_first, cf, tid, Ow, [&] {
+          ok = warps_sync(cbar, cphase) && ok;
+        });
+        if (!ok) {
+          alive = false;
+          break;
         }
         if (tid == 0) p.counters[bh] = 0;
       }
+    }
+    it0 = it1;
+    ++seg;
+    // the merge area is rewritten by the next segment's flush
+    if (it0 < nit && !warps_sync(cbar, cphase)) {
+      alive = false;
+      break;
     }
   }
   if (!alive) {
     if (lane == 0) report(p.err, SEER_DEVERR_TIMEOUT);
     sh[0] = 1;
     // drain the copies still in flight (bounded) before the CTA's shared memory is released
-    if (warp == 0 && lane == 0)
-      for (int it = consumed; it < nit && it < consumed + STAGES; ++it) mbar_wait(&full[it % STAGES], (it / STAGES) & 1);
+    if (warp == 0 && lane == 0) {
+      const long long t0 = clock64();
+      while (!sh[9] && clock64() - t0 < kWaitLimitCycles) {
+      }
+      for (int s = 0; s < STAGES; ++s)
+        if (issued[s] > observed[s]) mbar_wait(&full[s], observed[s] & 1);
+    }
     return;
   }
 
@@ -760,36 +818,38 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NW, STAGES>::kThreads)
     if (clamp_cnt(p, bh) != 0) continue;
     const int b = bh / p.Hkv, h = bh - b * p.Hkv;
     const size_t qh0 = (size_t)b * p.Hq + (size_t)h * g;
-    for (int e = tid; e < g * D; e += NW * 32) {
+    for (int e = tid; e < g * D; e += CW * 32) {
       p.out[qh0 * D + e] = 0;
       if (e < g && p.lse_out) p.lse_out[qh0 + e] = -INFINITY;
     }
   }
 }
 
-// ring depth per shape (stage = 2 * BLK * D * 2 bytes; one CTA per SM)
+// ring depth and consumer groups per shape (stage = 2 * BLK * D * 2 bytes; one CTA per SM)
 #ifndef SEER_DECODE_STAGES_128_64
 #define SEER_DECODE_STAGES_128_64 4
 #endif
 template <int D, int BLK>
 struct Choice;
-template <> struct Choice<64, 64> { static constexpr int NW = 4, ST = 6; };
-template <> struct Choice<64, 128> { static constexpr int NW = 4, ST = 4; };
-template <> struct Choice<128, 64> { static constexpr int NW = 4, ST = SEER_DECODE_STAGES_128_64; };
-template <> struct Choice<128, 128> { static constexpr int NW = 4, ST = 2; };
+template <> struct Choice<64, 64> { static constexpr int NWG = 4, NG = 2, ST = 6; };
+template <> struct Choice<64, 128> { static constexpr int NWG = 4, NG = 2, ST = 4; };
+template <> struct Choice<128, 64> { static constexpr int NWG = 4, NG = 2, ST = SEER_DECODE_STAGES_128_64; };
+template <> struct Choice<128, 128> { static constexpr int NWG = 4, NG = 2, ST = 2; };
+
+template <int D, int BLK>
+using ShapeOf = DecodeShape<D, BLK, Choice<D, BLK>::NWG, Choice<D, BLK>::NG, Choice<D, BLK>::ST>;
 
 template <int D, int BLK>
 size_t smem_bytes(int B, int BH) {
-  using C = Choice<D, BLK>;
-  return DecodeShape<D, BLK, C::NW, C::ST>::kSmemFixed + (size_t)(B + BH + 1 + 8) * 4;
+  return ShapeOf<D, BLK>::kSmemFixed + (size_t)(B + BH + 1 + 16) * 4;
 }
 
 template <int D, int BLK>
 cudaError_t launch_t(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p, int grid_flat,
                      cudaStream_t st) {
-  constexpr int NW = Choice<D, BLK>::NW, ST = Choice<D, BLK>::ST;
-  using Sh = DecodeShape<D, BLK, NW, ST>;
-  auto kern = sparse_decode_kernel<D, BLK, NW, ST>;
+  using C = Choice<D, BLK>;
+  using Sh = ShapeOf<D, BLK>;
+  auto kern = sparse_decode_kernel<D, BLK, C::NWG, C::NG, C::ST>;
   static std::atomic<uint64_t> attr_done{0};
   cudaError_t e = ensure_smem_limit(kern, (int)smem_bytes<D, BLK>(kMaxDecodeB, kMaxDecodeBH), attr_done);
   if (e != cudaSuccess) return e;
@@ -800,9 +860,9 @@ cudaError_t launch_t(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeP
 
 template <int D, int BLK>
 int ctas_per_sm_t() {
-  constexpr int NW = Choice<D, BLK>::NW, ST = Choice<D, BLK>::ST;
-  using Sh = DecodeShape<D, BLK, NW, ST>;
-  auto kern = sparse_decode_kernel<D, BLK, NW, ST>;
+  using C = Choice<D, BLK>;
+  using Sh = ShapeOf<D, BLK>;
+  auto kern = sparse_decode_kernel<D, BLK, C::NWG, C::NG, C::ST>;
   static std::atomic<uint64_t> attr_done{0};
   const int smax = (int)smem_bytes<D, BLK>(kMaxDecodeB, kMaxDecodeBH);
   if (ensure_smem_limit(kern, smax, attr_done) != cudaSuccess) return 1;
