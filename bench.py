@@ -69,6 +69,22 @@ def _dist():
     return world, rank, local
 
 
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank decodes its own batch (weak scaling): a distinct seed per rank."""
+    return base_seed + 7919 * rank
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The slowest rank's time: every rank takes part in the same all-reduce."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def _peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -76,6 +92,23 @@ def _peaks():
         return float(p["hbm_gbs"]), "measured"
     except Exception:
         return 6650.0, "fallback"
+
+
+def _profiled_traffic():
+    """DRAM bytes (read + write) per launch of the decode kernel from the committed ncu summary,
+    or None when the kernel source has changed since those counters were taken."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "sparse_decode_kernel.qwen3-8b-32k-decode.md")) as f:
+            fields = dict(line.split(": ", 1) for line in f.read().splitlines() if ": " in line
+                          and line.split(": ", 1)[0] in ("source_sha256", "traffic_bytes_per_launch"))
+        with open(os.path.join(ROOT, "block_sparse_attention_attngate_b200", "csrc", "sparse_decode.cu"), "rb") as f:
+            current = hashlib.sha256(f.read()).hexdigest()
+        if fields.get("source_sha256", "").strip() != current:
+            return None
+        return int(fields["traffic_bytes_per_launch"])
+    except Exception:
+        return None
 
 
 class ClockSampler:
@@ -230,7 +263,7 @@ def run_seer(args):
     from synthetic import config, make_inputs
 
     cfg = config(WORKLOAD["cid"], **({"budget": args.budget} if args.budget else {}))
-    cfg = config(WORKLOAD["cid"], seed=cfg.seed + 7919 * rank, **({"budget": args.budget} if args.budget else {}))
+    cfg = config(WORKLOAD["cid"], seed=rank_seed(cfg.seed, rank), **({"budget": args.budget} if args.budget else {}))
     inp = make_inputs(cfg)
     B, Hq, Hkv, d, dg, blk = cfg.B, cfg.Hq, cfg.Hkv, cfg.head_dim, cfg.gate_dim, cfg.block
     NB = inp.max_blocks
@@ -288,12 +321,8 @@ def run_seer(args):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def ranks_max(x: float) -> float:
+        return max_over_ranks(x, world, dev)
 
     def timed(fn, n):
         with torch.cuda.stream(stream):
@@ -319,11 +348,11 @@ def run_seer(args):
         time.sleep(0.3)
         ms_step = timed(lambda i: graphs[i % R].replay(), args.steps)
     clocks = clk.summary()
-    ms_step = max_over_ranks(ms_step)
+    ms_step = ranks_max(ms_step)
 
     # ---------------- per-part device times (eager launches, same replica rotation)
     def part(fn):
-        return max_over_ranks(timed(fn, args.steps)) * 1e3
+        return ranks_max(timed(fn, args.steps)) * 1e3
 
     def run_decode(i):
         st = reps[i % R]["step"]
@@ -399,7 +428,7 @@ def run_seer(args):
         o = rp["step"].run(rp["q"], seqlens, stream=stream)
         out_host.copy_(o.view(torch.int16).view(-1), non_blocking=True)
 
-    e2e_ms = max_over_ranks(timed(e2e, args.steps))
+    e2e_ms = ranks_max(timed(e2e, args.steps))
     h2d = B * Hq * d * 2
     d2h = B * Hq * d * 2
 
@@ -436,7 +465,8 @@ def run_seer(args):
         "bytes": {"decode_algorithmic": nbytes["decode"], "step_algorithmic": nbytes["step"]},
         "step_gbs": step_gbs,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": None, "kernel": "sparse_decode_kernel", "peak_kind": peak_kind},
+                     "traffic": _profiled_traffic(), "traffic_unit": "bytes per launch (ncu dram read+write)",
+                     "kernel": "sparse_decode_kernel", "peak_kind": peak_kind},
         "e2e": {"value": e2e_ms * 1e3, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
