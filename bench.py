@@ -50,7 +50,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="seer", choices=["seer", "reference"])
-    ap.add_argument("--num-split", type=int, default=0)
+    ap.add_argument("--num-split", type=int, default=None,
+                    help="decode schedule: -1 capacity, 0 balanced, >= 1 the pages' grid (default: the step's own)")
     ap.add_argument("--replicas", type=int, default=3)
     ap.add_argument("--budget", type=int, default=0, help="override the token budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -399,7 +400,7 @@ def run_seer(args):
     # ---------------- dense path: every block of every (b, h), same kernel
     dense_idx = torch.arange(NB, dtype=torch.int32, device=dev).expand(B, Hkv, NB).contiguous()
     dense_cnt = torch.full((B, Hkv), NB, dtype=torch.int32, device=dev)
-    dense_ns = args.num_split
+    dense_ns = reps[0]["step"].num_split   # the dense lists sit at their capacity too
     dense_ws = S.alloc_workspace(shape, NB, dense_ns, dev)
     dense_out = torch.empty(B, Hq, d, dtype=torch.bfloat16, device=dev)
 

@@ -16,16 +16,29 @@ constexpr int kCL = SEER_GATE_CLUSTER;
 template <int D, int DG>
 __global__ void __cluster_dims__(kCL, 1, 1) __launch_bounds__(kThreads) gate_score_kernel(const GateParams p) {
   __shared__ GateSmem<D, DG, kCL> sm;
+  __shared__ uint64_t wq_bar;
+  extern __shared__ uint4 wq_raw[];   // this CTA's W_q rows
+  uint16_t* wq_s = reinterpret_cast<uint16_t*>(wq_raw);
   cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int b = blockIdx.z, h = blockIdx.y;
+  if (threadIdx.x == 0) gate_prefetch_wq<D, DG, kCL>(p, h, rank, &wq_bar, wq_s);   // weights: no wait needed
   pdl_wait();
   pdl_trigger();
-  gate_cluster<D, DG, kCL, kThreads>(p, blockIdx.z, blockIdx.y, (int)cluster.block_rank(), cluster, sm, nullptr);
+  GateQuery<D, DG, kCL, kThreads> q;
+  q.load(p, b, h);
+  const int L = max(p.seqlens[b], 0);
+  gate_cluster<D, DG, kCL, kThreads>(p, b, h, rank, L, q, cluster, sm, &wq_bar, wq_s, nullptr);
 }
 
 template <int D, int DG>
 cudaError_t launch_t(const GateParams& p, cudaStream_t s) {
+  auto kern = gate_score_kernel<D, DG>;
+  static std::atomic<uint64_t> attr_done{0};
+  cudaError_t e = ensure_smem_limit(kern, (int)gate_wq_bytes<D, DG, kCL>(kMaxGroup), attr_done);
+  if (e != cudaSuccess) return e;
   dim3 grid(kCL, p.Hkv, p.B);
-  return launch_pdl(gate_score_kernel<D, DG>, grid, dim3(kThreads), 0, s, p);
+  return launch_pdl(kern, grid, dim3(kThreads), gate_wq_bytes<D, DG, kCL>(p.g), s, p);
 }
 
 }  // namespace

@@ -1,6 +1,7 @@
 // C ABI of libseer (declared in include/seer.h): argument validation, TMA
 // descriptor encoding (cached), launch-shape choices and kernel launches.
 // Nothing here allocates device memory or synchronises the host.
+#include <cstdint>
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
@@ -284,10 +285,11 @@ int flat_grid(const seer_dims_t* d, DevFacts* df) { return df->sms * decode_occ(
 // CTA (a CTA's first and last segment are the only ones that can belong to a (b, h) split
 // across CTAs).  Grid schedule: num_split slots per (b, h).
 size_t ws_layout(const seer_dims_t* d, int32_t ns, int flat_ctas, size_t* off_lse, size_t* off_o) {
+  // ns <= 0: one of the one-wave schedules (balanced or capacity), 2 slots per CTA
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
   const size_t g = (size_t)(d->num_q_heads / d->num_kv_heads);
   const size_t bh = (size_t)d->batch * d->num_kv_heads;
-  const size_t slots = ns == 0 ? 2 * (size_t)flat_ctas : bh * ns;
+  const size_t slots = ns <= 0 ? 2 * (size_t)flat_ctas : bh * ns;
   const size_t rec = up(bh * 4);
   const size_t lse = up(slots * g * 4);
   const size_t o = slots * g * d->head_dim * 4;
@@ -470,10 +472,10 @@ int32_t seer_sparse_decode_auto_split(const seer_dims_t* dims, int32_t capacity)
 }
 
 size_t seer_sparse_decode_workspace_bytes(const seer_dims_t* dims, int32_t capacity, int32_t num_split) {
-  if (check_dims(dims) != SEER_OK || capacity < 1 || num_split < 0) return 0;
+  if (check_dims(dims) != SEER_OK || capacity < 1 || num_split < -1) return 0;
   const int32_t ns = num_split > capacity ? capacity : num_split;
   int ctas = 0;
-  if (ns == 0) {
+  if (ns <= 0) {
     int dev;
     DevFacts* df;
     if (device_facts(&dev, &df) != SEER_OK) return 0;
@@ -494,16 +496,18 @@ seer_status seer_sparse_decode(const seer_dims_t* dims, const void* q, const see
   if (!q || !block_idx || !block_cnt || !seqlens || !out) return fail(SEER_ERR_INVALID_ARG, "NULL pointer argument");
   if (!aligned16(q) || !aligned16(out)) return fail(SEER_ERR_INVALID_ARG, "q / out not 16-byte aligned");
   if (capacity < 1) return fail(SEER_ERR_INVALID_ARG, "capacity must be >= 1");
-  if (num_split < 0) return fail(SEER_ERR_INVALID_ARG, "num_split must be >= 0");
+  if (num_split < -1) return fail(SEER_ERR_INVALID_ARG, "num_split must be >= -1");
   int dev;
   DevFacts* df;
   if ((st = device_facts(&dev, &df)) != SEER_OK) return st;
   if (dims->batch > seer::kMaxDecodeB) return fail(SEER_ERR_UNSUPPORTED, "batch %d > %d", dims->batch, seer::kMaxDecodeB);
   int32_t ns = num_split > capacity ? capacity : num_split;
-  if (ns == 0 && dims->batch * dims->num_kv_heads > seer::kMaxDecodeBH)
-    return fail(SEER_ERR_UNSUPPORTED, "balanced schedule needs batch*num_kv_heads <= %d; pass num_split >= 1",
+  if (ns <= 0 && dims->batch * dims->num_kv_heads > seer::kMaxDecodeBH)
+    return fail(SEER_ERR_UNSUPPORTED, "one-wave schedules need batch*num_kv_heads <= %d; pass num_split >= 1",
                 seer::kMaxDecodeBH);
-  const int ctas = ns == 0 ? flat_grid(dims, df) : 0;
+  if (ns == -1 && (int64_t)dims->batch * dims->num_kv_heads * capacity > INT32_MAX / 2)
+    return fail(SEER_ERR_UNSUPPORTED, "capacity schedule: batch*num_kv_heads*capacity too large");
+  const int ctas = ns <= 0 ? flat_grid(dims, df) : 0;
   size_t off_lse, off_o;
   const size_t need = ws_layout(dims, ns, ctas, &off_lse, &off_o);
   if (need > 0) {
@@ -533,9 +537,9 @@ seer_status seer_sparse_decode(const seer_dims_t* dims, const void* q, const see
   p.Hkv = dims->num_kv_heads;
   p.g = dims->num_q_heads / dims->num_kv_heads;
   p.cap = capacity;
-  p.flat = ns == 0;
-  p.ns = ns;
-  p.per_split = ns ? (capacity + ns - 1) / ns : capacity;
+  p.flat = ns == 0 ? 1 : (ns == -1 ? 2 : 0);
+  p.ns = ns > 0 ? ns : 0;
+  p.per_split = ns > 0 ? (capacity + ns - 1) / ns : capacity;
   const float scale = dims->softmax_scale > 0.f ? dims->softmax_scale : 1.0f / sqrtf((float)dims->head_dim);
   p.scale_log2 = scale * 1.4426950408889634f;
   uint8_t* ws = static_cast<uint8_t*>(workspace);

@@ -126,7 +126,8 @@ struct DecodeParams {
   int32_t k_paged, v_paged;
   int32_t k_perm[3], v_perm[3];   // TMA dim (1..3) that holds token / head / batch-or-page
   int32_t B, Hq, Hkv, g;
-  int32_t flat;             // 1: balanced ranges over a persistent grid; 0: (split, kv head, batch) grid
+  int32_t flat;             // 0: (split, kv head, batch) grid; one-wave ranges over 1: the concatenated
+                            // lists (balanced), 2: every list padded to its capacity (capacity schedule)
   int32_t cap, ns, per_split;
   float scale_log2;         // softmax scale * log2(e)
   float* o_part;            // [B, Hq, ns, D]

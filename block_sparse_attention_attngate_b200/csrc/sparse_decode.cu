@@ -253,6 +253,7 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
   const int tid = threadIdx.x;
   const int BH = p.B * p.Hkv;
   const int g = p.g;
+  auto seq_len = [&](int b) { return p.flat == 2 ? max(__ldg(p.seqlens + b), 0) : slen[b]; };
   if (tid == 0) {
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
@@ -276,8 +277,15 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
   pdl_trigger();
 
   // ---------------------------------------------------------------- lengths, list prefix, this CTA's range
-  for (int i = tid; i < p.B; i += S::kThreads) slen[i] = max(p.seqlens[i], 0);
-  if (p.flat) {
+  // (the capacity schedule reads nothing here: its prefix is bh * capacity, and the lengths are
+  // read where they are used)
+  if (p.flat != 2)
+    for (int i = tid; i < p.B; i += S::kThreads) slen[i] = max(p.seqlens[i], 0);
+  if (p.flat == 2) {
+    for (int i = tid; i <= BH; i += S::kThreads) pre[i] = i * p.cap;
+    __syncthreads();
+  }
+  if (p.flat == 1) {
     // each thread sums a contiguous run of counts, then one block-wide exclusive scan
     const int per_t = (BH + S::kThreads - 1) / S::kThreads;
     const int base = tid * per_t;
@@ -312,6 +320,8 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
     }
     if (tid == S::kThreads - 1) pre[BH] = before + incl;
     __syncthreads();
+  }
+  if (p.flat) {
     if (tid == 0) {
       const int W = pre[BH];
       const long long G = min((long long)gridDim.x, (long long)max(W, 1));
@@ -418,7 +428,12 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
       }
       first = (it == 0 || pos == 0) ? kSegFirst : 0;
       const int b = bh / p.Hkv;
-      const int nblk = (slen[b] + BLK - 1) / BLK;
+      if (p.flat == 2) {   // list positions past the count are padding
+        const int c = p.cnt[bh];
+        if (pos == 0 && c > p.cap) report(p.err, SEER_DEVERR_COUNT);
+        if (pos >= c) return;
+      }
+      const int nblk = (seq_len(b) + BLK - 1) / BLK;
       const int blk = p.idx[(size_t)bh * p.cap + pos];
       bool ok = blk >= 0 && blk < nblk;
       if (!ok) report(p.err, SEER_DEVERR_BLOCK_INDEX);
@@ -558,7 +573,7 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
 #pragma unroll
     for (int i = 0; i < S::kDK; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
     float m_run = -INFINITY, l_run = 0.f;
-    const int L = slen[bh / p.Hkv];
+    const int L = seq_len(bh / p.Hkv);
 
     for (int it = it0 + ((cg - it0 % NG) + NG) % NG; it < it1; it += NG) {
       const int s = it % STAGES;
@@ -811,7 +826,9 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
     return;
   }
 
-  // (b, h) pairs with an empty list: zeros and lse = -inf
+  // (b, h) pairs with an empty list: zeros and lse = -inf (the capacity schedule's ranges cover
+  // every (b, h), so an empty list already came out that way)
+  if (p.flat == 2) return;
   const int first_bh = p.flat ? (int)blockIdx.x : (blockIdx.x == 0 ? (int)(blockIdx.z * p.Hkv + blockIdx.y) : BH);
   const int step_bh = p.flat ? (int)gridDim.x : BH;
   for (int bh = first_bh; bh < BH; bh += step_bh) {

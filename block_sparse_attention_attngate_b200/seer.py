@@ -287,7 +287,8 @@ class DecodeStep:
 
     def __init__(self, shape: Shape, k: KVCache, v: KVCache, w_q: torch.Tensor, w_k: torch.Tensor,
                  kcomp: torch.Tensor, valid_blocks: torch.Tensor, mode: int = SELECT_TOPK, token_budget: int = 0,
-                 tau: float = 0.0, capacity: Optional[int] = None, num_split: int = 0, k_nope: Optional[KVCache] = None,
+                 tau: float = 0.0, capacity: Optional[int] = None, num_split: Optional[int] = None,
+                 k_nope: Optional[KVCache] = None,
                  device=None):
         dev = device or w_q.device
         self.shape, self.k, self.v, self.w_q, self.w_k = shape, k, v, w_q, w_k
@@ -304,7 +305,11 @@ class DecodeStep:
         self.logits = torch.empty(B, Hkv, shape.max_blocks, dtype=torch.float32, device=dev)
         self.block_idx = torch.empty(B, Hkv, capacity, dtype=torch.int32, device=dev)
         self.block_cnt = torch.empty(B, Hkv, dtype=torch.int32, device=dev)
-        self.num_split = num_split    # 0 = the balanced schedule
+        if num_split is None:
+            # top-k lists sit at (or near) their capacity: the capacity schedule needs no scan of
+            # the counts; other modes use the balanced schedule
+            num_split = -1 if mode == SELECT_TOPK else 0
+        self.num_split = num_split    # -1 capacity, 0 balanced, >= 1 the pages' grid
         self.workspace = alloc_workspace(shape, capacity, self.num_split, dev)
         self.out = torch.empty(B, Hq, shape.head_dim, dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)

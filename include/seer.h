@@ -186,14 +186,14 @@ seer_status seer_decode_plan(const seer_dims_t* dims, const seer_kv_t* k_nope, c
 
 /*
  * A split count for the pages' (num_split, Hkv, B) grid that fills one wave of the SMs (host
- * heuristic, no device reads).  seer_sparse_decode uses its own balanced schedule when given
- * num_split == 0; pass this value to get the grid schedule instead.
+ * heuristic, no device reads).  seer_sparse_decode uses its own one-wave schedules when given
+ * num_split == 0 or -1; pass this value to get the grid schedule instead.
  */
 int32_t seer_sparse_decode_auto_split(const seer_dims_t* dims, int32_t capacity);
 
 /*
  * Workspace bytes seer_sparse_decode needs for `num_split`: one arrival counter per (b, h) plus
- * fp32 partial outputs and LSEs -- 2 slots per CTA of the balanced schedule (num_split == 0),
+ * fp32 partial outputs and LSEs -- 2 slots per CTA of the one-wave schedules (num_split 0, -1),
  * num_split slots per (b, h) for the grid schedule, none for num_split == 1.  The counters must
  * be zero before the first call (e.g. allocate zero-filled); every completed call leaves them
  * zero again.
@@ -215,13 +215,18 @@ size_t seer_sparse_decode_workspace_bytes(const seer_dims_t* dims, int32_t capac
  *     max_selected_blocks, not from the sequence length).
  *   num_split == 0: balanced -- the concatenation of all lists is cut into equal contiguous
  *     ranges, one per CTA of a grid with one CTA per SM slot.
- * In both, a (b, h) computed by several CTAs is merged (LSE combine) by the last of them.
+ *   num_split == -1: capacity -- as balanced, but every list counts as `capacity` positions
+ *     (those at or past block_cnt are skipped), so the ranges need no scan of the counts and the
+ *     first tiles are requested one round trip after the launch's inputs are ready.  Best when
+ *     the counts are at or near the capacity (top-k with a fixed budget); with short lists the
+ *     skipped positions leave CTAs idle.  Requires batch*Hkv*capacity < 2^30.
+ * In all, a (b, h) computed by several CTAs is merged (LSE combine) by the last of them.
  *
  *   q          device bf16 [B, Hq, d]  (post-RoPE query, as the model uses it)
  *   k, v       K and V caches (see seer_kv_t)
  *   block_idx  device int32 [B, Hkv, capacity]; block_cnt device int32 [B, Hkv]
  *   seqlens    device int32 [B]
- *   num_split  0 = balanced schedule, >= 1 = grid schedule; must match the workspace size
+ *   num_split  0 = balanced, -1 = capacity, >= 1 = grid schedule; must match the workspace size
  *   workspace  device, >= seer_sparse_decode_workspace_bytes(dims, capacity, num_split) bytes
  *   out        device bf16 [B, Hq, d]
  *   lse_out    device fp32 [B, Hq] or NULL

@@ -141,7 +141,8 @@ def test_decode_validation(lib, S):
     assert _decode(lib, S, d, _kv(S, layout=1), good) == 1         # paged without a block table
     assert _decode(lib, S, d, _kv(S, layout=3), good) == 1
     assert _decode(lib, S, d, good, good, q=ctypes.c_void_p(4098)) == 1
-    assert _decode(lib, S, d, good, good, ns=-1) == 1
+    assert _decode(lib, S, d, good, good, ns=-2) == 1
+    assert b"num_split" in lib.seer_last_error()
     # a well-formed call reaches the CUDA runtime; without a GPU it reports a CUDA error, not a crash
     st = _decode(lib, S, d, good, good)
     assert st in (0, 4)
@@ -154,6 +155,7 @@ def test_workspace_formula(lib, S):
         up = lambda x: (x + 255) // 256 * 256
         assert n == up(8 * 8 * 4) + up(8 * 32 * ns * 4) + 8 * 32 * ns * 128 * 4
     assert lib.seer_sparse_decode_workspace_bytes(ctypes.byref(d), 65, 1) == 0
+    assert lib.seer_sparse_decode_workspace_bytes(ctypes.byref(d), 65, -2) == 0
     bad = _dims(S, head_dim=80)
     assert lib.seer_sparse_decode_workspace_bytes(ctypes.byref(bad), 65, 2) == 0
 

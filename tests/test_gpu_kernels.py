@@ -179,7 +179,7 @@ def test_kcomp_incremental_freeze_and_rebuild():
 # ------------------------------------------------------------------ sparse decode on oracle block lists
 
 @pytest.mark.parametrize("d,blk,g", [(128, 64, 4), (128, 128, 5), (64, 64, 8), (64, 128, 1), (128, 64, 2)])
-@pytest.mark.parametrize("ns", [1, 2, 3, 0])
+@pytest.mark.parametrize("ns", [1, 2, 3, 0, -1])
 def test_sparse_decode_vs_oracle(d, blk, g, ns):
     Hkv = 2
     cfg = config(1, B=3, Hq=g * Hkv, Hkv=Hkv, head_dim=d, gate_dim=64, block=blk, seed=900 + d + blk + g)
@@ -210,10 +210,11 @@ def test_sparse_decode_vs_oracle(d, blk, g, ns):
             check_lse(lh[b, h * g:(h + 1) * g], rl, f"b{b} h{h}")
 
 
-@pytest.mark.parametrize("ns", [0, 3])
+@pytest.mark.parametrize("ns", [0, 3, -1])
 def test_sparse_decode_many_short_lists(ns):
     """Many (b, h) pairs with short lists: the balanced schedule packs several whole lists into
-    one CTA range and splits others across CTAs; the grid schedule leaves most splits empty."""
+    one CTA range and splits others across CTAs; the grid schedule leaves most splits empty; the
+    capacity schedule skips every position past a list's count (an empty list included)."""
     blk, d, g, Hkv = 64, 128, 4, 8
     cfg = config(1, B=32, Hq=g * Hkv, Hkv=Hkv, head_dim=d, gate_dim=64, block=blk, seed=4242)
     rng = np.random.default_rng(3)
@@ -317,7 +318,7 @@ def test_sparse_decode_edges_and_device_errors():
     idx[1, 0, :1] = [0]; cnt[1, 0] = 1          # L < b: only the partial block
     cnt[2, 0] = 0                               # empty list
     idx[3, 0, :2] = [0, 2]; cnt[3, 0] = 2       # full block + one-token partial
-    for ns in (1, 2):
+    for ns in (1, 2, 0, -1):
         out = torch.full((cfg.B, cfg.Hq, d), 7.0, dtype=torch.bfloat16, device="cuda")
         lse = torch.empty((cfg.B, cfg.Hq), dtype=torch.float32, device="cuda")
         err = torch.zeros(1, dtype=torch.int32, device="cuda")
