@@ -505,8 +505,8 @@ seer_status seer_sparse_decode(const seer_dims_t* dims, const void* q, const see
   if (ns <= 0 && dims->batch * dims->num_kv_heads > seer::kMaxDecodeBH)
     return fail(SEER_ERR_UNSUPPORTED, "one-wave schedules need batch*num_kv_heads <= %d; pass num_split >= 1",
                 seer::kMaxDecodeBH);
-  if (ns == -1 && (int64_t)dims->batch * dims->num_kv_heads * capacity > INT32_MAX / 2)
-    return fail(SEER_ERR_UNSUPPORTED, "capacity schedule: batch*num_kv_heads*capacity too large");
+  if (ns <= 0 && (int64_t)dims->batch * dims->num_kv_heads * capacity >= (int64_t)1 << 30)
+    return fail(SEER_ERR_UNSUPPORTED, "one-wave schedules need batch*num_kv_heads*capacity < 2^30");
   const int ctas = ns <= 0 ? flat_grid(dims, df) : 0;
   size_t off_lse, off_o;
   const size_t need = ws_layout(dims, ns, ctas, &off_lse, &off_o);

@@ -99,19 +99,20 @@ __device__ __forceinline__ int clamp_cnt(const DecodeParams& p, int i) {
   return c < 0 ? 0 : (c > p.cap ? p.cap : c);
 }
 
-// floor(a / b) for 0 <= a < 2^53, 0 < b: a double quotient, then exact integer corrections
-// (a 64-bit integer division is a long software sequence; this is a few instructions)
-__device__ __forceinline__ long long floor_div(long long a, long long b) {
-  long long q = (long long)((double)a / (double)b);
-  while (q > 0 && q * b > a) --q;
-  while ((q + 1) * b <= a) ++q;
-  return q;
+// Balanced schedule: CTA c of G owns flattened positions [lo(c), lo(c+1)), lo(c) = floor(c*W/G).
+// W < 2^30 and G <= 2^15 (host-checked): with W = qG + r, c*W/G = c*q + c*r/G and c*r < 2^30,
+// so 32-bit integer arithmetic is exact (a 64-bit division is a long software sequence).
+__device__ __forceinline__ int range_lo(int c, int W, int G) {
+  const int q = W / G, r = W - (W / G) * G;
+  return c * q + (c * r) / G;
 }
-// Balanced schedule: CTA c of G owns flattened positions [lo(c), lo(c+1)).
-__device__ __forceinline__ long long range_lo(long long c, long long W, long long G) { return floor_div(c * W, G); }
-// The CTA whose range holds position `pos`.
-__device__ __forceinline__ int cta_of(long long pos, long long W, long long G) {
-  return (int)floor_div((pos + 1) * G - 1, W);
+// The CTA whose range holds position `pos` (0 <= pos < W): a float estimate of pos*G/W, then
+// exact corrections against range_lo.
+__device__ __forceinline__ int cta_of(int pos, int W, int G) {
+  int c = min(G - 1, max(0, (int)((float)pos * (float)G / (float)W)));
+  while (c + 1 < G && range_lo(c + 1, W, G) <= pos) ++c;
+  while (c > 0 && range_lo(c, W, G) > pos) --c;
+  return c;
 }
 // Last index i in [0, n) with pre[i] <= x (pre non-decreasing, pre[0] = 0 <= x).
 __device__ __forceinline__ int bh_of(const int* pre, int n, int x) {
@@ -324,19 +325,20 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
   if (p.flat) {
     if (tid == 0) {
       const int W = pre[BH];
-      const long long G = min((long long)gridDim.x, (long long)max(W, 1));
-      const long long c = blockIdx.x;
-      long long p0 = 0, p1 = 0;
+      const int G = min((int)gridDim.x, max(W, 1));
+      const int c = blockIdx.x;
+      int p0 = 0, p1 = 0;
       if (c < G && W > 0) {
         p0 = range_lo(c, W, G);
         p1 = range_lo(c + 1, W, G);
       }
-      const int bf = p1 > p0 ? bh_of(pre, BH, (int)p0) : 0;
-      const int bl = p1 > p0 ? bh_of(pre, BH, (int)p1 - 1) : 0;
+      // (b, h) of the first and last positions: the capacity schedule's prefix is bh * capacity
+      const int bf = p1 > p0 ? (p.flat == 2 ? p0 / p.cap : bh_of(pre, BH, p0)) : 0;
+      const int bl = p1 > p0 ? (p.flat == 2 ? (p1 - 1) / p.cap : bh_of(pre, BH, p1 - 1)) : 0;
       sh[2] = W;
-      sh[3] = (int)G;
-      sh[4] = (int)p0;
-      sh[5] = (int)p1;
+      sh[3] = G;
+      sh[4] = p0;
+      sh[5] = p1;
       sh[6] = bf;
       sh[7] = pre[bf];
       sh[16] = bl;
@@ -370,7 +372,7 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
       // split bookkeeping of the CTA's first and last segments (a middle one is a whole (b, h)):
       // the CTA of the first piece, the piece count and the first piece's partial slot
       if (nit > 0) {
-        const long long W = sh[2], G = sh[3];
+        const int W = sh[2], G = sh[3];
         const int bf = sh[6], bl = sh[16];
         const int cf_f = cta_of(pre[bf], W, G), cf_l = cta_of(pre[bl], W, G);
         sh[10] = cf_f;
@@ -428,13 +430,15 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
       }
       first = (it == 0 || pos == 0) ? kSegFirst : 0;
       const int b = bh / p.Hkv;
+      // the count (capacity schedule), the length and the block index, requested together
+      const int c = p.flat == 2 ? p.cnt[bh] : p.cap;
+      const int Lb = seq_len(b);
+      const int blk = p.idx[(size_t)bh * p.cap + pos];
       if (p.flat == 2) {   // list positions past the count are padding
-        const int c = p.cnt[bh];
         if (pos == 0 && c > p.cap) report(p.err, SEER_DEVERR_COUNT);
         if (pos >= c) return;
       }
-      const int nblk = (seq_len(b) + BLK - 1) / BLK;
-      const int blk = p.idx[(size_t)bh * p.cap + pos];
+      const int nblk = (Lb + BLK - 1) / BLK;
       bool ok = blk >= 0 && blk < nblk;
       if (!ok) report(p.err, SEER_DEVERR_BLOCK_INDEX);
       kb = vb = b;

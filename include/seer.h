@@ -219,7 +219,8 @@ size_t seer_sparse_decode_workspace_bytes(const seer_dims_t* dims, int32_t capac
  *     (those at or past block_cnt are skipped), so the ranges need no scan of the counts and the
  *     first tiles are requested one round trip after the launch's inputs are ready.  Best when
  *     the counts are at or near the capacity (top-k with a fixed budget); with short lists the
- *     skipped positions leave CTAs idle.  Requires batch*Hkv*capacity < 2^30.
+ *     skipped positions leave CTAs idle.
+ * Both one-wave schedules require batch*Hkv <= 4096 and batch*Hkv*capacity < 2^30.
  * In all, a (b, h) computed by several CTAs is merged (LSE combine) by the last of them.
  *
  *   q          device bf16 [B, Hq, d]  (post-RoPE query, as the model uses it)
