@@ -146,7 +146,55 @@ __device__ void merge_partials(const DecodeParams& p, int bh, int nseg, int slot
   const int b = bh / p.Hkv, h = bh - b * p.Hkv;
   const size_t qh0 = (size_t)b * p.Hq + (size_t)h * g;
   const int ng = nseg * g;
-  if (ng <= kEpi) {
+  constexpr int EPT = (kMaxGroup * D + NT - 1) / NT;
+  constexpr int MAXS = 4;   // pieces whose partial outputs are loaded together with the LSEs
+  constexpr bool kRegs = EPT <= 8;   // the outputs of MAXS pieces fit in registers (NT >= 128)
+  if (kRegs && nseg <= MAXS && ng <= kEpi) {
+    // one round trip: every piece's LSEs and this thread's outputs are requested at once
+    float ov[MAXS][kRegs ? EPT : 1];
+#pragma unroll
+    for (int k = 0; k < MAXS; ++k) {
+      const size_t sl = (size_t)split_slot(p, bh, k < nseg ? k : 0, slot_first, cf);
+#pragma unroll
+      for (int u = 0; u < EPT; ++u) {
+        const int e = u * NT + t;
+        const int j = e / D;
+        if (kRegs) ov[k][kRegs ? u : 0] = (k < nseg && e < g * D) ? __ldcg(p.o_part + (sl * g + j) * D + (e - j * D)) : 0.f;
+      }
+    }
+    float* Mh = wsc + kEpi;
+    float* Zh = Mh + kMaxGroup;
+    for (int i = t; i < ng; i += NT)
+      wsc[i] = __ldcg(p.lse_part + (size_t)split_slot(p, bh, i / g, slot_first, cf) * g + (i % g));
+    sync();
+    if (t < g) {
+      float M = -INFINITY;
+      for (int k = 0; k < nseg; ++k) M = fmaxf(M, wsc[k * g + t]);
+      float Z = 0.f;
+      if (M != -INFINITY)
+        for (int k = 0; k < nseg; ++k) Z += expf(wsc[k * g + t] - M);
+      Mh[t] = M;
+      Zh[t] = Z;
+    }
+    sync();
+#pragma unroll
+    for (int u = 0; u < EPT; ++u) {
+      const int e = u * NT + t;
+      if (e < g * D) {
+        const int j = e / D, cc = e - j * D;
+        const float M = Mh[j], Z = Zh[j];
+        float acc = 0.f;
+        if (M != -INFINITY && Z > 0.f) {
+#pragma unroll
+          for (int k = 0; k < MAXS; ++k)
+            if (k < nseg) acc += expf(wsc[k * g + j] - M) / Z * ov[k][kRegs ? u : 0];
+        }
+        __nv_bfloat16 ob = __float2bfloat16_rn(acc);
+        p.out[(qh0 + j) * D + cc] = *reinterpret_cast<uint16_t*>(&ob);
+        if (cc == 0 && p.lse_out) p.lse_out[qh0 + j] = Z > 0.f ? M + logf(Z) : -INFINITY;
+      }
+    }
+  } else if (ng <= kEpi) {
     // partial LSEs -> shared; per-head max and weight sum; weights w[k][j] = exp(lse - M) / Z
     float* Mh = wsc + kEpi;
     float* Zh = Mh + kMaxGroup;
@@ -169,7 +217,6 @@ __device__ void merge_partials(const DecodeParams& p, int bh, int nseg, int slot
       wsc[i] = (M != -INFINITY && Z > 0.f) ? expf(wsc[i] - M) / Z : 0.f;
     }
     sync();
-    constexpr int EPT = (kMaxGroup * D + NT - 1) / NT;
     float acc[EPT];
 #pragma unroll
     for (int u = 0; u < EPT; ++u) acc[u] = 0.f;
