@@ -55,6 +55,7 @@ def parse():
     ap.add_argument("--replicas", type=int, default=3)
     ap.add_argument("--budget", type=int, default=0, help="override the token budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the sparsity sweep rows")
     ap.add_argument("--cpu-sample", type=int, default=16, help="(b, h) pairs in the oracle sample")
     ap.add_argument("--only", default="all", choices=["all", "decode"],
                     help="decode: run just the sparse-decode launches (a small target for profilers)")
@@ -245,6 +246,102 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------------------- GPU arm
+
+def sweep_rows(S, dev, stream, peak, shape2, reps2, seqlens2, cfg2, inp2, iters=60, warm=5):
+    """The roofline rows besides the headline step: config 2 at k = 52 (89.8 % sparse) and the
+    64k sweep (config 4) at 50/75/90/95 % sparsity plus its all-blocks dense path.  Block lists
+    come from the plan kernel; the sparse decode alone is timed (eager launches rotating over
+    three replicas of the K/V cache, CUDA events)."""
+    import torch
+    from synthetic import SWEEP_SPARSITIES, config, make_inputs, sweep_budget
+
+    def time_decode(steps_, q_list, seql):
+        R = len(steps_)
+
+        def one(i):
+            st = steps_[i % R]
+            S.sparse_decode(st.shape, q_list[i % R], st.k, st.v, st.block_idx, st.block_cnt, seql, st.out,
+                            st.workspace, st.num_split, st.lse, st.err, stream=stream)
+        with torch.cuda.stream(stream):
+            for i in range(warm):
+                one(i)
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for i in range(iters):
+                one(i)
+            e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1) / iters * 1e3
+
+    def row(cfg, inp, steps_, q_list, seql, extra):
+        st = steps_[0]
+        with torch.cuda.stream(stream):
+            for r, s_ in enumerate(steps_):
+                s_.run(q_list[r], seql, stream=stream)
+        stream.synchronize()
+        cnt_h, idx_h = st.block_cnt.cpu().numpy(), st.block_idx.cpu().numpy()
+        nb = algorithmic_bytes(cfg, inp.seqlens, cnt_h, idx_h, st.capacity, inp.max_blocks)
+        us = time_decode(steps_, q_list, seql)
+        gbs = nb["decode"] / (us * 1e-6) / 1e9
+        out = {"decode_us": us, "achieved_gbs": gbs, "frac": gbs / peak, "bytes": nb["decode"],
+               "sparsity": 1.0 - float(cnt_h.mean()) / inp.max_blocks, "num_split": st.num_split}
+        out.update(extra)
+        return out
+
+    def steps_for(shape, reps_kv, w_q, w_k, kcs, valids, budget):
+        return [S.DecodeStep(shape, S.KVCache.contiguous(k), S.KVCache.contiguous(v), w_q, w_k, kc, valid,
+                             mode=S.SELECT_TOPK, token_budget=budget)
+                for (k, v), kc, valid in zip(reps_kv, kcs, valids)]
+
+    res = {}
+    # config 2 at k = 52
+    b52 = 3277
+    st2 = steps_for(shape2, [(rp["k"], rp["v"]) for rp in reps2], reps2[0]["step"].w_q, reps2[0]["step"].w_k,
+                    [rp["step"].kcomp for rp in reps2], [rp["step"].valid_blocks for rp in reps2], b52)
+    res["qwen3-8b-32k-k52"] = row(cfg2, inp2, st2, [rp["q"] for rp in reps2], seqlens2,
+                                  {"token_budget": b52, "k": -(-b52 // cfg2.block)})
+    del st2
+    # config 4: 64k context, sparsity sweep and the dense path
+    cfg4 = config(4)
+    inp4 = make_inputs(cfg4)
+
+    def up(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+    NB4 = inp4.max_blocks
+    shape4 = S.Shape(cfg4.B, cfg4.Hq, cfg4.Hkv, cfg4.head_dim, cfg4.gate_dim, cfg4.block, NB4, cfg4.rope_base)
+    w_q4, w_k4 = up(inp4.w_q), up(inp4.w_k)
+    seq4 = torch.from_numpy(inp4.seqlens).to(dev)
+    k4, v4 = up(inp4.k), up(inp4.v)
+    kv4 = [(k4, v4)] + [(k4.clone(), v4.clone()) for _ in range(2)]
+    q4 = [up(inp4.q) for _ in range(3)]
+    kcs4, valids4 = [], []
+    for k, _ in kv4:
+        kc = torch.zeros(cfg4.B, cfg4.Hkv, NB4, cfg4.gate_dim, dtype=torch.bfloat16, device=dev)
+        valid = torch.zeros(cfg4.B, cfg4.Hkv, dtype=torch.int32, device=dev)
+        S.kcomp_update(shape4, S.KVCache.contiguous(k), seq4, valid, w_k4, kc)
+        kcs4.append(kc)
+        valids4.append(valid)
+    rows = []
+    for sp in SWEEP_SPARSITIES:
+        bud = sweep_budget(cfg4.length, sp)
+        st4 = steps_for(shape4, kv4, w_q4, w_k4, kcs4, valids4, bud)
+        rows.append(row(cfg4, inp4, st4, q4, seq4, {"target_sparsity": sp, "token_budget": bud,
+                                                      "k": -(-bud // cfg4.block)}))
+        del st4
+    res["sweep-64k"] = rows
+    # the all-blocks dense path on the same inputs (same kernel, every block selected)
+    st_d = steps_for(shape4, kv4, w_q4, w_k4, kcs4, valids4, cfg4.length)
+    dense = row(cfg4, inp4, st_d, q4, seq4, {"token_budget": cfg4.length, "k": NB4})
+    res["dense-64k"] = dense
+    for r_ in rows:
+        r_["speedup_vs_dense"] = dense["decode_us"] / r_["decode_us"]
+    del st_d, kv4, k4, v4
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res
+
 
 def run_seer(args):
     import torch
@@ -476,6 +573,24 @@ def run_seer(args):
     d2h = B * Hq * d * 2
 
     # ---------------- CPU oracle on a bounded sample (rank 0, single GPU only)
+    # ---------------- per-step spread: an event after every replay (separate from the headline)
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            graphs[i % R].replay()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(101)]
+        evs[0].record(stream)
+        for i in range(100):
+            graphs[i % R].replay()
+            evs[i + 1].record(stream)
+    evs[-1].synchronize()
+    per_step = [evs[i].elapsed_time(evs[i + 1]) * 1e3 for i in range(100)]
+    step_pct = [float(np.percentile(per_step, q)) for q in (10, 50, 90)]
+
+    # ---------------- the other roofline rows (single GPU)
+    sweep = None
+    if world == 1 and not args.no_sweep:
+        sweep = sweep_rows(S, dev, stream, peak, shape, reps, seqlens, cfg, inp)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rng = np.random.default_rng(0)
@@ -510,6 +625,8 @@ def run_seer(args):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": _profiled_traffic(), "traffic_unit": "bytes per launch (ncu dram read+write)",
                      "kernel": "sparse_decode_kernel", "peak_kind": peak_kind},
+        "step_us_p10_p50_p90": step_pct,
+        "sweep": sweep,
         "e2e": {"value": e2e_ms * 1e3, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "mode": "graph replay of DecodeStep.run per step; query H2D and output D2H on their own "
                         "copy streams, overlapping the neighbouring steps' compute"},
