@@ -296,6 +296,32 @@ def sweep_rows(S, dev, stream, peak, shape2, reps2, seqlens2, cfg2, inp2, iters=
                 for (k, v), kc, valid in zip(reps_kv, kcs, valids)]
 
     res = {}
+    # decode ground truth (full attention scores of every block) on the 32k step: reads all of K
+    sh_t = shape2
+    ws_t = S.alloc_truth_workspace(sh_t, dev)
+    sc_t = torch.empty(cfg2.B, cfg2.Hkv, inp2.max_blocks, dtype=torch.float32, device=dev)
+    kvs_t = [S.KVCache.contiguous(rp["k"]) for rp in reps2]
+
+    def truth(i):
+        S.gate_truth(sh_t, reps2[i % len(reps2)]["q"], kvs_t[i % len(reps2)], seqlens2, sc_t, ws_t, stream=stream)
+    with torch.cuda.stream(stream):
+        for i in range(warm):
+            truth(i)
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(iters):
+            truth(i)
+        e1.record(stream)
+    e1.synchronize()
+    us_t = e0.elapsed_time(e1) / iters * 1e3
+    k_bytes = int(sum(int(L) for L in inp2.seqlens)) * cfg2.Hkv * cfg2.head_dim * 2
+    t_bytes = k_bytes + cfg2.B * cfg2.Hq * cfg2.head_dim * 2 + cfg2.B * cfg2.Hkv * inp2.max_blocks * 4
+    res["ground-truth-32k"] = {"us": us_t, "bytes": t_bytes, "achieved_gbs": t_bytes / (us_t * 1e-6) / 1e9,
+                               "frac": t_bytes / (us_t * 1e-6) / 1e9 / peak,
+                               "what": "seer_gate_truth: all of K read once (K bytes + q + scores)"}
+    del ws_t, sc_t
     # config 2 at k = 52
     b52 = 3277
     st2 = steps_for(shape2, [(rp["k"], rp["v"]) for rp in reps2], reps2[0]["step"].w_q, reps2[0]["step"].w_k,

@@ -555,4 +555,73 @@ seer_status seer_sparse_decode(const seer_dims_t* dims, const void* q, const see
   return SEER_OK;
 }
 
+// ---------------------------------------------------------------- decode ground truth
+
+namespace {
+// counters [BH] | per-chunk (max, sum) [BH][nchunk][warps][8][2] | block maxima [BH][NB][warps][8]
+size_t truth_layout(const seer_dims_t* d, int* nchunk, size_t* off_part, size_t* off_bmax) {
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  const size_t bh = (size_t)d->batch * d->num_kv_heads;
+  const int nc = (d->max_blocks + seer::truth_chunk_blocks() - 1) / seer::truth_chunk_blocks();
+  const size_t w = (size_t)seer::truth_warps() * seer::kMaxGroup;
+  *nchunk = nc;
+  *off_part = up(bh * 4);
+  *off_bmax = *off_part + up(bh * nc * w * 2 * 4);
+  return *off_bmax + bh * d->max_blocks * w * 4;
+}
+}  // namespace
+
+size_t seer_gate_truth_workspace_bytes(const seer_dims_t* dims) {
+  if (check_dims(dims) != SEER_OK) return 0;
+  int nc;
+  size_t a, b;
+  return truth_layout(dims, &nc, &a, &b);
+}
+
+seer_status seer_gate_truth(const seer_dims_t* dims, const void* q, const seer_kv_t* k, const int32_t* seqlens,
+                            float* scores, float* log_scores, void* workspace, size_t workspace_bytes,
+                            int32_t* err_word, void* stream) {
+  seer_status st = check_dims(dims);
+  if (st != SEER_OK) return st;
+  if ((st = check_kv(dims, k, "k")) != SEER_OK) return st;
+  if (!q || !seqlens || !scores || !workspace) return fail(SEER_ERR_INVALID_ARG, "NULL pointer argument");
+  if (!aligned16(q) || !aligned16(scores) || (log_scores && !aligned16(log_scores)) || !aligned16(workspace))
+    return fail(SEER_ERR_INVALID_ARG, "pointer not 16-byte aligned");
+  int nc;
+  size_t off_part, off_bmax;
+  const size_t need = truth_layout(dims, &nc, &off_part, &off_bmax);
+  if (workspace_bytes < need)
+    return fail(SEER_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", workspace_bytes, need);
+  int dev;
+  DevFacts* df;
+  if ((st = device_facts(&dev, &df)) != SEER_OK) return st;
+  CUtensorMap tk;
+  seer::TruthParams p;
+  if ((st = tensor_map(dims, k, "k", &tk, p.k_perm)) != SEER_OK) return st;
+  p.q = static_cast<const uint16_t*>(q);
+  p.seqlens = seqlens;
+  p.k_paged = k->layout == SEER_KV_PAGED;
+  p.k_table = k->block_table;
+  p.k_maxp = k->max_pages_per_seq;
+  p.k_pages = k->num_pages;
+  p.B = dims->batch;
+  p.Hq = dims->num_q_heads;
+  p.Hkv = dims->num_kv_heads;
+  p.g = dims->num_q_heads / dims->num_kv_heads;
+  p.NB = dims->max_blocks;
+  p.nchunk = nc;
+  const float scale = dims->softmax_scale > 0.f ? dims->softmax_scale : 1.0f / sqrtf((float)dims->head_dim);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.scores = scores;
+  p.log_scores = log_scores;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  p.counters = reinterpret_cast<int32_t*>(ws);
+  p.part = reinterpret_cast<float*>(ws + off_part);
+  p.bmax = reinterpret_cast<float*>(ws + off_bmax);
+  p.err = err_word;
+  cudaError_t e = seer::launch_gate_truth(tk, p, dims->head_dim, dims->block_size, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "gate_truth launch");
+  return SEER_OK;
+}
+
 }  // extern "C"

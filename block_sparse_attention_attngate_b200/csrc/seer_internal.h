@@ -141,6 +141,28 @@ cudaError_t launch_sparse_decode(const CUtensorMap& tk, const CUtensorMap& tv, c
                                  int D, int BLK, int grid_flat, cudaStream_t s);
 int decode_ctas_per_sm(int D, int BLK);
 
+// ---------------------------------------------------------------- decode ground truth
+struct TruthParams {
+  const uint16_t* q;        // [B, Hq, D]
+  const int32_t* seqlens;   // [B]
+  const int32_t* k_table;   // paged block table or null
+  int32_t k_maxp;
+  int64_t k_pages;
+  int32_t k_paged;
+  int32_t k_perm[3];
+  int32_t B, Hq, Hkv, g, NB, nchunk;
+  float scale_log2;         // softmax scale * log2(e)
+  float* scores;            // [B, Hkv, NB]
+  float* log_scores;        // [B, Hkv, NB] or null
+  float* bmax;              // workspace [B*Hkv, NB, warps, 8]
+  float* part;              // workspace [B*Hkv, nchunk, warps, 8, 2]
+  int32_t* counters;        // workspace [B*Hkv] (zero between calls)
+  int32_t* err;
+};
+cudaError_t launch_gate_truth(const CUtensorMap& tk, const TruthParams& p, int D, int BLK, cudaStream_t s);
+int truth_chunk_blocks();
+int truth_warps();
+
 // Record `msg` as the text seer_last_error() returns on this thread; returns `status`.
 int set_last_error(int status, const char* msg);
 

@@ -28,8 +28,8 @@ DEVERR_BLOCK_INDEX, DEVERR_PAGE_INDEX, DEVERR_COUNT, DEVERR_TIMEOUT = 1, 2, 4, 8
 
 EXPORTED = (
     "seer_kcomp_update", "seer_gate_score", "seer_select_blocks", "seer_decode_plan", "seer_sparse_decode_auto_split",
-    "seer_sparse_decode_workspace_bytes", "seer_sparse_decode", "seer_sparse_decode_noalloc", "seer_last_error",
-    "seer_version",
+    "seer_sparse_decode_workspace_bytes", "seer_sparse_decode", "seer_sparse_decode_noalloc",
+    "seer_gate_truth_workspace_bytes", "seer_gate_truth", "seer_last_error", "seer_version",
 )
 
 
@@ -67,6 +67,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "seer_sparse_decode_workspace_bytes": (SZ, [DP, I32, I32]),
         "seer_sparse_decode": (I32, [DP, P, KP, KP, P, P, P, I32, I32, P, SZ, P, P, P, P]),
         "seer_sparse_decode_noalloc": (I32, [DP, P, KP, KP, P, P, P, I32, I32, P, P, P, P]),
+        "seer_gate_truth_workspace_bytes": (SZ, [DP]),
+        "seer_gate_truth": (I32, [DP, P, KP, P, P, P, P, SZ, P, P]),
         "seer_last_error": (ctypes.c_char_p, []),
         "seer_version": (ctypes.c_char_p, []),
     }
@@ -276,6 +278,33 @@ def sparse_decode_noalloc(shape: Shape, q: torch.Tensor, k: KVCache, v: KVCache,
     _check(_lib.seer_sparse_decode_noalloc(ctypes.byref(dims), _ptr(q), ctypes.byref(k.desc), ctypes.byref(v.desc),
                                            _ptr(block_idx), _ptr(block_cnt), _ptr(seqlens), block_idx.shape[-1],
                                            int(num_split), _ptr(out), _ptr(lse), _ptr(err), _stream(stream)))
+
+
+def gate_truth_workspace_bytes(shape: Shape) -> int:
+    dims = shape.c()
+    return int(_lib.seer_gate_truth_workspace_bytes(ctypes.byref(dims)))
+
+
+def alloc_truth_workspace(shape: Shape, device=None) -> torch.Tensor:
+    """Zero-filled workspace for gate_truth (its arrival counters must start at zero)."""
+    return torch.zeros(max(gate_truth_workspace_bytes(shape), 16), dtype=torch.uint8, device=device or "cuda")
+
+
+def gate_truth(shape: Shape, q: torch.Tensor, k: KVCache, seqlens: torch.Tensor, scores: torch.Tensor,
+               workspace: torch.Tensor, log_scores: Optional[torch.Tensor] = None, err: Optional[torch.Tensor] = None,
+               stream=None):
+    """Decode ground-truth block scores from full attention (see seer_gate_truth)."""
+    _need(q, torch.bfloat16, "q")
+    _need(seqlens, torch.int32, "seqlens")
+    _need(scores, torch.float32, "scores")
+    if log_scores is not None:
+        _need(log_scores, torch.float32, "log_scores")
+    if err is not None:
+        _need(err, torch.int32, "err")
+    dims = shape.c()
+    _check(_lib.seer_gate_truth(ctypes.byref(dims), _ptr(q), ctypes.byref(k.desc), _ptr(seqlens), _ptr(scores),
+                                _ptr(log_scores), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                _ptr(err), _stream(stream)))
 
 
 class DecodeStep:

@@ -265,6 +265,34 @@ seer_status seer_sparse_decode_noalloc(const seer_dims_t* dims, const void* q, c
                                        int32_t capacity, int32_t num_split, void* out,
                                        float* lse_out, int32_t* err_word, void* stream);
 
+/*
+ * seer_gate_truth -- decode ground-truth block scores from full attention [CP Knowl 3]: the
+ * target the AttnGate is distilled towards, usable in its place ("oracle" selection).
+ *
+ * For each (b, h) with L = seqlens[b] and nblk = ceil(L / block_size) (capped at max_blocks):
+ *   p_j[t]  = softmax_t(scale * q[b, h*g+j] . K[b, h, t]) over t < L, for the g heads j of the group
+ *   raw[n]  = max_j max_{t in block n, t < L} p_j[t]                     (n < nblk)
+ *   scores[b, h, n] = raw[n] / sum_n' raw[n'] for n < nblk, 0 for n >= nblk (all 0 when L = 0)
+ *   log_scores[b, h, n] = log(scores[b, h, n]) (-inf where 0), if log_scores is not NULL:
+ *     top-k or threshold selection on these (seer_select_blocks) picks blocks by ground truth.
+ * Unlike the gate, the partial last block is scored too.
+ *
+ *   q           device bf16 [B, Hq, d] (the attention query: post-RoPE)
+ *   k           the attention K cache (see seer_kv_t)
+ *   seqlens     device int32 [B]
+ *   scores      device fp32 [B, Hkv, max_blocks]; log_scores the same or NULL
+ *   workspace   device, >= seer_gate_truth_workspace_bytes(dims) bytes, 16-byte aligned; its
+ *               first B*Hkv int32 are arrival counters that must be zero before the first call
+ *               (every completed call leaves them zero)
+ *   err_word    device int32 or NULL (SEER_DEVERR_* bits ORed in)
+ * Reads all of K once (HBM-bound).  Calls on the same workspace must not overlap on the GPU.
+ */
+size_t seer_gate_truth_workspace_bytes(const seer_dims_t* dims);
+seer_status seer_gate_truth(const seer_dims_t* dims, const void* q, const seer_kv_t* k,
+                            const int32_t* seqlens, float* scores, float* log_scores,
+                            void* workspace, size_t workspace_bytes, int32_t* err_word,
+                            void* stream);
+
 /* Thread-local text describing the last non-OK status returned on this thread. */
 const char* seer_last_error(void);
 
