@@ -56,6 +56,11 @@ __global__ void __cluster_dims__(kCL, 1, 1) __launch_bounds__(kThreads) plan_ker
   const int rank = (int)cluster.block_rank();
   const int h = blockIdx.y, b = blockIdx.z, bh = b * p.g.Hkv + h;
   if (threadIdx.x == 0) gate_prefetch_wq<D, DG, kCL>(p.g, h, rank, &wq_bar, wq_s);   // weights: no wait needed
+  // The parameters are fixed for the launch: bring them into the constant cache before the wait
+  // (the RoPE table alone spans eight 64-byte lines), so no first use afterwards waits on memory.
+  asm volatile("" ::"d"(p.g.theta[threadIdx.x % kMaxHalfGate]), "l"(p.g.q), "l"(p.g.kcomp), "l"(p.g.seqlens),
+               "l"(p.s.idx), "l"(p.s.cnt), "l"(p.k.valid), "r"(p.s.NB), "r"(p.s.cap), "r"(p.s.kblocks),
+               "d"(p.s.tau), "r"(p.update_cache));
   pdl_wait();
   pdl_trigger();
   GateQuery<D, DG, kCL, kThreads> q;

@@ -321,17 +321,38 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
     sh[9] = 0;
     fence_barrier_init();
   }
+  __syncthreads();   // barrier inits visible to every warp (before the wait: off the critical path)
+  // The parameters are fixed for the launch: bring the ones the first loads depend on into the
+  // constant cache now, so their first use after the wait does not cost a memory round trip.
+  asm volatile("" ::"l"(p.q), "l"(p.idx), "l"(p.cnt), "l"(p.seqlens), "l"(p.k_table), "l"(p.counters),
+               "l"(p.err), "l"(p.out), "r"(p.cap), "r"(p.flat), "r"(p.B), "r"(p.Hkv), "r"(p.k_perm[0]),
+               "r"(p.v_perm[2]), "r"(p.per_split), "f"(p.scale_log2));
   pdl_wait();
   pdl_trigger();
 
   // ---------------------------------------------------------------- lengths, list prefix, this CTA's range
-  // (the capacity schedule reads nothing here: its prefix is bh * capacity, and the lengths are
-  // read where they are used)
+  // (the capacity schedule reads nothing here: its prefix is bh * capacity, the lengths are read
+  // where they are used, and its producer warp computes its own range and starts at once -- the
+  // other warps run this prologue behind a named barrier that leaves the producer out)
+  const bool fast = p.flat == 2;
+  int pp0 = 0, pnit = 0, pbh = 0;   // the producer's range start, length and (grid schedule) (b, h)
+  auto cta_sync = [&]() {
+    if (fast) asm volatile("bar.sync 1, %0;" ::"r"((CW + 1) * 32) : "memory");
+    else __syncthreads();
+  };
+  if (fast && warp == CW) {
+    const int W = BH * p.cap, G = min((int)gridDim.x, max(W, 1)), c = blockIdx.x;
+    if (c < G && W > 0) {
+      pp0 = range_lo(c, W, G);
+      pnit = range_lo(c + 1, W, G) - pp0;
+    }
+  } else {
   if (p.flat != 2)
     for (int i = tid; i < p.B; i += S::kThreads) slen[i] = max(p.seqlens[i], 0);
   if (p.flat == 2) {
-    for (int i = tid; i <= BH; i += S::kThreads) pre[i] = i * p.cap;
-    __syncthreads();
+    const int t2 = warp < CW ? tid : tid - 32;   // the (CW+1)*32 threads other than the producer
+    for (int i = t2; i <= BH; i += (CW + 1) * 32) pre[i] = i * p.cap;
+    cta_sync();
   }
   if (p.flat == 1) {
     // each thread sums a contiguous run of counts, then one block-wide exclusive scan
@@ -410,8 +431,12 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
     sh[17] = 1;
     pre[0] = c;  // the grid schedule keeps its one list length here
   }
-  __syncthreads();
-  const int nit = sh[5] - sh[4];
+  cta_sync();
+  pp0 = sh[4];
+  pnit = sh[5] - sh[4];
+  pbh = sh[6];
+  }
+  const int nit = pnit;
 
   if (warp == CW + 1) {
     // ------------------------------------------------------------ epilogue warp
@@ -458,8 +483,8 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
 
   if (warp == CW) {
     // ------------------------------------------------------------ producer warp
-    const int p0 = sh[4];
-    const int fixed_bh = sh[6];
+    const int p0 = pp0;
+    const int fixed_bh = pbh;
     // resolve list position `it` of this CTA (one lane per position)
     auto resolve = [&](int it, int& n, int& bh, int& first, int& kb, int& kt, int& vb, int& vt) {
       n = -1;
@@ -468,7 +493,11 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
       kb = vb = kt = vt = 0;
       if (it >= nit) return;
       int pos;
-      if (p.flat) {
+      if (fast) {
+        const int x = p0 + it;
+        bh = x / p.cap;
+        pos = x - bh * p.cap;
+      } else if (p.flat) {
         const int x = p0 + it;
         bh = bh_of(pre, BH, x);
         pos = x - pre[bh];

@@ -68,7 +68,7 @@ extern "C" seer_status seer_sparse_decode_noalloc(const seer_dims_t* dims, const
                                                   int32_t* err_word, void* stream) {
   if (!dims) return (seer_status)seer::set_last_error(SEER_ERR_INVALID_ARG, "dims is NULL");
   if (capacity < 1) return (seer_status)seer::set_last_error(SEER_ERR_INVALID_ARG, "capacity must be >= 1");
-  if (num_split < 0) return (seer_status)seer::set_last_error(SEER_ERR_INVALID_ARG, "num_split must be >= 0");
+  if (num_split < -1) return (seer_status)seer::set_last_error(SEER_ERR_INVALID_ARG, "num_split must be >= -1");
   const int32_t ns = num_split;
   const size_t need = seer_sparse_decode_workspace_bytes(dims, capacity, ns);
   if (need > kNoAllocScratchBytes) {

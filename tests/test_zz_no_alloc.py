@@ -29,7 +29,8 @@ def _close(a, b, what):
     assert max_abs <= OUT_MAX_ABS and rel <= OUT_REL_L2, f"{what}: max-abs {max_abs:.2e} rel {rel:.2e}"
 
 
-def test_noalloc_matches_workspace_entry_point_twice():
+@pytest.mark.parametrize("ns", [3, -1])
+def test_noalloc_matches_workspace_entry_point_twice(ns):
     import block_sparse_attention_attngate_b200 as S
     from block_sparse_attention_attngate_b200 import seer
 
@@ -44,7 +45,6 @@ def test_noalloc_matches_workspace_entry_point_twice():
     idx_h, cnt_h = make_block_lists(99, lengths, Hkv, blk, cap, density=0.5)
     idx, cnt = torch.from_numpy(idx_h).cuda(), torch.from_numpy(cnt_h).cuda()
     seq = torch.from_numpy(inp.seqlens).cuda()
-    ns = 3
     ref = torch.empty(cfg.B, cfg.Hq, d, dtype=torch.bfloat16, device="cuda")
     ref_lse = torch.empty(cfg.B, cfg.Hq, dtype=torch.float32, device="cuda")
     S.sparse_decode(sh, q, kk, vv, idx, cnt, seq, ref, S.alloc_workspace(sh, cap, ns), num_split=ns, lse=ref_lse)
