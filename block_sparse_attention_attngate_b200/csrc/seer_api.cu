@@ -563,7 +563,7 @@ size_t truth_layout(const seer_dims_t* d, int* nchunk, size_t* off_part, size_t*
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
   const size_t bh = (size_t)d->batch * d->num_kv_heads;
   const int nc = (d->max_blocks + seer::truth_chunk_blocks() - 1) / seer::truth_chunk_blocks();
-  const size_t w = (size_t)seer::truth_warps() * seer::kMaxGroup;
+  const size_t w = seer::kMaxGroup;
   *nchunk = nc;
   *off_part = up(bh * 4);
   *off_bmax = *off_part + up(bh * nc * w * 2 * 4);
@@ -610,6 +610,7 @@ seer_status seer_gate_truth(const seer_dims_t* dims, const void* q, const seer_k
   p.g = dims->num_q_heads / dims->num_kv_heads;
   p.NB = dims->max_blocks;
   p.nchunk = nc;
+  p.nitems = dims->batch * dims->num_kv_heads * nc;
   const float scale = dims->softmax_scale > 0.f ? dims->softmax_scale : 1.0f / sqrtf((float)dims->head_dim);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.scores = scores;
@@ -619,7 +620,8 @@ seer_status seer_gate_truth(const seer_dims_t* dims, const void* q, const seer_k
   p.part = reinterpret_cast<float*>(ws + off_part);
   p.bmax = reinterpret_cast<float*>(ws + off_bmax);
   p.err = err_word;
-  cudaError_t e = seer::launch_gate_truth(tk, p, dims->head_dim, dims->block_size, static_cast<cudaStream_t>(stream));
+  cudaError_t e = seer::launch_gate_truth(tk, p, dims->head_dim, dims->block_size, df->sms,
+                                          static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "gate_truth launch");
   return SEER_OK;
 }

@@ -151,17 +151,17 @@ struct TruthParams {
   int32_t k_paged;
   int32_t k_perm[3];
   int32_t B, Hq, Hkv, g, NB, nchunk;
+  int32_t nitems;           // B * Hkv * nchunk work items
   float scale_log2;         // softmax scale * log2(e)
   float* scores;            // [B, Hkv, NB]
   float* log_scores;        // [B, Hkv, NB] or null
-  float* bmax;              // workspace [B*Hkv, NB, warps, 8]
-  float* part;              // workspace [B*Hkv, nchunk, warps, 8, 2]
+  float* bmax;              // workspace [B*Hkv, NB, 8]: per head, the block's score maximum (log2 domain)
+  float* part;              // workspace [B*Hkv, nchunk, 8, 2]: per head, the chunk's (max, sum of exp2)
   int32_t* counters;        // workspace [B*Hkv] (zero between calls)
   int32_t* err;
 };
-cudaError_t launch_gate_truth(const CUtensorMap& tk, const TruthParams& p, int D, int BLK, cudaStream_t s);
+cudaError_t launch_gate_truth(const CUtensorMap& tk, const TruthParams& p, int D, int BLK, int sms, cudaStream_t s);
 int truth_chunk_blocks();
-int truth_warps();
 
 // Record `msg` as the text seer_last_error() returns on this thread; returns `status`.
 int set_last_error(int status, const char* msg);
