@@ -327,14 +327,18 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
   asm volatile("" ::"l"(p.q), "l"(p.idx), "l"(p.cnt), "l"(p.seqlens), "l"(p.k_table), "l"(p.counters),
                "l"(p.err), "l"(p.out), "r"(p.cap), "r"(p.flat), "r"(p.B), "r"(p.Hkv), "r"(p.k_perm[0]),
                "r"(p.v_perm[2]), "r"(p.per_split), "f"(p.scale_log2));
-  pdl_wait();
-  pdl_trigger();
+  const bool fast = p.flat == 2;
+  // (the capacity schedule's producer warp waits for the launch's inputs further down, after a dry
+  // pass over its issue code)
+  if (!(fast && warp == CW)) {
+    pdl_wait();
+    pdl_trigger();
+  }
 
   // ---------------------------------------------------------------- lengths, list prefix, this CTA's range
   // (the capacity schedule reads nothing here: its prefix is bh * capacity, the lengths are read
   // where they are used, and its producer warp computes its own range and starts at once -- the
   // other warps run this prologue behind a named barrier that leaves the producer out)
-  const bool fast = p.flat == 2;
   int pp0 = 0, pnit = 0, pbh = 0;   // the producer's range start, length and (grid schedule) (b, h)
   auto cta_sync = [&]() {
     if (fast) asm volatile("bar.sync 1, %0;" ::"r"((CW + 1) * 32) : "memory");
@@ -486,6 +490,7 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
     const int p0 = pp0;
     const int fixed_bh = pbh;
     // resolve list position `it` of this CTA (one lane per position)
+    bool dry = false;
     auto resolve = [&](int it, int& n, int& bh, int& first, int& kb, int& kt, int& vb, int& vt) {
       n = -1;
       bh = fixed_bh;
@@ -511,18 +516,18 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
       const int Lb = seq_len(b);
       const int blk = p.idx[(size_t)bh * p.cap + pos];
       if (p.flat == 2) {   // list positions past the count are padding
-        if (pos == 0 && c > p.cap) report(p.err, SEER_DEVERR_COUNT);
+        if (pos == 0 && c > p.cap && !dry) report(p.err, SEER_DEVERR_COUNT);
         if (pos >= c) return;
       }
       const int nblk = (Lb + BLK - 1) / BLK;
       bool ok = blk >= 0 && blk < nblk;
-      if (!ok) report(p.err, SEER_DEVERR_BLOCK_INDEX);
+      if (!ok && !dry) report(p.err, SEER_DEVERR_BLOCK_INDEX);
       kb = vb = b;
       kt = vt = blk * BLK;
       if (ok && p.k_paged) {
         const int pg = blk < p.k_maxp ? p.k_table[(size_t)b * p.k_maxp + blk] : -1;
         if (pg < 0 || pg >= p.k_pages) {
-          report(p.err, SEER_DEVERR_PAGE_INDEX);
+          if (!dry) report(p.err, SEER_DEVERR_PAGE_INDEX);
           ok = false;
         }
         kb = pg;
@@ -531,7 +536,7 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
       if (ok && p.v_paged) {
         const int pg = blk < p.v_maxp ? p.v_table[(size_t)b * p.v_maxp + blk] : -1;
         if (pg < 0 || pg >= p.v_pages) {
-          report(p.err, SEER_DEVERR_PAGE_INDEX);
+          if (!dry) report(p.err, SEER_DEVERR_PAGE_INDEX);
           ok = false;
         }
         vb = pg;
@@ -541,69 +546,82 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
     };
     const uint64_t stream_pol = l2_evict_first_policy();   // each K/V tile is read once
     const uint32_t qbytes = (uint32_t)(g * D * 2);
-    int nq = 0;   // segments whose q copy was issued
-    int cn_, cb_, cf_, ckb, ckt, cvb, cvt;   // current chunk (this lane's position)
-    resolve(lane, cn_, cb_, cf_, ckb, ckt, cvb, cvt);
-    bool abort = false;
-    for (int chunk = 0; chunk * 32 < nit && !abort; ++chunk) {
-      int nn, nb, nf, nkb, nkt, nvb, nvt;   // next chunk, fetched while this one issues
-      resolve((chunk + 1) * 32 + lane, nn, nb, nf, nkb, nkt, nvb, nvt);
-      const int count = min(32, nit - chunk * 32);
-      for (int j = 0; j < count; ++j) {
-        const int it = chunk * 32 + j;
-        const int n = __shfl_sync(0xffffffffu, cn_, j);
-        const int bh = __shfl_sync(0xffffffffu, cb_, j);
-        const int first = __shfl_sync(0xffffffffu, cf_, j);
-        const int kb = __shfl_sync(0xffffffffu, ckb, j), kt = __shfl_sync(0xffffffffu, ckt, j);
-        const int vb = __shfl_sync(0xffffffffu, cvb, j), vt = __shfl_sync(0xffffffffu, cvt, j);
-        if (lane == 0) {
-          if (first) {
-            // the segment's q rows -> segment buffer nq & 1, once the segment two back has read it
-            const int k = nq & 1, u = nq >> 1;
-            if (u >= 1 && !mbar_wait(&qempty[k], (u - 1) & 1)) {
+    // The capacity schedule's range needs none of the launch's inputs, so its producer makes a dry
+    // pass over the resolve / issue loop before it waits for them (two positions; the lists are
+    // read but the values are dropped, and no copy, barrier arrival or report is made).  Run for the
+    // first time after the wait, this code delayed the first tile request by ~0.7 us more.
+#pragma unroll 1
+    for (int pass = fast ? 0 : 1; pass < 2; ++pass) {
+      dry = pass == 0;
+      if (fast && !dry) {
+        pdl_wait();
+        pdl_trigger();
+      }
+      int nq = 0;   // segments whose q copy was issued
+      int cn_, cb_, cf_, ckb, ckt, cvb, cvt;   // current chunk (this lane's position)
+      resolve(lane, cn_, cb_, cf_, ckb, ckt, cvb, cvt);
+      bool abort = false;
+      for (int chunk = 0; chunk * 32 < nit && !abort; ++chunk) {
+        int nn, nb, nf, nkb, nkt, nvb, nvt;   // next chunk, fetched while this one issues
+        resolve((chunk + 1) * 32 + lane, nn, nb, nf, nkb, nkt, nvb, nvt);
+        const int count = min(dry ? 2 : 32, nit - chunk * 32);
+        for (int j = 0; j < count; ++j) {
+          const int it = chunk * 32 + j;
+          const int n = __shfl_sync(0xffffffffu, cn_, j);
+          const int bh = __shfl_sync(0xffffffffu, cb_, j);
+          const int first = __shfl_sync(0xffffffffu, cf_, j);
+          const int kb = __shfl_sync(0xffffffffu, ckb, j), kt = __shfl_sync(0xffffffffu, ckt, j);
+          const int vb = __shfl_sync(0xffffffffu, cvb, j), vt = __shfl_sync(0xffffffffu, cvt, j);
+          if (lane == 0 && !dry) {
+            if (first) {
+              // the segment's q rows -> segment buffer nq & 1, once the segment two back has read it
+              const int k = nq & 1, u = nq >> 1;
+              if (u >= 1 && !mbar_wait(&qempty[k], (u - 1) & 1)) {
+                report(p.err, SEER_DEVERR_TIMEOUT);
+                sh[0] = 1;
+              }
+              if (!sh[0]) {
+                const int b = bh / p.Hkv, h = bh - b * p.Hkv;
+                mbar_arrive_expect_tx(&qfull[k], qbytes);
+                bulk_load(qseg + k * S::kQBytes, p.q + ((size_t)b * p.Hq + (size_t)h * g) * D, qbytes, &qfull[k]);
+              }
+              ++nq;
+            }
+            const int s = it % STAGES;
+            if (!sh[0] && it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) - 1) & 1)) {
               report(p.err, SEER_DEVERR_TIMEOUT);
               sh[0] = 1;
             }
             if (!sh[0]) {
-              const int b = bh / p.Hkv, h = bh - b * p.Hkv;
-              mbar_arrive_expect_tx(&qfull[k], qbytes);
-              bulk_load(qseg + k * S::kQBytes, p.q + ((size_t)b * p.Hq + (size_t)h * g) * D, qbytes, &qfull[k]);
+              info[s].n = n;
+              if (n >= 0) {
+                mbar_arrive_expect_tx(&full[s], 2u * S::kTile);
+                const int h = bh % p.Hkv;
+                uint8_t* kdst = ring + s * 2 * S::kTile;
+                uint8_t* vdst = kdst + S::kTile;
+                int c1, c2, c3;
+                tile_coords(p.k_perm, kt, h, kb, c1, c2, c3);
+  #pragma unroll
+                for (int bx = 0; bx < S::kNBox; ++bx)
+                  tma_load_4d_hint(kdst + bx * S::kBox, &tmK, &full[s], bx * 64, c1, c2, c3, stream_pol);
+                tile_coords(p.v_perm, vt, h, vb, c1, c2, c3);
+  #pragma unroll
+                for (int bx = 0; bx < S::kNBox; ++bx)
+                  tma_load_4d_hint(vdst + bx * S::kBox, &tmV, &full[s], bx * 64, c1, c2, c3, stream_pol);
+              } else {
+                mbar_arrive(&full[s]);
+              }
+              issued[s] = issued[s] + 1;
             }
-            ++nq;
           }
-          const int s = it % STAGES;
-          if (!sh[0] && it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) - 1) & 1)) {
-            report(p.err, SEER_DEVERR_TIMEOUT);
-            sh[0] = 1;
-          }
-          if (!sh[0]) {
-            info[s].n = n;
-            if (n >= 0) {
-              mbar_arrive_expect_tx(&full[s], 2u * S::kTile);
-              const int h = bh % p.Hkv;
-              uint8_t* kdst = ring + s * 2 * S::kTile;
-              uint8_t* vdst = kdst + S::kTile;
-              int c1, c2, c3;
-              tile_coords(p.k_perm, kt, h, kb, c1, c2, c3);
-#pragma unroll
-              for (int bx = 0; bx < S::kNBox; ++bx)
-                tma_load_4d_hint(kdst + bx * S::kBox, &tmK, &full[s], bx * 64, c1, c2, c3, stream_pol);
-              tile_coords(p.v_perm, vt, h, vb, c1, c2, c3);
-#pragma unroll
-              for (int bx = 0; bx < S::kNBox; ++bx)
-                tma_load_4d_hint(vdst + bx * S::kBox, &tmV, &full[s], bx * 64, c1, c2, c3, stream_pol);
-            } else {
-              mbar_arrive(&full[s]);
-            }
-            issued[s] = issued[s] + 1;
+          if (__shfl_sync(0xffffffffu, (int)sh[0], 0)) {
+            abort = true;
+            break;
           }
         }
-        if (__shfl_sync(0xffffffffu, (int)sh[0], 0)) {
-          abort = true;
-          break;
-        }
+        cn_ = nn; cb_ = nb; cf_ = nf; ckb = nkb; ckt = nkt; cvb = nvb; cvt = nvt;
+        if (dry) break;
       }
-      cn_ = nn; cb_ = nb; cf_ = nf; ckb = nkb; ckt = nkt; cvb = nvb; cvt = nvt;
     }
     if (lane == 0) {
       __threadfence_block();
