@@ -138,7 +138,9 @@ __device__ __forceinline__ int split_slot(const DecodeParams& p, int bh, int k, 
 
 // Merge the nseg partials (o, lse) of one (b, h) into bf16 out (and lse_out), by the NT threads
 // whose index is `t` (0 <= t < NT).  `wsc` is shared scratch of >= kEpi + 2*kMaxGroup floats;
-// `sync()` is a barrier among those NT threads.  Partials are read with L2-coherent loads.
+// `sync()` is a barrier among those NT threads.  Partials are read with L2-coherent loads, four
+// channels at a time; the outputs of the first MAXS pieces are requested together with every
+// piece's LSE (one round trip up to MAXS pieces), and each piece's weight is formed once per head.
 template <int D, int NT, int kEpi, typename Sync>
 __device__ void merge_partials(const DecodeParams& p, int bh, int nseg, int slot_first, int cf, int t, float* wsc,
                                Sync sync) {
@@ -146,98 +148,85 @@ __device__ void merge_partials(const DecodeParams& p, int bh, int nseg, int slot
   const int b = bh / p.Hkv, h = bh - b * p.Hkv;
   const size_t qh0 = (size_t)b * p.Hq + (size_t)h * g;
   const int ng = nseg * g;
-  constexpr int EPT = (kMaxGroup * D + NT - 1) / NT;
-  constexpr int MAXS = 4;   // pieces whose partial outputs are loaded together with the LSEs
-  constexpr bool kRegs = EPT <= 8;   // the outputs of MAXS pieces fit in registers (NT >= 128)
-  if (kRegs && nseg <= MAXS && ng <= kEpi) {
-    // one round trip: every piece's LSEs and this thread's outputs are requested at once
-    float ov[MAXS][kRegs ? EPT : 1];
-#pragma unroll
-    for (int k = 0; k < MAXS; ++k) {
-      const size_t sl = (size_t)split_slot(p, bh, k < nseg ? k : 0, slot_first, cf);
-#pragma unroll
-      for (int u = 0; u < EPT; ++u) {
-        const int e = u * NT + t;
-        const int j = e / D;
-        if (kRegs) ov[k][kRegs ? u : 0] = (k < nseg && e < g * D) ? __ldcg(p.o_part + (sl * g + j) * D + (e - j * D)) : 0.f;
-      }
-    }
-    float* Mh = wsc + kEpi;
-    float* Zh = Mh + kMaxGroup;
-    for (int i = t; i < ng; i += NT)
-      wsc[i] = __ldcg(p.lse_part + (size_t)split_slot(p, bh, i / g, slot_first, cf) * g + (i % g));
-    sync();
-    if (t < g) {
-      float M = -INFINITY;
-      for (int k = 0; k < nseg; ++k) M = fmaxf(M, wsc[k * g + t]);
-      float Z = 0.f;
-      if (M != -INFINITY)
-        for (int k = 0; k < nseg; ++k) Z += expf(wsc[k * g + t] - M);
-      Mh[t] = M;
-      Zh[t] = Z;
-    }
-    sync();
-#pragma unroll
-    for (int u = 0; u < EPT; ++u) {
-      const int e = u * NT + t;
-      if (e < g * D) {
-        const int j = e / D, cc = e - j * D;
-        const float M = Mh[j], Z = Zh[j];
-        float acc = 0.f;
-        if (M != -INFINITY && Z > 0.f) {
-#pragma unroll
-          for (int k = 0; k < MAXS; ++k)
-            if (k < nseg) acc += expf(wsc[k * g + j] - M) / Z * ov[k][kRegs ? u : 0];
-        }
-        __nv_bfloat16 ob = __float2bfloat16_rn(acc);
-        p.out[(qh0 + j) * D + cc] = *reinterpret_cast<uint16_t*>(&ob);
-        if (cc == 0 && p.lse_out) p.lse_out[qh0 + j] = Z > 0.f ? M + logf(Z) : -INFINITY;
-      }
-    }
-  } else if (ng <= kEpi) {
-    // partial LSEs -> shared; per-head max and weight sum; weights w[k][j] = exp(lse - M) / Z
-    float* Mh = wsc + kEpi;
-    float* Zh = Mh + kMaxGroup;
-    for (int i = t; i < ng; i += NT)
-      wsc[i] = __ldcg(p.lse_part + (size_t)split_slot(p, bh, i / g, slot_first, cf) * g + (i % g));
-    sync();
-    if (t < g) {
-      float M = -INFINITY;
-      for (int k = 0; k < nseg; ++k) M = fmaxf(M, wsc[k * g + t]);
-      float Z = 0.f;
-      if (M != -INFINITY)
-        for (int k = 0; k < nseg; ++k) Z += expf(wsc[k * g + t] - M);
-      Mh[t] = M;
-      Zh[t] = Z;
-    }
-    sync();
-    for (int i = t; i < ng; i += NT) {
-      const int j = i % g;
-      const float M = Mh[j], Z = Zh[j];
-      wsc[i] = (M != -INFINITY && Z > 0.f) ? expf(wsc[i] - M) / Z : 0.f;
-    }
-    sync();
-    float acc[EPT];
-#pragma unroll
-    for (int u = 0; u < EPT; ++u) acc[u] = 0.f;
-    for (int k = 0; k < nseg; ++k) {
+  constexpr int G4 = kMaxGroup * D / 4;              // float4 groups of the largest query group
+  constexpr int EPT4 = (G4 + NT - 1) / NT;           // per thread
+  constexpr int MAXS = EPT4 <= 2 ? 4 : 2;            // pieces whose outputs are requested together
+  const int n4 = g * D / 4;
+  if (ng <= kEpi) {
+    auto load = [&](int k, int u) {
+      const int q4 = u * NT + t;
+      if (k >= nseg || q4 >= n4) return make_float4(0.f, 0.f, 0.f, 0.f);
+      const int j = (4 * q4) / D, cc = 4 * q4 - j * D;
       const size_t sl = (size_t)split_slot(p, bh, k, slot_first, cf);
+      return __ldcg(reinterpret_cast<const float4*>(p.o_part + (sl * g + j) * D + cc));
+    };
+    float4 ov[MAXS][EPT4];
 #pragma unroll
-      for (int u = 0; u < EPT; ++u) {
-        const int e = u * NT + t;
-        if (e < g * D) {
-          const int j = e / D;
-          acc[u] += wsc[k * g + j] * __ldcg(p.o_part + (sl * g + j) * D + (e - j * D));
+    for (int k = 0; k < MAXS; ++k)
+#pragma unroll
+      for (int u = 0; u < EPT4; ++u) ov[k][u] = load(k, u);
+    float* Mh = wsc + kEpi;
+    float* Zh = Mh + kMaxGroup;
+    for (int i = t; i < ng; i += NT)
+      wsc[i] = __ldcg(p.lse_part + (size_t)split_slot(p, bh, i / g, slot_first, cf) * g + (i % g));
+    sync();
+    // per head: the largest LSE, the weight sum and, in place, each piece's weight
+    if (t < g) {
+      float M = -INFINITY;
+      for (int k = 0; k < nseg; ++k) M = fmaxf(M, wsc[k * g + t]);
+      float Z = 0.f;
+      if (M != -INFINITY)
+        for (int k = 0; k < nseg; ++k) Z += expf(wsc[k * g + t] - M);
+      const float inv = Z > 0.f ? 1.f / Z : 0.f;
+      for (int k = 0; k < nseg; ++k) wsc[k * g + t] = Z > 0.f ? expf(wsc[k * g + t] - M) * inv : 0.f;
+      Mh[t] = M;
+      Zh[t] = Z;
+    }
+    sync();
+    float4 acc[EPT4];
+#pragma unroll
+    for (int u = 0; u < EPT4; ++u) {
+      acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      const int q4 = u * NT + t;
+      const int j = q4 < n4 ? (4 * q4) / D : 0;
+#pragma unroll
+      for (int k = 0; k < MAXS; ++k) {
+        const float w = k < nseg ? wsc[k * g + j] : 0.f;
+        acc[u].x += w * ov[k][u].x;
+        acc[u].y += w * ov[k][u].y;
+        acc[u].z += w * ov[k][u].z;
+        acc[u].w += w * ov[k][u].w;
+      }
+    }
+    // pieces past the first MAXS (another round trip per MAXS of them)
+    for (int k0 = MAXS; k0 < nseg; k0 += MAXS) {
+#pragma unroll
+      for (int k = 0; k < MAXS; ++k)
+#pragma unroll
+        for (int u = 0; u < EPT4; ++u) ov[k][u] = load(k0 + k, u);
+#pragma unroll
+      for (int u = 0; u < EPT4; ++u) {
+        const int q4 = u * NT + t;
+        const int j = q4 < n4 ? (4 * q4) / D : 0;
+#pragma unroll
+        for (int k = 0; k < MAXS; ++k) {
+          const float w = k0 + k < nseg ? wsc[(k0 + k) * g + j] : 0.f;
+          acc[u].x += w * ov[k][u].x;
+          acc[u].y += w * ov[k][u].y;
+          acc[u].z += w * ov[k][u].z;
+          acc[u].w += w * ov[k][u].w;
         }
       }
     }
 #pragma unroll
-    for (int u = 0; u < EPT; ++u) {
-      const int e = u * NT + t;
-      if (e < g * D) {
-        const int j = e / D, cc = e - j * D;
-        __nv_bfloat16 ob = __float2bfloat16_rn(acc[u]);
-        p.out[(qh0 + j) * D + cc] = *reinterpret_cast<uint16_t*>(&ob);
+    for (int u = 0; u < EPT4; ++u) {
+      const int q4 = u * NT + t;
+      if (q4 < n4) {
+        const int j = (4 * q4) / D, cc = 4 * q4 - j * D;
+        uint2 pk;
+        pk.x = pack_bf16(acc[u].x, acc[u].y);
+        pk.y = pack_bf16(acc[u].z, acc[u].w);
+        *reinterpret_cast<uint2*>(p.out + (qh0 + j) * D + cc) = pk;
         if (cc == 0 && p.lse_out) p.lse_out[qh0 + j] = Zh[j] > 0.f ? Mh[j] + logf(Zh[j]) : -INFINITY;
       }
     }
