@@ -57,8 +57,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="skip the sparsity sweep rows")
     ap.add_argument("--cpu-sample", type=int, default=16, help="(b, h) pairs in the oracle sample")
-    ap.add_argument("--only", default="all", choices=["all", "decode"],
-                    help="decode: run just the sparse-decode launches (a small target for profilers)")
+    ap.add_argument("--only", default="all", choices=["all", "decode", "truth"],
+                    help="decode / truth: run just the sparse-decode / ground-truth launches (small targets "
+                         "for profilers)")
     return ap.parse_args()
 
 
@@ -96,15 +97,15 @@ def _peaks():
         return 6650.0, "fallback"
 
 
-def _profiled_traffic():
-    """DRAM bytes (read + write) per launch of the decode kernel from the committed ncu summary,
-    or None when the kernel source has changed since those counters were taken."""
+def _profiled_traffic(summary="sparse_decode_kernel.qwen3-8b-32k-decode.md", source="sparse_decode.cu"):
+    """DRAM bytes (read + write) per launch of a kernel from its committed ncu summary, or None
+    when the kernel source has changed since those counters were taken."""
     import hashlib
     try:
-        with open(os.path.join(ROOT, "profiles", "sparse_decode_kernel.qwen3-8b-32k-decode.md")) as f:
+        with open(os.path.join(ROOT, "profiles", summary)) as f:
             fields = dict(line.split(": ", 1) for line in f.read().splitlines() if ": " in line
                           and line.split(": ", 1)[0] in ("source_sha256", "traffic_bytes_per_launch"))
-        with open(os.path.join(ROOT, "block_sparse_attention_attngate_b200", "csrc", "sparse_decode.cu"), "rb") as f:
+        with open(os.path.join(ROOT, "block_sparse_attention_attngate_b200", "csrc", source), "rb") as f:
             current = hashlib.sha256(f.read()).hexdigest()
         if fields.get("source_sha256", "").strip() != current:
             return None
@@ -320,6 +321,7 @@ def sweep_rows(S, dev, stream, peak, shape2, reps2, seqlens2, cfg2, inp2, iters=
     t_bytes = k_bytes + cfg2.B * cfg2.Hq * cfg2.head_dim * 2 + cfg2.B * cfg2.Hkv * inp2.max_blocks * 4
     res["ground-truth-32k"] = {"us": us_t, "bytes": t_bytes, "achieved_gbs": t_bytes / (us_t * 1e-6) / 1e9,
                                "frac": t_bytes / (us_t * 1e-6) / 1e9 / peak,
+                               "traffic": _profiled_traffic("truth_kernel.qwen3-8b-32k-ground-truth.md", "gate_truth.cu"),
                                "what": "seer_gate_truth: all of K read once (K bytes + q + scores)"}
     del ws_t, sc_t
     # config 2 at k = 52
@@ -427,6 +429,17 @@ def run_seer(args):
         stream.synchronize()
         if rank == 0:
             print(json.dumps({"only": "decode", "launches": args.warmup + args.steps, "replicas": R}), flush=True)
+        return 0
+    if args.only == "truth":
+        ws_t = S.alloc_truth_workspace(shape, dev)
+        sc_t = torch.empty(B, Hkv, NB, dtype=torch.float32, device=dev)
+        with torch.cuda.stream(stream):
+            for i in range(args.warmup + args.steps):
+                S.gate_truth(shape, reps[i % R]["q"], S.KVCache.contiguous(reps[i % R]["k"]), seqlens, sc_t, ws_t,
+                             stream=stream)
+        stream.synchronize()
+        if rank == 0:
+            print(json.dumps({"only": "truth", "launches": args.warmup + args.steps, "replicas": R}), flush=True)
         return 0
     # warm once eagerly (first-call set-up happens outside capture), then capture one graph per replica
     with torch.cuda.stream(stream):
