@@ -129,6 +129,38 @@ def kcomp_update(k_nope: np.ndarray, length: int, valid: int, w_k: np.ndarray,
     return nfull
 
 
+def kcomp_append(state: np.ndarray, k_new: np.ndarray, length: int, valid: int, w_k: np.ndarray,
+                 kcomp: np.ndarray, block: int, base: float) -> int:
+    """The same cache update, one appended token at a time, from running block statistics.
+
+    The cache is updated once every b generated tokens from the latest b keys [CP Knowl 5], so a
+    decoder only needs those keys' per-channel max, min and sum, not a pre-RoPE copy of the whole
+    context.  `k_new` [d] is the pre-RoPE key of token length-1; `state` [3, d] holds the running
+    max / min / sum of the current block's keys (restarted at a block's first token).  When the
+    token completes block n, kcomp[n] = bf16(RoPE_{n*b}(W_k . [max | min | sum/b])) and the fill
+    count becomes n+1 (the block's earlier entries must already be there: valid == n).
+    Returns the new fill count.
+    """
+    if length <= 0:
+        return valid
+    n, pos = divmod(length - 1, block)
+    k = np.asarray(k_new, dtype=np.float64)
+    if pos == 0:
+        state[0], state[1], state[2] = k, k, k
+    else:
+        state[0] = np.maximum(state[0], k)
+        state[1] = np.minimum(state[1], k)
+        state[2] = state[2] + k
+    if pos != block - 1:
+        return valid
+    if valid != n:
+        raise ValueError(f"block {n} completes with {valid} entries present")
+    pooled = np.concatenate([state[0], state[1], state[2] / block])
+    y = np.asarray(w_k, dtype=np.float64) @ pooled
+    kcomp[n] = round_to_bf16(rope(y, n * block, base))
+    return n + 1
+
+
 def q_gate(q_nope: np.ndarray, w_q: np.ndarray, length: int, base: float) -> np.ndarray:
     """Gate query of one KV head: RoPE_{L-1}(W_q . reshape(q_group, [g*d])).
 

@@ -378,6 +378,31 @@ def check_kcomp_incremental():
         assert np.array_equal(cache[n], O.k_gate_entry(keys[n * b:(n + 1) * b], wk, n, b, 1e4))
 
 
+def check_kcomp_append_matches_rebuild():
+    """Token-by-token appends from running max/min/sum give the block-pooling cache exactly
+    (max and min exactly; the sum/b average within fp64 rounding), each entry appearing when its
+    block's last token arrives; a block first token restarts the statistics."""
+    rng = np.random.default_rng(15)
+    for d, dg, b, Lmax in ((4, 6, 8, 45), (3, 4, 5, 23)):
+        keys = rng.standard_normal((Lmax, d))
+        wk = rng.standard_normal((dg, 3 * d))
+        cache = np.full((Lmax // b + 1, dg), np.nan)
+        state = np.full((3, d), 1e9)             # garbage: the first token must restart it
+        valid = 0
+        for L in range(1, Lmax + 1):
+            valid = O.kcomp_append(state, keys[L - 1], L, valid, wk, cache, b, 1e4)
+            assert valid == L // b, f"fill count at L={L}"
+            blk = keys[(L - 1) // b * b:L]
+            _close(state[0], blk.max(0), 0, "running max")
+            _close(state[1], blk.min(0), 0, "running min")
+            _close(state[2], blk.sum(0), 1e-12, "running sum")
+        rebuilt = np.full_like(cache, np.nan)
+        O.kcomp_update(keys, Lmax, 0, wk, rebuilt, b, 1e4)
+        nf = Lmax // b
+        assert np.array_equal(np.isnan(cache), np.isnan(rebuilt)), "entries present differ"
+        _close(cache[:nf], rebuilt[:nf], 2.0 ** -7, "rolling vs rebuild")
+
+
 def check_memory_ratio():
     """K Compression Cache = 1/128 of the KV cache at b=64 with d_gate = d, same element size."""
     b, d, dg, L = 64, 128, 128, 65536

@@ -103,6 +103,31 @@ def _gt_mean_over_group(q, k, length, block, scale):
     return gt / gt.sum()
 
 
+def _append_no_restart(state, k_new, length, valid, w_k, kcomp, block, base):
+    n, pos = divmod(length - 1, block)
+    k = np.asarray(k_new, float)
+    state[0] = np.maximum(state[0], k); state[1] = np.minimum(state[1], k); state[2] = state[2] + k
+    if pos != block - 1:
+        return valid
+    y = np.asarray(w_k, float) @ np.concatenate([state[0], state[1], state[2] / block])
+    kcomp[n] = O.round_to_bf16(O.rope(y, n * block, base))
+    return n + 1
+
+
+def _append_rope_at_last(state, k_new, length, valid, w_k, kcomp, block, base):
+    n, pos = divmod(length - 1, block)
+    k = np.asarray(k_new, float)
+    if pos == 0:
+        state[0], state[1], state[2] = k, k, k
+    else:
+        state[0] = np.maximum(state[0], k); state[1] = np.minimum(state[1], k); state[2] = state[2] + k
+    if pos != block - 1:
+        return valid
+    y = np.asarray(w_k, float) @ np.concatenate([state[0], state[1], state[2] / block])
+    kcomp[n] = O.round_to_bf16(O.rope(y, length - 1, base))
+    return n + 1
+
+
 ATTEND = O.attend
 
 MUTANTS = {
@@ -120,6 +145,8 @@ MUTANTS = {
     "attention_scale": ("attend", _attend_noscale),
     "combine_weights": ("combine", _combine_linear),
     "gt_group_mean": ("decode_ground_truth", _gt_mean_over_group),
+    "append_no_restart": ("kcomp_append", _append_no_restart),
+    "append_rope_position": ("kcomp_append", _append_rope_at_last),
 }
 
 
