@@ -533,6 +533,27 @@ def run_seer(args):
 
     kcomp_fill_us = part(run_kcomp_fill)
 
+    # the cache from running block statistics (no pre-RoPE context copy): a step that folds one
+    # key per (b, h) into the statistics, and one whose token completes a block for every (b, h)
+    app_state = S.alloc_kcomp_state(shape, dev)
+    app_knew = torch.randn(B, Hkv, d, device=dev).to(torch.bfloat16)
+    app_mid = torch.full((B,), (NB - 1) * blk + 5, dtype=torch.int32, device=dev)
+    app_end = torch.full((B,), NB * blk, dtype=torch.int32, device=dev)
+    app_valid = torch.full((args.warmup + args.steps + 1, B, Hkv), NB - 1, dtype=torch.int32, device=dev)
+    app_row = [0]
+    app_kc = torch.zeros_like(reps[0]["step"].kcomp)   # its own cache: the step's stays as it is
+
+    def run_append_fold(i):
+        S.kcomp_append(shape, app_knew, app_mid, app_state, app_valid[0], w_k, app_kc, stream=stream)
+
+    def run_append_fill(i):
+        row = app_valid[app_row[0] % app_valid.shape[0]]
+        app_row[0] += 1
+        S.kcomp_append(shape, app_knew, app_end, app_state, row, w_k, app_kc, stream=stream)
+
+    append_fold_us = part(run_append_fold)
+    append_fill_us = part(run_append_fill)
+
     # ---------------- dense path: every block of every (b, h), same kernel
     dense_idx = torch.arange(NB, dtype=torch.int32, device=dev).expand(B, Hkv, NB).contiguous()
     dense_cnt = torch.full((B, Hkv), NB, dtype=torch.int32, device=dev)
@@ -657,6 +678,7 @@ def run_seer(args):
                          f"per rotation > 126 MB L2)", "parallelism": f"dp{world} (independent batches)"},
         "parts_us": {"decode_plan": plan_us, "sparse_decode": decode_us,
                      "unfused": {"kcomp_update_noop": kcomp_noop_us, "kcomp_update_fill": kcomp_fill_us,
+                                 "kcomp_append_fold": append_fold_us, "kcomp_append_fill": append_fill_us,
                                  "gate_score": gate_us, "select_blocks": select_us}},
         "dense_path_us": dense_us, "speedup_vs_dense": dense_us / decode_us,
         "bytes": {"decode_algorithmic": nbytes["decode"], "step_algorithmic": nbytes["step"]},

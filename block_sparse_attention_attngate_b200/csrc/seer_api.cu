@@ -344,6 +344,59 @@ seer_status seer_kcomp_update(const seer_dims_t* dims, const seer_kv_t* k_nope, 
   return SEER_OK;
 }
 
+size_t seer_kcomp_state_bytes(const seer_dims_t* dims) {
+  if (check_dims(dims) != SEER_OK) return 0;
+  return (size_t)dims->batch * dims->num_kv_heads * 3 * dims->head_dim * sizeof(float);
+}
+
+seer_status seer_kcomp_append(const seer_dims_t* dims, const void* k_new, const int32_t* seqlens, float* state,
+                              int32_t* valid_blocks, const void* w_k, void* kcomp, int32_t* err_word,
+                              void* stream) {
+  seer_status st = check_dims(dims);
+  if (st != SEER_OK) return st;
+  if (!k_new || !seqlens || !state || !valid_blocks || !w_k || !kcomp)
+    return fail(SEER_ERR_INVALID_ARG, "NULL pointer argument");
+  if (!aligned16(k_new) || !aligned16(state) || !aligned16(w_k) || !aligned16(kcomp))
+    return fail(SEER_ERR_INVALID_ARG, "k_new / state / w_k / kcomp not 16-byte aligned");
+  seer::AppendParams p{};
+  rope_thetas(dims, p.theta);
+  p.k_new = static_cast<const uint16_t*>(k_new);
+  p.seqlens = seqlens;
+  p.valid = valid_blocks;
+  p.state = state;
+  p.w_k = static_cast<const uint16_t*>(w_k);
+  p.kcomp = static_cast<uint16_t*>(kcomp);
+  p.B = dims->batch;
+  p.Hkv = dims->num_kv_heads;
+  p.NB = dims->max_blocks;
+  p.err = err_word;
+  cudaError_t e = seer::launch_kcomp_append(p, dims->head_dim, dims->block_size, dims->gate_dim,
+                                            static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "kcomp_append launch");
+  return SEER_OK;
+}
+
+seer_status seer_kcomp_state_init(const seer_dims_t* dims, const seer_kv_t* k_nope, const int32_t* seqlens,
+                                  float* state, int32_t* err_word, void* stream) {
+  seer_status st = check_dims(dims);
+  if (st != SEER_OK) return st;
+  if ((st = check_kv(dims, k_nope, "k_nope")) != SEER_OK) return st;
+  if (!seqlens || !state) return fail(SEER_ERR_INVALID_ARG, "NULL pointer argument");
+  if (!aligned16(state)) return fail(SEER_ERR_INVALID_ARG, "state not 16-byte aligned");
+  seer::AppendParams p{};
+  p.k = plain(k_nope);
+  p.seqlens = seqlens;
+  p.state = state;
+  p.B = dims->batch;
+  p.Hkv = dims->num_kv_heads;
+  p.NB = dims->max_blocks;
+  p.err = err_word;
+  cudaError_t e = seer::launch_kcomp_state_init(p, dims->head_dim, dims->block_size,
+                                                static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "kcomp_state_init launch");
+  return SEER_OK;
+}
+
 seer_status seer_gate_score(const seer_dims_t* dims, const void* q_nope, const void* w_q, const void* kcomp,
                             const int32_t* seqlens, float* logits, float* q_gate_out, void* stream) {
   seer_status st = check_dims(dims);

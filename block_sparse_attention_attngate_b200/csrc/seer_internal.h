@@ -77,6 +77,22 @@ struct KcompParams {
 cudaError_t launch_kcomp_update(const KcompParams& p, int D, int BLK, int DG, int grid_x,
                                 cudaStream_t s);
 
+// ---------------------------------------------------------------- cache from running block statistics
+struct AppendParams {
+  double theta[kMaxHalfGate];   // base^(-2i/d_gate), computed on the host in fp64
+  const uint16_t* k_new;   // [B, Hkv, D] pre-RoPE key of token seqlens[b]-1 (append)
+  KvPlain k;               // pre-RoPE key cache (state init)
+  const int32_t* seqlens;
+  int32_t* valid;          // [B, Hkv] fill counts, read and advanced
+  float* state;            // [B, Hkv, 3, D] running max / min / sum of the current block
+  const uint16_t* w_k;     // [Hkv, DG, 3D]
+  uint16_t* kcomp;         // [B, Hkv, NB, DG]
+  int32_t B, Hkv, NB;
+  int32_t* err;
+};
+cudaError_t launch_kcomp_append(const AppendParams& p, int D, int BLK, int DG, cudaStream_t s);
+cudaError_t launch_kcomp_state_init(const AppendParams& p, int D, int BLK, cudaStream_t s);
+
 // ---------------------------------------------------------------- gate score
 struct GateParams {
   double theta[kMaxHalfGate];   // base^(-2i/d_gate), computed on the host in fp64

@@ -27,7 +27,7 @@ SELECT_TOPK, SELECT_THRESHOLD, SELECT_TOPP = 0, 1, 2
 DEVERR_BLOCK_INDEX, DEVERR_PAGE_INDEX, DEVERR_COUNT, DEVERR_TIMEOUT = 1, 2, 4, 8
 
 EXPORTED = (
-    "seer_kcomp_update", "seer_gate_score", "seer_select_blocks", "seer_decode_plan", "seer_sparse_decode_auto_split",
+    "seer_kcomp_update", "seer_kcomp_state_bytes", "seer_kcomp_append", "seer_kcomp_state_init", "seer_gate_score", "seer_select_blocks", "seer_decode_plan", "seer_sparse_decode_auto_split",
     "seer_sparse_decode_workspace_bytes", "seer_sparse_decode", "seer_sparse_decode_noalloc",
     "seer_gate_truth_workspace_bytes", "seer_gate_truth", "seer_last_error", "seer_version",
 )
@@ -60,6 +60,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     DP, KP = ctypes.POINTER(Dims), ctypes.POINTER(KVDesc)
     sig = {
         "seer_kcomp_update": (I32, [DP, KP, P, P, P, P, P]),
+        "seer_kcomp_state_bytes": (SZ, [DP]),
+        "seer_kcomp_append": (I32, [DP, P, P, P, P, P, P, P, P]),
+        "seer_kcomp_state_init": (I32, [DP, KP, P, P, P, P]),
         "seer_gate_score": (I32, [DP, P, P, P, P, P, P, P]),
         "seer_select_blocks": (I32, [DP, P, P, I32, I32, F32, P, P, I32, P]),
         "seer_decode_plan": (I32, [DP, KP, P, P, P, P, P, P, P, P, I32, I32, F32, P, P, I32, P]),
@@ -168,6 +171,42 @@ def kcomp_update(shape: Shape, k_nope: KVCache, seqlens: torch.Tensor, valid_blo
     dims = shape.c()
     _check(_lib.seer_kcomp_update(ctypes.byref(dims), ctypes.byref(k_nope.desc), _ptr(seqlens),
                                   _ptr(valid_blocks), _ptr(w_k), _ptr(kcomp), _stream(stream)))
+
+
+def kcomp_state_bytes(shape: Shape) -> int:
+    dims = shape.c()
+    return int(_lib.seer_kcomp_state_bytes(ctypes.byref(dims)))
+
+
+def alloc_kcomp_state(shape: Shape, device=None) -> torch.Tensor:
+    """Running block statistics for kcomp_append: fp32 [B, Hkv, 3, d] (max, min, sum)."""
+    return torch.zeros((shape.batch, shape.num_kv_heads, 3, shape.head_dim), dtype=torch.float32, device=device or "cuda")
+
+
+def kcomp_append(shape: Shape, k_new: torch.Tensor, seqlens: torch.Tensor, state: torch.Tensor,
+                 valid_blocks: torch.Tensor, w_k: torch.Tensor, kcomp: torch.Tensor,
+                 err: Optional[torch.Tensor] = None, stream=None):
+    """Fold each sequence's appended pre-RoPE key [B, Hkv, d] into the running block statistics;
+    a completed block writes its K Compression Cache entry (see seer_kcomp_append)."""
+    _need(k_new, torch.bfloat16, "k_new")
+    _need(seqlens, torch.int32, "seqlens")
+    _need(state, torch.float32, "state")
+    _need(valid_blocks, torch.int32, "valid_blocks")
+    _need(w_k, torch.bfloat16, "w_k")
+    _need(kcomp, torch.bfloat16, "kcomp")
+    dims = shape.c()
+    _check(_lib.seer_kcomp_append(ctypes.byref(dims), _ptr(k_new), _ptr(seqlens), _ptr(state), _ptr(valid_blocks),
+                                  _ptr(w_k), _ptr(kcomp), _ptr(err) if err is not None else None, _stream(stream)))
+
+
+def kcomp_state_init(shape: Shape, k_nope: KVCache, seqlens: torch.Tensor, state: torch.Tensor,
+                     err: Optional[torch.Tensor] = None, stream=None):
+    """Prime the running block statistics from the key cache (see seer_kcomp_state_init)."""
+    _need(seqlens, torch.int32, "seqlens")
+    _need(state, torch.float32, "state")
+    dims = shape.c()
+    _check(_lib.seer_kcomp_state_init(ctypes.byref(dims), ctypes.byref(k_nope.desc), _ptr(seqlens), _ptr(state),
+                                      _ptr(err) if err is not None else None, _stream(stream)))
 
 
 def gate_score(shape: Shape, q_nope: torch.Tensor, w_q: torch.Tensor, kcomp: torch.Tensor, seqlens: torch.Tensor,
@@ -312,17 +351,23 @@ class DecodeStep:
 
     Owns the step's scratch tensors (logits, index lists, workspace, output) so a
     decode loop (or a CUDA graph capturing `run`) reuses them every step.
+
+    With `kcomp_state` (alloc_kcomp_state; primed by kcomp_state_init when the sequences resume
+    mid-block) the K Compression Cache is kept from running block statistics: each `run` takes
+    the appended tokens' pre-RoPE keys `k_new` [B, Hkv, d] and no pre-RoPE copy of the context
+    is read (kcomp_append, then the plan without its cache update).
     """
 
     def __init__(self, shape: Shape, k: KVCache, v: KVCache, w_q: torch.Tensor, w_k: torch.Tensor,
                  kcomp: torch.Tensor, valid_blocks: torch.Tensor, mode: int = SELECT_TOPK, token_budget: int = 0,
                  tau: float = 0.0, capacity: Optional[int] = None, num_split: Optional[int] = None,
-                 k_nope: Optional[KVCache] = None,
+                 k_nope: Optional[KVCache] = None, kcomp_state: Optional[torch.Tensor] = None,
                  device=None):
         dev = device or w_q.device
         self.shape, self.k, self.v, self.w_q, self.w_k = shape, k, v, w_q, w_k
         self.k_nope = k_nope or k
         self.kcomp, self.valid_blocks = kcomp, valid_blocks
+        self.kcomp_state = kcomp_state
         self.mode, self.token_budget, self.tau = mode, token_budget, tau
         if capacity is None:
             if mode == SELECT_TOPK:
@@ -345,12 +390,20 @@ class DecodeStep:
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
 
     def run(self, q: torch.Tensor, seqlens: torch.Tensor, q_nope: Optional[torch.Tensor] = None, stream=None,
-            fused: bool = True):
+            fused: bool = True, k_new: Optional[torch.Tensor] = None):
         """One decode step.  fused=True plans with seer_decode_plan (one launch); fused=False makes
-        the three separate calls (kcomp_update, gate_score, select_blocks) instead."""
+        the three separate calls (kcomp_update, gate_score, select_blocks) instead.  With running
+        block statistics (kcomp_state), `k_new` holds the appended tokens' pre-RoPE keys."""
         s = self.shape
         qn = q if q_nope is None else q_nope
-        if fused:
+        if self.kcomp_state is not None:
+            if k_new is None:
+                raise ValueError("a step with running block statistics needs k_new, the appended pre-RoPE keys")
+            kcomp_append(s, k_new, seqlens, self.kcomp_state, self.valid_blocks, self.w_k, self.kcomp, self.err,
+                         stream)
+            decode_plan(s, seqlens, self.kcomp, qn, self.w_q, self.mode, self.block_idx, self.block_cnt,
+                        self.token_budget, self.tau, logits=self.logits, stream=stream)
+        elif fused:
             decode_plan(s, seqlens, self.kcomp, qn, self.w_q, self.mode, self.block_idx, self.block_cnt,
                         self.token_budget, self.tau, k_nope=self.k_nope, valid_blocks=self.valid_blocks, w_k=self.w_k,
                         logits=self.logits, stream=stream)

@@ -124,6 +124,54 @@ seer_status seer_kcomp_update(const seer_dims_t* dims, const seer_kv_t* k_nope,
                               void* kcomp, void* stream);
 
 /*
+ * seer_kcomp_append -- the same cache update from running block statistics, one appended
+ * token per sequence and call [CP Knowl 2, Knowl 5: the cache updates once every b generated
+ * tokens from the latest b keys, so their per-channel max, min and sum are all it needs].
+ *
+ * Each sequence b has just appended token t = seqlens[b] - 1 (seqlens after the append;
+ * seqlens[b] <= 0: nothing appended, nothing done).  With n = floor(t / b), i = t mod b and
+ * x = k_new[b, h, :]:
+ *   i == 0:  state[b, h] = (x, x, x)                                   (the block restarts)
+ *   i  > 0:  state[b, h] = (max(state.max, x), min(state.min, x), state.sum + x)
+ *   i == b-1 (the token completes block n):
+ *            kcomp[b, h, n, :] = bf16( RoPE_{n*b}( W_k[h] . [max | min | sum/b] ) )
+ *            valid_blocks[b, h] = n + 1
+ * which equals what seer_kcomp_update computes for block n from the K cache (fp32 sums).  The
+ * completing call requires valid_blocks[b, h] == n and n < max_blocks; otherwise it writes
+ * no entry and ORs SEER_DEVERR_COUNT into *err_word.  No pre-RoPE copy of the context is needed:
+ * the state is 3*d fp32 per (b, h).
+ *
+ *   k_new         device bf16 [B, Hkv, d]: the pre-RoPE keys of the appended tokens
+ *   seqlens       device int32 [B] (after the append)
+ *   state         device fp32 [B, Hkv, 3, d] (running max, min, sum; seer_kcomp_state_bytes);
+ *                 read and written.  A sequence that continues mid-block must have it primed
+ *                 by seer_kcomp_state_init; one at a block boundary needs nothing.
+ *   valid_blocks  device int32 [B, Hkv], read and advanced
+ *   w_k, kcomp    as seer_kcomp_update
+ *   err_word      device int32 or NULL (SEER_DEVERR_* bits ORed in)
+ * One CTA per (b, h).  Calls must be made in token order, one per appended token.
+ */
+size_t seer_kcomp_state_bytes(const seer_dims_t* dims);
+seer_status seer_kcomp_append(const seer_dims_t* dims, const void* k_new, const int32_t* seqlens,
+                              float* state, int32_t* valid_blocks, const void* w_k, void* kcomp,
+                              int32_t* err_word, void* stream);
+
+/*
+ * seer_kcomp_state_init -- prime the running block statistics of seer_kcomp_append from the
+ * key cache: for every (b, h), the per-channel max, min and sum of the pre-RoPE keys of tokens
+ * [floor(L_b / b) * b, L_b) (the current, incomplete block; empty at a block boundary:
+ * -inf, +inf, 0).  Reads at most b - 1 keys per (b, h).  Page or capacity errors set
+ * SEER_DEVERR_PAGE_INDEX / SEER_DEVERR_COUNT in *err_word and leave the empty statistics.
+ *
+ *   k_nope   pre-RoPE key cache (see seer_kv_t)
+ *   seqlens  device int32 [B]
+ *   state    device fp32 [B, Hkv, 3, d], written
+ */
+seer_status seer_kcomp_state_init(const seer_dims_t* dims, const seer_kv_t* k_nope,
+                                  const int32_t* seqlens, float* state, int32_t* err_word,
+                                  void* stream);
+
+/*
  * seer_gate_score -- AttnGate block logits [CP Knowl 1-2; PN design 1].
  *
  *   Q_gate[b, h] = RoPE_{L_b - 1}( W_q[h] . concat_j q_nope[b, h*g + j, :] )   (fp32, not rounded)

@@ -169,6 +169,18 @@ def test_kcomp_and_gate_validation(lib, S):
     assert lib.seer_gate_score(ctypes.byref(d), P, P, P, P, P, ctypes.c_void_p(4097), None) == 1
 
 
+def test_kcomp_append_validation(lib, S):
+    d = _dims(S)
+    k = _kv(S)
+    n = 8 * 8 * 3 * 128 * 4                       # B * Hkv * 3 * d fp32
+    assert lib.seer_kcomp_state_bytes(ctypes.byref(d)) == n
+    assert lib.seer_kcomp_state_bytes(ctypes.byref(_dims(S, head_dim=80))) == 0
+    assert lib.seer_kcomp_append(ctypes.byref(d), P, P, None, P, P, P, None, None) == 1
+    assert lib.seer_kcomp_append(ctypes.byref(d), P, P, ctypes.c_void_p(4100), P, P, P, None, None) == 1
+    assert lib.seer_kcomp_state_init(ctypes.byref(d), ctypes.byref(k), None, P, None, None) == 1
+    assert lib.seer_kcomp_state_init(ctypes.byref(d), ctypes.byref(k), P, ctypes.c_void_p(4100), None, None) == 1
+
+
 def test_missing_library_fails_loudly(tmp_path):
     from block_sparse_attention_attngate_b200 import seer
     with pytest.raises(ImportError):
