@@ -316,6 +316,35 @@ def decode_ground_truth(q: np.ndarray, k: np.ndarray, length: int, block: int,
     return gt / gt.sum()
 
 
+def prefill_ground_truth(q: np.ndarray, k: np.ndarray, v: np.ndarray, block: int,
+                         scale: float) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Causal attention of a whole sequence for one KV head, with the block-level target of
+    every query position beside it (the training-side ground truth [CP Knowl 3, Knowl 4]).
+
+    q: [g, L, d] (the GQA group's query heads), k, v: [L, d].  Query i attends keys 0..i.
+    Returns o [g, L, d], lse [g, L] and gt [L, ceil(L/b)]: row i is the decode target of
+    query position i -- the softmax map's row 1-D max-pooled over each block's (visible)
+    columns, max over the g heads, normalised to sum to 1; blocks past position i are 0.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    kk = np.asarray(k, dtype=np.float64)
+    vv = np.asarray(v, dtype=np.float64)
+    g, L, _ = q.shape
+    s = scale * np.einsum("hid,td->hit", q, kk)
+    visible = np.tril(np.ones((L, L), dtype=bool))
+    s = np.where(visible[None], s, NEG_INF)
+    m = s.max(axis=2, keepdims=True)
+    e = np.exp(s - m)
+    z = e.sum(axis=2, keepdims=True)
+    p = e / z
+    o = np.einsum("hit,td->hid", p, vv)
+    lse = (m + np.log(z))[..., 0]
+    nblk = -(-L // block)
+    pooled = np.stack([p[:, :, n * block:min((n + 1) * block, L)].max(axis=2) for n in range(nblk)], axis=2)
+    gt = pooled.max(axis=0)
+    return o, lse, gt / gt.sum(axis=1, keepdims=True)
+
+
 # ----------------------------------------------------------------------------
 # One whole decode step for one (batch, kv-head)
 # ----------------------------------------------------------------------------

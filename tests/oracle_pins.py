@@ -349,6 +349,50 @@ def check_ground_truth():
     assert gt.shape == (7,) and abs(gt.sum() - 1) < 1e-12 and np.all(gt > 0)
 
 
+def check_prefill_ground_truth():
+    """Prefill target vs three other things: every row i is the (pinned) decode target of query
+    i over keys 0..i; the output is torch's float64 causal attention; and the pages' tile
+    recurrence (per-tile row maxima r, running max m and normaliser l, then exp(r - m) / l)
+    reproduces each head's pooled probabilities before the group max."""
+    import torch
+    rng = np.random.default_rng(16)
+    g, L, d, b = 3, 37, 8, 8
+    q = rng.standard_normal((g, L, d))
+    k = rng.standard_normal((L, d))
+    v = rng.standard_normal((L, d))
+    scale = 0.4
+    o, lse, gt = O.prefill_ground_truth(q, k, v, b, scale)
+    nb = -(-L // b)
+    assert gt.shape == (L, nb)
+    for i in range(L):
+        ref = O.decode_ground_truth(q[:, i], k, i + 1, b, scale)
+        _close(gt[i, :len(ref)], ref, 1e-12, f"row {i}")
+        assert np.all(gt[i, len(ref):] == 0), f"row {i}: blocks past the position"
+    tq = torch.from_numpy(q)[None]
+    ref_o = torch.nn.functional.scaled_dot_product_attention(
+        tq, torch.from_numpy(k)[None, None].expand(1, g, L, d), torch.from_numpy(v)[None, None].expand(1, g, L, d),
+        is_causal=True, scale=scale)[0].numpy()
+    _close(o, ref_o, 1e-10, "causal attention output")
+    for h in range(g):
+        for i in range(L):
+            m, l, r = -math.inf, 0.0, []
+            for n in range(nb):
+                t = np.arange(n * b, min((n + 1) * b, i + 1))
+                if len(t) == 0:
+                    break
+                sij = scale * (k[t] @ q[h, i])
+                rij = sij.max()
+                mn = max(m, rij)
+                l = l * math.exp(m - mn) + np.exp(sij - mn).sum()
+                m = mn
+                r.append(rij)
+            assert abs((m + math.log(l)) - lse[h, i]) < 1e-12, "lse"
+            s_row = scale * (k[:i + 1] @ q[h, i])
+            p_row = np.exp(s_row - s_row.max()) / np.exp(s_row - s_row.max()).sum()
+            pooled = [p_row[n * b:min((n + 1) * b, i + 1)].max() for n in range(len(r))]
+            _close(np.exp(np.array(r) - m) / l, pooled, 1e-12, "tile recurrence")
+
+
 # ---------------------------------------------------------------- K compression cache
 
 def check_kcomp_incremental():

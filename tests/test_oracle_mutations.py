@@ -128,6 +128,29 @@ def _append_rope_at_last(state, k_new, length, valid, w_k, kcomp, block, base):
     return n + 1
 
 
+def _prefill_unmasked(q, k, v, block, scale):
+    q = np.asarray(q, float); kk = np.asarray(k, float); vv = np.asarray(v, float)
+    s = scale * np.einsum("hid,td->hit", q, kk)                  # future keys left visible
+    p = np.exp(s - s.max(2, keepdims=True)); p /= p.sum(2, keepdims=True)
+    L = q.shape[1]; nb = -(-L // block)
+    pooled = np.stack([p[:, :, n * block:min((n + 1) * block, L)].max(2) for n in range(nb)], 2).max(0)
+    return np.einsum("hit,td->hid", p, vv), np.log(np.exp(s).sum(2)), pooled / pooled.sum(1, keepdims=True)
+
+
+def _prefill_norm_then_max(q, k, v, block, scale):
+    o, lse, _ = REAL_PREFILL(q, k, v, block, scale)
+    q = np.asarray(q, float); kk = np.asarray(k, float)
+    g, L, _ = q.shape
+    s = scale * np.einsum("hid,td->hit", q, kk)
+    s = np.where(np.tril(np.ones((L, L), bool))[None], s, -np.inf)
+    p = np.exp(s - s.max(2, keepdims=True)); p /= p.sum(2, keepdims=True)
+    nb = -(-L // block)
+    pooled = np.stack([p[:, :, n * block:min((n + 1) * block, L)].max(2) for n in range(nb)], 2)
+    pooled = pooled / pooled.sum(2, keepdims=True)                # normalised per head first
+    return o, lse, pooled.max(0)
+
+
+REAL_PREFILL = O.prefill_ground_truth
 ATTEND = O.attend
 
 MUTANTS = {
@@ -147,6 +170,8 @@ MUTANTS = {
     "gt_group_mean": ("decode_ground_truth", _gt_mean_over_group),
     "append_no_restart": ("kcomp_append", _append_no_restart),
     "append_rope_position": ("kcomp_append", _append_rope_at_last),
+    "prefill_unmasked": ("prefill_ground_truth", _prefill_unmasked),
+    "prefill_norm_then_max": ("prefill_ground_truth", _prefill_norm_then_max),
 }
 
 
