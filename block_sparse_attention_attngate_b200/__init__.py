@@ -12,7 +12,7 @@ _PUBLIC = (
     "KV_PAGED", "LIB_PATH", "SELECT_THRESHOLD", "SELECT_TOPK", "SELECT_TOPP", "DecodeStep", "Dims", "KVCache",
     "KVDesc", "SeerError", "Shape", "alloc_truth_workspace", "alloc_workspace", "decode_plan", "gate_score",
     "gate_truth", "gate_truth_workspace_bytes", "kcomp_update", "kcomp_append", "kcomp_state_init",
-    "kcomp_state_bytes", "alloc_kcomp_state", "select_blocks",
+    "kcomp_state_bytes", "alloc_kcomp_state", "prefill_gt", "prefill_gt_workspace_bytes", "select_blocks",
     "sparse_decode", "sparse_decode_auto_split", "sparse_decode_noalloc", "sparse_decode_workspace_bytes", "version",
 )
 

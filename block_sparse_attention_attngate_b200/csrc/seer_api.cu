@@ -344,6 +344,59 @@ seer_status seer_kcomp_update(const seer_dims_t* dims, const seer_kv_t* k_nope, 
   return SEER_OK;
 }
 
+size_t seer_prefill_gt_workspace_bytes(const seer_dims_t* dims, int32_t max_len) {
+  if (check_dims(dims) != SEER_OK || max_len < 1) return 0;
+  return (size_t)dims->batch * dims->num_q_heads * dims->max_blocks * (size_t)max_len * sizeof(float);
+}
+
+seer_status seer_prefill_gt(const seer_dims_t* dims, const void* q, int32_t max_len, const seer_kv_t* k,
+                            const seer_kv_t* v, const int32_t* seqlens, void* out, float* lse_out, float* gt,
+                            void* workspace, size_t workspace_bytes, int32_t* err_word, void* stream) {
+  seer_status st = check_dims(dims);
+  if (st != SEER_OK) return st;
+  if ((st = check_kv(dims, k, "k")) != SEER_OK) return st;
+  if ((st = check_kv(dims, v, "v")) != SEER_OK) return st;
+  if (k->layout != SEER_KV_CONTIGUOUS || v->layout != SEER_KV_CONTIGUOUS)
+    return fail(SEER_ERR_UNSUPPORTED, "prefill attention takes contiguous K/V caches");
+  if (!q || !seqlens || !out || !gt || !workspace) return fail(SEER_ERR_INVALID_ARG, "NULL pointer argument");
+  if (max_len < 1) return fail(SEER_ERR_INVALID_ARG, "max_len must be >= 1");
+  if ((int64_t)dims->max_blocks * dims->block_size < max_len)
+    return fail(SEER_ERR_INVALID_ARG, "max_blocks * block_size < max_len");
+  if (!aligned16(q) || !aligned16(out) || !aligned16(gt) || !aligned16(workspace) || (lse_out && !aligned16(lse_out)))
+    return fail(SEER_ERR_INVALID_ARG, "pointer not 16-byte aligned");
+  const size_t need = seer_prefill_gt_workspace_bytes(dims, max_len);
+  if (workspace_bytes < need)
+    return fail(SEER_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", workspace_bytes, need);
+  int dev;
+  DevFacts* df;
+  if ((st = device_facts(&dev, &df)) != SEER_OK) return st;
+  CUtensorMap tk, tv;
+  seer::PrefillParams p{};
+  if ((st = tensor_map(dims, k, "k", &tk, p.k_perm)) != SEER_OK) return st;
+  if ((st = tensor_map(dims, v, "v", &tv, p.v_perm)) != SEER_OK) return st;
+  p.q = static_cast<const uint16_t*>(q);
+  p.o = static_cast<uint16_t*>(out);
+  p.lse = lse_out;
+  p.gt = gt;
+  p.rmax = static_cast<float*>(workspace);
+  p.seqlens = seqlens;
+  p.B = dims->batch;
+  p.Hq = dims->num_q_heads;
+  p.Hkv = dims->num_kv_heads;
+  p.g = dims->num_q_heads / dims->num_kv_heads;
+  p.NB = dims->max_blocks;
+  p.T = max_len;
+  const int64_t cap = k->num_tokens < v->num_tokens ? k->num_tokens : v->num_tokens;
+  p.kcap = cap > max_len ? max_len : (int32_t)cap;
+  const float scale = dims->softmax_scale > 0.f ? dims->softmax_scale : 1.0f / sqrtf((float)dims->head_dim);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.err = err_word;
+  cudaError_t e = seer::launch_prefill_gt(tk, tv, p, dims->head_dim, dims->block_size, max_len,
+                                          static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "prefill_gt launch");
+  return SEER_OK;
+}
+
 size_t seer_kcomp_state_bytes(const seer_dims_t* dims) {
   if (check_dims(dims) != SEER_OK) return 0;
   return (size_t)dims->batch * dims->num_kv_heads * 3 * dims->head_dim * sizeof(float);

@@ -93,6 +93,23 @@ struct AppendParams {
 cudaError_t launch_kcomp_append(const AppendParams& p, int D, int BLK, int DG, cudaStream_t s);
 cudaError_t launch_kcomp_state_init(const AppendParams& p, int D, int BLK, cudaStream_t s);
 
+// ---------------------------------------------------------------- prefill attention + block target
+struct PrefillParams {
+  const uint16_t* q;       // [B, Hq, T, D]
+  uint16_t* o;             // [B, Hq, T, D]
+  float* lse;              // [B, Hq, T] or null
+  float* gt;               // [B, Hkv, T, NB]
+  float* rmax;             // workspace [B, Hq, NB, T]: each row's tile maxima (log2 domain)
+  const int32_t* seqlens;  // [B]
+  int32_t k_perm[3], v_perm[3];
+  int32_t B, Hq, Hkv, g, NB, T;
+  int32_t kcap;            // tokens the K and V caches hold per sequence
+  float scale_log2;
+  int32_t* err;
+};
+cudaError_t launch_prefill_gt(const CUtensorMap& tk, const CUtensorMap& tv, const PrefillParams& p, int D, int BLK,
+                              int max_len, cudaStream_t s);
+
 // ---------------------------------------------------------------- gate score
 struct GateParams {
   double theta[kMaxHalfGate];   // base^(-2i/d_gate), computed on the host in fp64

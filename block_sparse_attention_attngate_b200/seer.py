@@ -29,7 +29,8 @@ DEVERR_BLOCK_INDEX, DEVERR_PAGE_INDEX, DEVERR_COUNT, DEVERR_TIMEOUT = 1, 2, 4, 8
 EXPORTED = (
     "seer_kcomp_update", "seer_kcomp_state_bytes", "seer_kcomp_append", "seer_kcomp_state_init", "seer_gate_score", "seer_select_blocks", "seer_decode_plan", "seer_sparse_decode_auto_split",
     "seer_sparse_decode_workspace_bytes", "seer_sparse_decode", "seer_sparse_decode_noalloc",
-    "seer_gate_truth_workspace_bytes", "seer_gate_truth", "seer_last_error", "seer_version",
+    "seer_gate_truth_workspace_bytes", "seer_gate_truth", "seer_prefill_gt_workspace_bytes", "seer_prefill_gt",
+    "seer_last_error", "seer_version",
 )
 
 
@@ -72,6 +73,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "seer_sparse_decode_noalloc": (I32, [DP, P, KP, KP, P, P, P, I32, I32, P, P, P, P]),
         "seer_gate_truth_workspace_bytes": (SZ, [DP]),
         "seer_gate_truth": (I32, [DP, P, KP, P, P, P, P, SZ, P, P]),
+        "seer_prefill_gt_workspace_bytes": (SZ, [DP, I32]),
+        "seer_prefill_gt": (I32, [DP, P, I32, KP, KP, P, P, P, P, P, SZ, P, P]),
         "seer_last_error": (ctypes.c_char_p, []),
         "seer_version": (ctypes.c_char_p, []),
     }
@@ -317,6 +320,29 @@ def sparse_decode_noalloc(shape: Shape, q: torch.Tensor, k: KVCache, v: KVCache,
     _check(_lib.seer_sparse_decode_noalloc(ctypes.byref(dims), _ptr(q), ctypes.byref(k.desc), ctypes.byref(v.desc),
                                            _ptr(block_idx), _ptr(block_cnt), _ptr(seqlens), block_idx.shape[-1],
                                            int(num_split), _ptr(out), _ptr(lse), _ptr(err), _stream(stream)))
+
+
+def prefill_gt_workspace_bytes(shape: Shape, max_len: int) -> int:
+    dims = shape.c()
+    return int(_lib.seer_prefill_gt_workspace_bytes(ctypes.byref(dims), int(max_len)))
+
+
+def prefill_gt(shape: Shape, q: torch.Tensor, k: KVCache, v: KVCache, seqlens: torch.Tensor, out: torch.Tensor,
+               gt: torch.Tensor, workspace: torch.Tensor, lse: Optional[torch.Tensor] = None,
+               err: Optional[torch.Tensor] = None, stream=None):
+    """Causal attention [B, Hq, T, d] with every position's block-level target gt [B, Hkv, T, max_blocks]
+    (see seer_prefill_gt); T = q.shape[2]."""
+    _need(q, torch.bfloat16, "q")
+    _need(seqlens, torch.int32, "seqlens")
+    _need(out, torch.bfloat16, "out")
+    _need(gt, torch.float32, "gt")
+    if lse is not None:
+        _need(lse, torch.float32, "lse")
+    dims = shape.c()
+    _check(_lib.seer_prefill_gt(ctypes.byref(dims), _ptr(q), int(q.shape[2]), ctypes.byref(k.desc),
+                                ctypes.byref(v.desc), _ptr(seqlens), _ptr(out), _ptr(lse) if lse is not None else None,
+                                _ptr(gt), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                _ptr(err) if err is not None else None, _stream(stream)))
 
 
 def gate_truth_workspace_bytes(shape: Shape) -> int:

@@ -341,6 +341,40 @@ seer_status seer_gate_truth(const seer_dims_t* dims, const void* q, const seer_k
                             void* workspace, size_t workspace_bytes, int32_t* err_word,
                             void* stream);
 
+/*
+ * seer_prefill_gt -- causal attention over whole sequences with the block-level target of every
+ * query position beside the output, extracted inside the attention forward [CP Knowl 3, Knowl 4]:
+ * per key tile (one block of b keys) each query row's maximum pre-softmax score r is kept, and
+ * once the row's final maximum m and normaliser l are known the block's score is exp(r - m) / l.
+ *
+ * For sequence b, query head i = h*g + j of KV head h and position t < L_b = seqlens[b]:
+ *   out[b, i, t] = sum_{u <= t} softmax_u(scale * q[b, i, t] . K[b, h, u]) V[b, h, u]
+ *   lse_out[b, i, t] = log sum_{u <= t} exp(scale * q[b, i, t] . K[b, h, u])
+ *   gt[b, h, t, n] = G[n] / sum_n' G[n'],   G[n] = max_j max_{u in block n, u <= t} softmax_u(...)
+ *                    for n <= t / b, and 0 for t / b < n < max_blocks
+ * i.e. row t of gt is the decode target (seer_gate_truth) of query position t.  Rows t >= L_b
+ * are not written.
+ *
+ *   q          device bf16 [B, Hq, max_len, d]
+ *   max_len    row capacity of q / out / lse_out / gt (>= every seqlens[b]; max_blocks*b >= max_len)
+ *   k, v       contiguous K / V caches (see seer_kv_t) holding >= seqlens[b] tokens; longer
+ *              sequences are cut to the caches' capacity and SEER_DEVERR_COUNT is set
+ *   seqlens    device int32 [B]
+ *   out        device bf16 [B, Hq, max_len, d]
+ *   lse_out    device fp32 [B, Hq, max_len] or NULL
+ *   gt         device fp32 [B, Hkv, max_len, max_blocks]
+ *   workspace  device, >= seer_prefill_gt_workspace_bytes(dims, max_len) bytes (each query row's
+ *              per-block score maxima, fp32 [B, Hq, max_blocks, max_len]), 16-byte aligned
+ *   err_word   device int32 or NULL (SEER_DEVERR_* bits ORed in)
+ * One CTA per (16 * floor(8 / g) positions, KV head, sequence); the group's query heads share
+ * every K/V tile.  Paged caches: SEER_ERR_UNSUPPORTED.
+ */
+size_t seer_prefill_gt_workspace_bytes(const seer_dims_t* dims, int32_t max_len);
+seer_status seer_prefill_gt(const seer_dims_t* dims, const void* q, int32_t max_len,
+                            const seer_kv_t* k, const seer_kv_t* v, const int32_t* seqlens,
+                            void* out, float* lse_out, float* gt, void* workspace,
+                            size_t workspace_bytes, int32_t* err_word, void* stream);
+
 /* Thread-local text describing the last non-OK status returned on this thread. */
 const char* seer_last_error(void);
 

@@ -181,6 +181,25 @@ def test_kcomp_append_validation(lib, S):
     assert lib.seer_kcomp_state_init(ctypes.byref(d), ctypes.byref(k), P, ctypes.c_void_p(4100), None, None) == 1
 
 
+def test_prefill_gt_validation(lib, S):
+    d = _dims(S)
+    k = _kv(S)
+    n = lib.seer_prefill_gt_workspace_bytes(ctypes.byref(d), 4096)
+    assert n == 8 * 32 * d.max_blocks * 4096 * 4
+    assert lib.seer_prefill_gt_workspace_bytes(ctypes.byref(d), 0) == 0
+    assert lib.seer_prefill_gt(ctypes.byref(d), None, 64, ctypes.byref(k), ctypes.byref(k), P, P, None, P, P,
+                               1 << 30, None, None) == 1
+    big = d.max_blocks * d.block_size + 1                  # rows past max_blocks * b
+    assert lib.seer_prefill_gt(ctypes.byref(d), P, big, ctypes.byref(k), ctypes.byref(k), P, P, None, P, P,
+                               1 << 40, None, None) == 1
+    assert lib.seer_prefill_gt(ctypes.byref(d), P, 64, ctypes.byref(k), ctypes.byref(k), P, P, None, P, P,
+                               16, None, None) == 1          # workspace too small
+    paged = _kv(S, layout=1, num_pages=64, block_table=4096, max_pages_per_seq=512, stride_b=8 * 64 * 128,
+                stride_h=64 * 128)
+    assert lib.seer_prefill_gt(ctypes.byref(d), P, 64, ctypes.byref(paged), ctypes.byref(paged), P, P, None, P, P,
+                               1 << 30, None, None) == 2     # paged caches: unsupported
+
+
 def test_missing_library_fails_loudly(tmp_path):
     from block_sparse_attention_attngate_b200 import seer
     with pytest.raises(ImportError):

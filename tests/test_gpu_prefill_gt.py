@@ -1,0 +1,69 @@
+"""Causal prefill attention with the per-position block-level target (seer_prefill_gt) against the
+CPU oracle.
+
+Tolerances.  Outputs and LSEs: the attention bar (max-abs 1e-2, rel-L2 5e-3; LSE as the decode
+test).  Targets: a block score is exp2(r - m) / l with r and m maxima of fp32 dot products of bf16
+inputs and l the sum of the bf16-rounded probabilities that also weight V, so l carries at most
+2^-9 relative error and the score the same plus fp32 exp2 rounding; GT_REL = 4e-3 is twice that
+bound, far below a dropped head, a wrong block, a missed mask or a missing normalisation."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import seer_oracle as O
+from seer_harness import bf16_bits, check_attention, check_lse, f64, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import block_sparse_attention_attngate_b200 as S
+
+GT_REL = 4e-3
+
+
+def _bf16_bits(x):
+    return (torch.from_numpy(np.asarray(x, np.float32)).to(torch.bfloat16).view(torch.int16).numpy()
+            .view(np.uint16))
+
+
+@pytest.mark.parametrize("d,blk,g,Hkv", [(128, 64, 4, 2), (128, 128, 2, 2), (64, 64, 8, 1), (64, 128, 1, 3),
+                                         (128, 64, 5, 1)])
+def test_prefill_gt_vs_oracle(d, blk, g, Hkv):
+    rng = np.random.default_rng(1300 + d + blk + g)
+    lengths = [300, 2 * blk + 7, 5]
+    B, Hq, T = len(lengths), g * Hkv, 320
+    NB = -(-T // blk)
+    q = _bf16_bits(rng.standard_normal((B, Hq, T, d)))
+    k = _bf16_bits(rng.standard_normal((B, Hkv, T, d)))
+    v = _bf16_bits(rng.standard_normal((B, Hkv, T, d)))
+    sh = S.Shape(B, Hq, Hkv, d, 64, blk, NB)
+    seq = torch.tensor(lengths, dtype=torch.int32, device="cuda")
+    out = torch.full((B, Hq, T, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((B, Hq, T), 7.0, dtype=torch.float32, device="cuda")
+    gt = torch.full((B, Hkv, T, NB), 7.0, dtype=torch.float32, device="cuda")
+    ws = torch.empty(S.prefill_gt_workspace_bytes(sh, T), dtype=torch.uint8, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    S.prefill_gt(sh, to_dev_bf16(q), S.KVCache.contiguous(to_dev_bf16(k)), S.KVCache.contiguous(to_dev_bf16(v)),
+                 seq, out, gt, ws, lse=lse, err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    o_h = f64(bf16_bits(out))
+    lse_h, gt_h = lse.cpu().numpy().astype(np.float64), gt.cpu().numpy().astype(np.float64)
+    scale = 1.0 / math.sqrt(d)
+    for b, L in enumerate(lengths):
+        for h in range(Hkv):
+            ro, rl, rg = O.prefill_ground_truth(f64(q[b, h * g:(h + 1) * g, :L]), f64(k[b, h, :L]),
+                                                f64(v[b, h, :L]), blk, scale)
+            for j in range(g):
+                check_attention(o_h[b, h * g + j, :L], ro[j], f"b{b} h{h} j{j}")
+                check_lse(lse_h[b, h * g + j, :L], rl[j], f"b{b} h{h} j{j}")
+            got = gt_h[b, h, :L, :rg.shape[1]]
+            bad = np.abs(got - rg) > GT_REL * rg + 1e-7
+            assert not bad.any(), f"b{b} h{h}: {int(bad.sum())} target entries off"
+            assert np.all(gt_h[b, h, :L, rg.shape[1]:] == 0.0), "entries past the blocks"
+            assert np.allclose(gt_h[b, h, :L].sum(axis=1), 1.0, atol=1e-5), "rows must sum to 1"
+            assert np.all(gt_h[b, h, L:] == 7.0), "rows past the length were written"
+        assert np.all(np.isnan(o_h[b, :, L:])), "outputs past the length were written"
