@@ -368,7 +368,54 @@ def sweep_rows(S, dev, stream, peak, shape2, reps2, seqlens2, cfg2, inp2, iters=
     del st_d, kv4, k4, v4
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
+    res["prefill-gt-8k"] = prefill_row(S, dev, stream)
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
     return res
+
+
+def prefill_row(S, dev, stream, L=8192, iters=10, warm=3):
+    """The training-side forward (causal attention + every position's block target) on one
+    Qwen3-8B-shaped sequence of L tokens, against the tensor roofline: algorithmic FLOPs
+    4 * d * L(L+1)/2 per query head (the causal QK^T and PV), measured bf16 peak (burst)."""
+    import torch
+    B, Hq, Hkv, d, blk = 1, 32, 8, 128, 64
+    NB = -(-L // blk)
+    gen = torch.Generator(device=dev).manual_seed(1234)
+    q = torch.randn(B, Hq, L, d, device=dev, generator=gen).to(torch.bfloat16)
+    k = torch.randn(B, Hkv, L, d, device=dev, generator=gen).to(torch.bfloat16)
+    v = torch.randn(B, Hkv, L, d, device=dev, generator=gen).to(torch.bfloat16)
+    sh = S.Shape(B, Hq, Hkv, d, d, blk, NB)
+    seq = torch.full((B,), L, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    gt = torch.empty(B, Hkv, L, NB, dtype=torch.float32, device=dev)
+    ws = torch.empty(S.prefill_gt_workspace_bytes(sh, L), dtype=torch.uint8, device=dev)
+    kv_k, kv_v = S.KVCache.contiguous(k), S.KVCache.contiguous(v)
+
+    def run():
+        S.prefill_gt(sh, q, kv_k, kv_v, seq, out, gt, ws, stream=stream)
+    with torch.cuda.stream(stream):
+        for _ in range(warm):
+            run()
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(iters):
+            run()
+        e1.record(stream)
+    e1.synchronize()
+    us = e0.elapsed_time(e1) / iters * 1e3
+    flops = 4.0 * d * L * (L + 1) / 2 * Hq * B
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak, kind = float(json.load(f)["bf16_tflops"]), "measured (burst)"
+    except Exception:
+        peak, kind = 1590.0, "fallback"
+    tf = flops / (us * 1e-6) / 1e12
+    return {"us": us, "tflops": tf, "peak_tflops": peak, "peak_kind": kind, "frac": tf / peak, "flops": flops,
+            "what": "seer_prefill_gt: causal attention + per-position block targets, B=1, L=%d, Hq=32, Hkv=8, "
+                    "d=128, b=64" % L}
 
 
 def run_seer(args):
