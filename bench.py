@@ -57,9 +57,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="skip the sparsity sweep rows")
     ap.add_argument("--cpu-sample", type=int, default=16, help="(b, h) pairs in the oracle sample")
-    ap.add_argument("--only", default="all", choices=["all", "decode", "truth"],
-                    help="decode / truth: run just the sparse-decode / ground-truth launches (small targets "
-                         "for profilers)")
+    ap.add_argument("--only", default="all", choices=["all", "decode", "truth", "prefill"],
+                    help="decode / truth / prefill: run just the sparse-decode / ground-truth / prefill-with-targets "
+                         "launches (small targets for profilers)")
     return ap.parse_args()
 
 
@@ -434,6 +434,13 @@ def run_seer(args):
 
     import block_sparse_attention_attngate_b200 as S
     from synthetic import config, make_inputs
+
+    if args.only == "prefill":
+        stream = torch.cuda.Stream(device=dev)
+        r = prefill_row(S, dev, stream, iters=args.steps, warm=args.warmup)
+        if rank == 0:
+            print(json.dumps({"only": "prefill", "launches": args.warmup + args.steps, "us": r["us"]}), flush=True)
+        return 0
 
     cfg = config(WORKLOAD["cid"], **({"budget": args.budget} if args.budget else {}))
     cfg = config(WORKLOAD["cid"], seed=rank_seed(cfg.seed, rank), **({"budget": args.budget} if args.budget else {}))
