@@ -330,25 +330,44 @@ __global__ void __launch_bounds__(PrefillShape<D, BLK>::kMaxThreads, 1)
     const int i = p0 + pi;
     const bool live = pi < P && i < L;
     const int nb_i = live ? i / BLK + 1 : 0;   // blocks with a key visible to position i
-    float sum = 0.f;
-    for (int n = sub; n < nb_i; n += 8) {
-      float v = 0.f;
-      for (int j = 0; j < g; ++j) {
-        const float r = __ldcg(r_b + ((size_t)j * p.NB + n) * p.T + i);
-        v = fmaxf(v, exp2f(r - ms[j * P + pi]) / ls[j * P + pi]);
+    // a block's score, four blocks at a time with every load issued before any use (two passes:
+    // the sum, then the normalised stores -- no store sits between a load and its successors)
+    auto scores4 = [&](int n0, float (&v)[4]) {
+      float r[4][kMaxGroup];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int j = 0; j < kMaxGroup; ++j)
+          r[u][j] = (j < g && n0 + 8 * u < nb_i) ? __ldcg(r_b + ((size_t)j * p.NB + n0 + 8 * u) * p.T + i) : -INFINITY;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        v[u] = 0.f;
+#pragma unroll
+        for (int j = 0; j < kMaxGroup; ++j)
+          if (j < g && n0 + 8 * u < nb_i) v[u] = fmaxf(v[u], exp2f(r[u][j] - ms[j * P + pi]) / ls[j * P + pi]);
       }
-      gt_b[(size_t)i * p.NB + n] = v;   // unnormalised for now; rescaled below by this thread
-      sum += v;
+    };
+    float sum = 0.f;
+    for (int n0 = sub; n0 < nb_i; n0 += 32) {
+      float v[4];
+      scores4(n0, v);
+      sum += (v[0] + v[1]) + (v[2] + v[3]);
     }
     sum += __shfl_xor_sync(0xffffffffu, sum, 1);
     sum += __shfl_xor_sync(0xffffffffu, sum, 2);
     sum += __shfl_xor_sync(0xffffffffu, sum, 4);
     const float inv = sum > 0.f ? 1.f / sum : 0.f;
-    if (live)
-      for (int n = sub; n < p.NB; n += 8) {
-        float* dst = gt_b + (size_t)i * p.NB + n;
-        *dst = n < nb_i ? *dst * inv : 0.f;
+    if (live) {
+      for (int n0 = sub; n0 < nb_i; n0 += 32) {
+        float v[4];
+        scores4(n0, v);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (n0 + 8 * u < nb_i) gt_b[(size_t)i * p.NB + n0 + 8 * u] = v[u] * inv;
       }
+      for (int n = (nb_i & ~7) + sub; n < p.NB; n += 8)
+        if (n >= nb_i) gt_b[(size_t)i * p.NB + n] = 0.f;
+    }
   }
 }
 
