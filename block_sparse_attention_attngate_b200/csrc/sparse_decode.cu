@@ -5,10 +5,13 @@
 // (chapterpal.com summary), Knowl 6: grid (batch, heads_kv, num_split); the
 // selected list [batch, heads_kv, max_selected_blocks] is split by its width,
 // and the kernel visits only the active block indices.  That grid is kept
-// (num_split >= 1).  The default schedule (num_split == 0) balances instead:
-// the concatenation of every (b, h)'s selected list is cut into equal
-// contiguous ranges, one per CTA of a grid with one CTA per SM, so ragged
-// counts and small batches still keep every SM streaming.
+// (num_split >= 1).  The one-wave schedules balance instead: the concatenation
+// of every (b, h)'s selected list is cut into equal contiguous ranges, one per
+// CTA of a grid with one CTA per SM, so ragged counts and small batches still
+// keep every SM streaming -- by the lists' counts (num_split == 0, a scan of
+// the counts first) or by their capacity (num_split == -1, no scan: positions
+// past a count are skipped; its producer makes a dry pass over its issue loop
+// before the launch dependency wait).
 //
 // The page's H100 kernel pads the query group to 64 rows for wgmma; here the
 // group (g <= 8 query heads) stays a 16-row mma.sync fragment: the work per KV
