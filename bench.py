@@ -40,6 +40,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 WORKLOAD = dict(cid=2, name="qwen3-8b-32k-decode-step")
+NOMINAL_HBM_GBS = 8000.0   # the B200's nominal HBM3e bandwidth (the metric's "~8 TB/s"), context beside the measured peak
 METRIC = "sparse decode attn µs/step & achieved HBM GB/s vs ~8 TB/s (32k ctx, 90% sparse)"
 UNIT = "us/step"
 
@@ -739,7 +740,8 @@ def run_seer(args):
         "step_gbs": step_gbs,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": _profiled_traffic(), "traffic_unit": "bytes per launch (ncu dram read+write)",
-                     "kernel": "sparse_decode_kernel", "peak_kind": peak_kind},
+                     "kernel": "sparse_decode_kernel", "peak_kind": peak_kind,
+                     "nominal_peak": NOMINAL_HBM_GBS, "frac_of_nominal": achieved / NOMINAL_HBM_GBS},
         "step_us_p10_p50_p90": step_pct,
         "sweep": sweep,
         "e2e": {"value": e2e_ms * 1e3, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
