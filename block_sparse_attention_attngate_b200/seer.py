@@ -106,6 +106,13 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _need_shape(t, shape, name: str):
+    """The kernels index these buffers by the problem shape: a smaller tensor would be written past."""
+    if not isinstance(t, torch.Tensor) or tuple(t.shape) != tuple(int(x) for x in shape):
+        got = tuple(t.shape) if isinstance(t, torch.Tensor) else type(t).__name__
+        raise ValueError(f"{name} must have shape {tuple(int(x) for x in shape)}, got {got}")
+
+
 def _need(t: torch.Tensor, dtype: torch.dtype, name: str, contiguous: bool = True):
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise TypeError(f"{name} must be a CUDA tensor")
@@ -191,6 +198,13 @@ def kcomp_append(shape: Shape, k_new: torch.Tensor, seqlens: torch.Tensor, state
                  err: Optional[torch.Tensor] = None, stream=None):
     """Fold each sequence's appended pre-RoPE key [B, Hkv, d] into the running block statistics;
     a completed block writes its K Compression Cache entry (see seer_kcomp_append)."""
+    B, H, d, dg = shape.batch, shape.num_kv_heads, shape.head_dim, shape.gate_dim
+    _need_shape(k_new, (B, H, d), "k_new")
+    _need_shape(seqlens, (B,), "seqlens")
+    _need_shape(state, (B, H, 3, d), "state")
+    _need_shape(valid_blocks, (B, H), "valid_blocks")
+    _need_shape(w_k, (H, dg, 3 * d), "w_k")
+    _need_shape(kcomp, (B, H, shape.max_blocks, dg), "kcomp")
     _need(k_new, torch.bfloat16, "k_new")
     _need(seqlens, torch.int32, "seqlens")
     _need(state, torch.float32, "state")
@@ -205,6 +219,8 @@ def kcomp_append(shape: Shape, k_new: torch.Tensor, seqlens: torch.Tensor, state
 def kcomp_state_init(shape: Shape, k_nope: KVCache, seqlens: torch.Tensor, state: torch.Tensor,
                      err: Optional[torch.Tensor] = None, stream=None):
     """Prime the running block statistics from the key cache (see seer_kcomp_state_init)."""
+    _need_shape(seqlens, (shape.batch,), "seqlens")
+    _need_shape(state, (shape.batch, shape.num_kv_heads, 3, shape.head_dim), "state")
     _need(seqlens, torch.int32, "seqlens")
     _need(state, torch.float32, "state")
     dims = shape.c()
@@ -332,6 +348,15 @@ def prefill_gt(shape: Shape, q: torch.Tensor, k: KVCache, v: KVCache, seqlens: t
                err: Optional[torch.Tensor] = None, stream=None):
     """Causal attention [B, Hq, T, d] with every position's block-level target gt [B, Hkv, T, max_blocks]
     (see seer_prefill_gt); T = q.shape[2]."""
+    if not isinstance(q, torch.Tensor) or q.dim() != 4:
+        raise ValueError("q must be a 4-D [B, Hq, T, d] tensor")
+    B, Hq, H, d, T = shape.batch, shape.num_q_heads, shape.num_kv_heads, shape.head_dim, int(q.shape[2])
+    _need_shape(q, (B, Hq, T, d), "q")
+    _need_shape(seqlens, (B,), "seqlens")
+    _need_shape(out, (B, Hq, T, d), "out")
+    _need_shape(gt, (B, H, T, shape.max_blocks), "gt")
+    if lse is not None:
+        _need_shape(lse, (B, Hq, T), "lse")
     _need(q, torch.bfloat16, "q")
     _need(seqlens, torch.int32, "seqlens")
     _need(out, torch.bfloat16, "out")
