@@ -113,6 +113,21 @@ def _need_shape(t, shape, name: str):
         raise ValueError(f"{name} must have shape {tuple(int(x) for x in shape)}, got {got}")
 
 
+def _need_lists(block_idx, block_cnt, B: int, H: int):
+    """Block lists [B, Hkv, capacity] and counts [B, Hkv] (the capacity is the list's last extent)."""
+    if not isinstance(block_idx, torch.Tensor) or block_idx.dim() != 3 or tuple(block_idx.shape[:2]) != (B, H):
+        got = tuple(block_idx.shape) if isinstance(block_idx, torch.Tensor) else type(block_idx).__name__
+        raise ValueError(f"block_idx must have shape ({B}, {H}, capacity), got {got}")
+    _need_shape(block_cnt, (B, H), "block_cnt")
+
+
+def _need_err(err):
+    if err is not None:
+        if not isinstance(err, torch.Tensor) or err.numel() < 1:
+            raise ValueError("err must hold one int32")
+        _need(err, torch.int32, "err")
+
+
 def _need(t: torch.Tensor, dtype: torch.dtype, name: str, contiguous: bool = True):
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise TypeError(f"{name} must be a CUDA tensor")
@@ -171,9 +186,31 @@ class KVCache:
                    block_table.data_ptr(), block_table.shape[1])
         return cls(d, (pool, block_table))
 
+    def check(self, shape: "Shape", name: str):
+        """The cache holds the shape's sequences, KV heads and head_dim (the library reads it by
+        (b, kv-head, token) from the descriptor's strides, so a smaller view would be read past)."""
+        if self.desc.layout == KV_CONTIGUOUS:
+            t = self._keep[0]
+            if t.shape[0] < shape.batch or t.shape[1] != shape.num_kv_heads or t.shape[3] != shape.head_dim:
+                raise ValueError(f"{name}: a [B >= {shape.batch}, {shape.num_kv_heads}, T, {shape.head_dim}] view "
+                                 f"is needed, got {tuple(t.shape)}")
+        else:
+            pool, table = self._keep
+            if (pool.shape[1] != shape.num_kv_heads or pool.shape[2] != shape.block_size
+                    or pool.shape[3] != shape.head_dim or table.dim() != 2 or table.shape[0] < shape.batch):
+                raise ValueError(f"{name}: a [P, {shape.num_kv_heads}, {shape.block_size}, {shape.head_dim}] pool "
+                                 f"and a [B >= {shape.batch}, pages] table are needed, got {tuple(pool.shape)} and "
+                                 f"{tuple(table.shape)}")
+
 
 def kcomp_update(shape: Shape, k_nope: KVCache, seqlens: torch.Tensor, valid_blocks: torch.Tensor,
                  w_k: torch.Tensor, kcomp: torch.Tensor, stream=None):
+    B, H, d, dg = shape.batch, shape.num_kv_heads, shape.head_dim, shape.gate_dim
+    k_nope.check(shape, "k_nope")
+    _need_shape(seqlens, (B,), "seqlens")
+    _need_shape(valid_blocks, (B, H), "valid_blocks")
+    _need_shape(w_k, (H, dg, 3 * d), "w_k")
+    _need_shape(kcomp, (B, H, shape.max_blocks, dg), "kcomp")
     _need(seqlens, torch.int32, "seqlens")
     _need(valid_blocks, torch.int32, "valid_blocks")
     _need(w_k, torch.bfloat16, "w_k")
@@ -205,6 +242,7 @@ def kcomp_append(shape: Shape, k_new: torch.Tensor, seqlens: torch.Tensor, state
     _need_shape(valid_blocks, (B, H), "valid_blocks")
     _need_shape(w_k, (H, dg, 3 * d), "w_k")
     _need_shape(kcomp, (B, H, shape.max_blocks, dg), "kcomp")
+    _need_err(err)
     _need(k_new, torch.bfloat16, "k_new")
     _need(seqlens, torch.int32, "seqlens")
     _need(state, torch.float32, "state")
@@ -219,6 +257,8 @@ def kcomp_append(shape: Shape, k_new: torch.Tensor, seqlens: torch.Tensor, state
 def kcomp_state_init(shape: Shape, k_nope: KVCache, seqlens: torch.Tensor, state: torch.Tensor,
                      err: Optional[torch.Tensor] = None, stream=None):
     """Prime the running block statistics from the key cache (see seer_kcomp_state_init)."""
+    k_nope.check(shape, "k_nope")
+    _need_err(err)
     _need_shape(seqlens, (shape.batch,), "seqlens")
     _need_shape(state, (shape.batch, shape.num_kv_heads, 3, shape.head_dim), "state")
     _need(seqlens, torch.int32, "seqlens")
@@ -230,6 +270,14 @@ def kcomp_state_init(shape: Shape, k_nope: KVCache, seqlens: torch.Tensor, state
 
 def gate_score(shape: Shape, q_nope: torch.Tensor, w_q: torch.Tensor, kcomp: torch.Tensor, seqlens: torch.Tensor,
                logits: torch.Tensor, q_gate: Optional[torch.Tensor] = None, stream=None):
+    B, Hq, H, d, dg = shape.batch, shape.num_q_heads, shape.num_kv_heads, shape.head_dim, shape.gate_dim
+    _need_shape(q_nope, (B, Hq, d), "q_nope")
+    _need_shape(w_q, (H, dg, shape.group * d), "w_q")
+    _need_shape(kcomp, (B, H, shape.max_blocks, dg), "kcomp")
+    _need_shape(seqlens, (B,), "seqlens")
+    _need_shape(logits, (B, H, shape.max_blocks), "logits")
+    if q_gate is not None:
+        _need_shape(q_gate, (B, H, dg), "q_gate")
     _need(q_nope, torch.bfloat16, "q_nope")
     _need(w_q, torch.bfloat16, "w_q")
     _need(kcomp, torch.bfloat16, "kcomp")
@@ -244,6 +292,10 @@ def gate_score(shape: Shape, q_nope: torch.Tensor, w_q: torch.Tensor, kcomp: tor
 
 def select_blocks(shape: Shape, logits: torch.Tensor, seqlens: torch.Tensor, mode: int, block_idx: torch.Tensor,
                   block_cnt: torch.Tensor, token_budget: int = 0, tau: float = 0.0, stream=None):
+    B, H = shape.batch, shape.num_kv_heads
+    _need_shape(logits, (B, H, shape.max_blocks), "logits")
+    _need_shape(seqlens, (B,), "seqlens")
+    _need_lists(block_idx, block_cnt, B, H)
     _need(logits, torch.float32, "logits")
     _need(seqlens, torch.int32, "seqlens")
     _need(block_idx, torch.int32, "block_idx")
@@ -260,6 +312,21 @@ def decode_plan(shape: Shape, seqlens: torch.Tensor, kcomp: torch.Tensor, q_nope
                 w_k: Optional[torch.Tensor] = None, logits: Optional[torch.Tensor] = None,
                 q_gate: Optional[torch.Tensor] = None, stream=None):
     """kcomp_update (when valid_blocks is given) + gate_score + select_blocks in one launch."""
+    B, Hq, H, d, dg = shape.batch, shape.num_q_heads, shape.num_kv_heads, shape.head_dim, shape.gate_dim
+    _need_shape(seqlens, (B,), "seqlens")
+    _need_shape(kcomp, (B, H, shape.max_blocks, dg), "kcomp")
+    _need_shape(q_nope, (B, Hq, d), "q_nope")
+    _need_shape(w_q, (H, dg, shape.group * d), "w_q")
+    _need_lists(block_idx, block_cnt, B, H)
+    if valid_blocks is not None:
+        _need_shape(valid_blocks, (B, H), "valid_blocks")
+        _need_shape(w_k, (H, dg, 3 * d), "w_k")
+        if k_nope is not None:
+            k_nope.check(shape, "k_nope")
+    if logits is not None:
+        _need_shape(logits, (B, H, shape.max_blocks), "logits")
+    if q_gate is not None:
+        _need_shape(q_gate, (B, H, dg), "q_gate")
     _need(seqlens, torch.int32, "seqlens")
     _need(kcomp, torch.bfloat16, "kcomp")
     _need(q_nope, torch.bfloat16, "q_nope")
@@ -298,10 +365,24 @@ def alloc_workspace(shape: Shape, capacity: int, num_split: int = 0, device=None
     return torch.zeros(max(n, 16), dtype=torch.uint8, device=device or "cuda")
 
 
+def _decode_shapes(shape: Shape, q, k: KVCache, v: KVCache, block_idx, block_cnt, seqlens, out, lse, err):
+    B, Hq, H, d = shape.batch, shape.num_q_heads, shape.num_kv_heads, shape.head_dim
+    _need_shape(q, (B, Hq, d), "q")
+    k.check(shape, "k")
+    v.check(shape, "v")
+    _need_lists(block_idx, block_cnt, B, H)
+    _need_shape(seqlens, (B,), "seqlens")
+    _need_shape(out, (B, Hq, d), "out")
+    if lse is not None:
+        _need_shape(lse, (B, Hq), "lse")
+    _need_err(err)
+
+
 def sparse_decode(shape: Shape, q: torch.Tensor, k: KVCache, v: KVCache, block_idx: torch.Tensor,
                   block_cnt: torch.Tensor, seqlens: torch.Tensor, out: torch.Tensor, workspace: Optional[torch.Tensor],
                   num_split: int = 0, lse: Optional[torch.Tensor] = None, err: Optional[torch.Tensor] = None,
                   stream=None):
+    _decode_shapes(shape, q, k, v, block_idx, block_cnt, seqlens, out, lse, err)
     _need(q, torch.bfloat16, "q")
     _need(block_idx, torch.int32, "block_idx")
     _need(block_cnt, torch.int32, "block_cnt")
@@ -327,11 +408,14 @@ def sparse_decode_noalloc(shape: Shape, q: torch.Tensor, k: KVCache, v: KVCache,
     The library's fixed 8 MiB scratch array takes the workspace's place: calls on one device
     must not overlap on the GPU, and the first call on a device must come before any capture.
     """
+    _decode_shapes(shape, q, k, v, block_idx, block_cnt, seqlens, out, lse, err)
     _need(q, torch.bfloat16, "q")
     _need(block_idx, torch.int32, "block_idx")
     _need(block_cnt, torch.int32, "block_cnt")
     _need(seqlens, torch.int32, "seqlens")
     _need(out, torch.bfloat16, "out")
+    if lse is not None:
+        _need(lse, torch.float32, "lse")
     dims = shape.c()
     _check(_lib.seer_sparse_decode_noalloc(ctypes.byref(dims), _ptr(q), ctypes.byref(k.desc), ctypes.byref(v.desc),
                                            _ptr(block_idx), _ptr(block_cnt), _ptr(seqlens), block_idx.shape[-1],
@@ -355,6 +439,9 @@ def prefill_gt(shape: Shape, q: torch.Tensor, k: KVCache, v: KVCache, seqlens: t
     _need_shape(seqlens, (B,), "seqlens")
     _need_shape(out, (B, Hq, T, d), "out")
     _need_shape(gt, (B, H, T, shape.max_blocks), "gt")
+    k.check(shape, "k")
+    v.check(shape, "v")
+    _need_err(err)
     if lse is not None:
         _need_shape(lse, (B, Hq, T), "lse")
     _need(q, torch.bfloat16, "q")
@@ -384,6 +471,14 @@ def gate_truth(shape: Shape, q: torch.Tensor, k: KVCache, seqlens: torch.Tensor,
                workspace: torch.Tensor, log_scores: Optional[torch.Tensor] = None, err: Optional[torch.Tensor] = None,
                stream=None):
     """Decode ground-truth block scores from full attention (see seer_gate_truth)."""
+    B, H = shape.batch, shape.num_kv_heads
+    _need_shape(q, (B, shape.num_q_heads, shape.head_dim), "q")
+    k.check(shape, "k")
+    _need_shape(seqlens, (B,), "seqlens")
+    _need_shape(scores, (B, H, shape.max_blocks), "scores")
+    if log_scores is not None:
+        _need_shape(log_scores, (B, H, shape.max_blocks), "log_scores")
+    _need_err(err)
     _need(q, torch.bfloat16, "q")
     _need(seqlens, torch.int32, "seqlens")
     _need(scores, torch.float32, "scores")
