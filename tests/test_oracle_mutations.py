@@ -3,7 +3,8 @@
 Every mutant below is a slip someone could make when writing the oracle from
 the pages: a swapped pooling order, a wrong RoPE sign or pairing, an
 off-by-one position, a dropped scale, the wrong tie rule, a non-strict
-threshold, a forgotten partial block, a mis-weighted combine.  A mutant that
+threshold, a top-p that stops short of p, a forgotten partial block, a
+mis-weighted combine, an unnormalised target.  A mutant that
 no pin catches would mean the pins do not fix that part of the definition.
 """
 
@@ -150,6 +151,76 @@ def _prefill_norm_then_max(q, k, v, block, scale):
     return o, lse, pooled.max(0)
 
 
+def _topp_one_short(logits, p, length, block):
+    nfull = length // block
+    s = O.gate_scores(np.asarray(logits, float)[:nfull])
+    order = sorted(range(nfull), key=lambda n: (-float(s[n]), n))
+    chosen, mass = [], 0.0
+    for n in order:                                              # stops before the mass reaches p
+        if mass + float(s[n]) > p:
+            break
+        chosen.append(n)
+        mass += float(s[n])
+    return O._with_partial(chosen, length, block)
+
+
+def _topp_ascending(logits, p, length, block):
+    nfull = length // block
+    s = O.gate_scores(np.asarray(logits, float)[:nfull])
+    chosen, mass = [], 0.0
+    for n in range(nfull):                                       # index order, not score order
+        if mass >= p:
+            break
+        chosen.append(n)
+        mass += float(s[n])
+    return O._with_partial(chosen, length, block)
+
+
+def _threshold_on_logits(logits, tau, length, block):
+    nfull = length // block
+    z = np.asarray(logits, float)[:nfull]                        # tau against the raw logits
+    return O._with_partial([n for n in range(nfull) if z[n] > tau], length, block)
+
+
+def _pool_avg_as_sum(keys):
+    keys = np.asarray(keys, float)
+    return np.concatenate([keys.max(0), keys.min(0), keys.sum(0)])
+
+
+def _k_gate_block_index(keys, w_k, n, block, base):
+    y = np.asarray(w_k, float) @ O.pool_block(keys)
+    return O.round_to_bf16(O.rope(y, n, base))                   # position n, not n * b
+
+
+def _gt_unnormalised(q, k, length, block, scale):
+    gt = REAL_GT(q, k, length, block, scale)
+    q = np.asarray(q, float); kk = np.asarray(k[:length], float)
+    s = scale * q @ kk.T
+    p = np.exp(s - s.max(1, keepdims=True)); p /= p.sum(1, keepdims=True)
+    nb = -(-length // block)
+    return np.array([[p[i, n * block:min((n + 1) * block, length)].max() for n in range(nb)]
+                     for i in range(len(q))]).max(0)
+
+
+def _gt_block_mean(q, k, length, block, scale):
+    q = np.asarray(q, float); kk = np.asarray(k[:length], float)
+    s = scale * q @ kk.T
+    p = np.exp(s - s.max(1, keepdims=True)); p /= p.sum(1, keepdims=True)
+    nb = -(-length // block)
+    col = np.array([[p[i, n * block:min((n + 1) * block, length)].mean() for n in range(nb)]
+                    for i in range(len(q))])                     # average-pooled columns
+    gt = col.max(0)
+    return gt / gt.sum()
+
+
+def _block_tokens_unclipped(blocks, length, block):
+    toks = []
+    for n in blocks:
+        toks.extend(range(n * block, (n + 1) * block))         # the partial block's tail kept
+    return np.asarray(toks, dtype=np.int64)
+
+
+REAL_GT = O.decode_ground_truth
 REAL_PREFILL = O.prefill_ground_truth
 ATTEND = O.attend
 
@@ -172,6 +243,14 @@ MUTANTS = {
     "append_rope_position": ("kcomp_append", _append_rope_at_last),
     "prefill_unmasked": ("prefill_ground_truth", _prefill_unmasked),
     "prefill_norm_then_max": ("prefill_ground_truth", _prefill_norm_then_max),
+    "topp_one_short": ("select_topp", _topp_one_short),
+    "topp_index_order": ("select_topp", _topp_ascending),
+    "threshold_on_logits": ("select_threshold", _threshold_on_logits),
+    "pool_avg_as_sum": ("pool_block", _pool_avg_as_sum),
+    "k_gate_block_index": ("k_gate_entry", _k_gate_block_index),
+    "gt_unnormalised": ("decode_ground_truth", _gt_unnormalised),
+    "gt_block_mean": ("decode_ground_truth", _gt_block_mean),
+    "partial_block_unclipped": ("block_tokens", _block_tokens_unclipped),
 }
 
 
