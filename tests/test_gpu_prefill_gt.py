@@ -29,9 +29,7 @@ def _bf16_bits(x):
             .view(np.uint16))
 
 
-@pytest.mark.parametrize("d,blk,g,Hkv", [(128, 64, 4, 2), (128, 128, 2, 2), (64, 64, 8, 1), (64, 128, 1, 3),
-                                         (128, 64, 5, 1)])
-def test_prefill_gt_vs_oracle(d, blk, g, Hkv):
+def _check_case(d, blk, g, Hkv, nan_tail):
     rng = np.random.default_rng(1300 + d + blk + g)
     lengths = [300, 2 * blk + 7, 5]
     B, Hq, T = len(lengths), g * Hkv, 320
@@ -39,6 +37,10 @@ def test_prefill_gt_vs_oracle(d, blk, g, Hkv):
     q = _bf16_bits(rng.standard_normal((B, Hq, T, d)))
     k = _bf16_bits(rng.standard_normal((B, Hkv, T, d)))
     v = _bf16_bits(rng.standard_normal((B, Hkv, T, d)))
+    if nan_tail:
+        for b, L in enumerate(lengths):
+            for x in (q, k, v):
+                x[b, :, L:] = 0x7FC0                     # bf16 quiet NaN past the length
     sh = S.Shape(B, Hq, Hkv, d, 64, blk, NB)
     seq = torch.tensor(lengths, dtype=torch.int32, device="cuda")
     out = torch.full((B, Hq, T, d), float("nan"), dtype=torch.bfloat16, device="cuda")
@@ -67,3 +69,16 @@ def test_prefill_gt_vs_oracle(d, blk, g, Hkv):
             assert np.allclose(gt_h[b, h, :L].sum(axis=1), 1.0, atol=1e-5), "rows must sum to 1"
             assert np.all(gt_h[b, h, L:] == 7.0), "rows past the length were written"
         assert np.all(np.isnan(o_h[b, :, L:])), "outputs past the length were written"
+
+
+@pytest.mark.parametrize("d,blk,g,Hkv", [(128, 64, 4, 2), (128, 128, 2, 2), (64, 64, 8, 1), (64, 128, 1, 3),
+                                         (128, 64, 5, 1)])
+def test_prefill_gt_vs_oracle(d, blk, g, Hkv):
+    _check_case(d, blk, g, Hkv, nan_tail=False)
+
+
+@pytest.mark.parametrize("d,blk,g,Hkv", [(128, 64, 4, 2), (64, 128, 1, 3)])
+def test_prefill_gt_nan_past_length(d, blk, g, Hkv):
+    """q, K and V rows past each sequence's length hold NaN (a cache's unused tail): none of it
+    reaches the outputs, the LSEs or the targets of the positions that exist."""
+    _check_case(d, blk, g, Hkv, nan_tail=True)
