@@ -3,7 +3,8 @@
 Sizes are small enough for the float64 oracle to finish in seconds while still
 spanning several tiles, splits and a ragged tail; edge cases cover empty
 lists, lengths shorter than one block, NaN-poisoned cache tails, paged
-layouts and out-of-range indices.
+layouts, out-of-range indices and selection rows up to the largest accepted
+max_blocks (8192).
 """
 
 import math
@@ -100,6 +101,48 @@ def test_select_topp_exact(kind):
             for h in range(Hkv):
                 ref = O.select_topp(logits[b, h].astype(np.float64), p32, int(seqlens[b]), block)
                 assert gpu_list(idx_h[b, h], cnt_h[b, h]) == ref, f"p {p} b{b} h{h}"
+
+
+@pytest.mark.parametrize("nb", [1000, 2000, 3000, 8192])
+@pytest.mark.parametrize("mode", ["topk", "threshold", "topp"])
+def test_select_long_rows(nb, mode):
+    """Rows past the small cases: 1000 and 2000 blocks (the register-resident path with 4 and 8 keys
+    a thread), 3000 and 8192 (the shared-memory path; 8192 is the largest max_blocks accepted)."""
+    B, Hkv, block = 2, 2, 64
+    seqlens = np.array([nb * block, (3 * nb // 4) * block + 17], dtype=np.int32)
+    logits = make_logits(41 + nb, B, Hkv, nb, "ties" if nb == 3000 else "normal")
+    sh = S.Shape(B, Hkv, Hkv, 64, 64, block, nb)
+    lg = torch.from_numpy(logits).cuda()
+    sl = torch.from_numpy(seqlens).cuda()
+    cnt = torch.empty((B, Hkv), dtype=torch.int32, device="cuda")
+    if mode == "topk":
+        settings = [nb // 10, nb - 1]
+    elif mode == "threshold":
+        settings = [1e-4, 0.5 / nb]
+    else:
+        settings = [0.5, 0.95]
+    for x in settings:
+        cap = min(nb, x + 1) if mode == "topk" else nb
+        idx = torch.full((B, Hkv, cap), -7, dtype=torch.int32, device="cuda")
+        if mode == "topk":
+            S.select_blocks(sh, lg, sl, S.SELECT_TOPK, idx, cnt, token_budget=x * block)
+        else:
+            x = float(np.float32(x))
+            S.select_blocks(sh, lg, sl, S.SELECT_THRESHOLD if mode == "threshold" else S.SELECT_TOPP, idx, cnt, tau=x)
+        idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
+        for b in range(B):
+            L = int(seqlens[b])
+            for h in range(Hkv):
+                z = logits[b, h].astype(np.float64)
+                got = gpu_list(idx_h[b, h], cnt_h[b, h])
+                assert np.all(idx_h[b, h, cnt_h[b, h]:] == -1)
+                if mode == "topk":
+                    assert got == O.select_topk(z, x, L, block), f"nb {nb} k {x} b{b} h{h}"
+                elif mode == "threshold":
+                    check_selection(got, O.select_threshold(z, x, L, block), O.gate_scores(z[:L // block]), x,
+                                    f"nb {nb} tau {x} b{b} h{h}")
+                else:
+                    assert got == O.select_topp(z, x, L, block), f"nb {nb} p {x} b{b} h{h}"
 
 
 # ------------------------------------------------------------------ gate score / kcomp
