@@ -16,7 +16,7 @@ import torch
 from oracle import seer_oracle as O
 from seer_harness import (OracleBH, bf16_bits, check_attention, check_kcomp_rows, check_logits, check_lse,
                           check_selection, f64, gpu_list, to_dev_bf16)
-from synthetic import config, make_block_lists, make_inputs, make_logits, paged_view
+from synthetic import bf16_bits_from_f32, config, make_block_lists, make_inputs, make_logits, paged_view
 
 pytestmark = pytest.mark.gpu
 
@@ -143,6 +143,50 @@ def test_select_long_rows(nb, mode):
                                     f"nb {nb} tau {x} b{b} h{h}")
                 else:
                     assert got == O.select_topp(z, x, L, block), f"nb {nb} p {x} b{b} h{h}"
+
+
+@pytest.mark.parametrize("nb", [2000, 8192])
+@pytest.mark.parametrize("mode", ["topk", "threshold", "topp"])
+def test_plan_long_rows(nb, mode):
+    """The fused plan (gate + selection, no cache update) on rows of 2000 and 8192 blocks: its logits
+    against the oracle's from the same cache, and its lists against the oracle's selection on the
+    logits the kernel produced (fp32, the selection's input)."""
+    B, Hkv, g, d, dg, block = 2, 2, 4, 128, 128, 64
+    Hq = g * Hkv
+    rng = np.random.default_rng(5000 + nb)
+    seqlens = np.array([nb * block, (3 * nb // 4) * block + 17], dtype=np.int32)
+    q = bf16_bits_from_f32(rng.standard_normal((B, Hq, d), dtype=np.float32))
+    w_q = bf16_bits_from_f32((rng.standard_normal((Hkv, dg, g * d)) / math.sqrt(g * d)).astype(np.float32))
+    kc = bf16_bits_from_f32(rng.standard_normal((B, Hkv, nb, dg), dtype=np.float32))
+    sh = S.Shape(B, Hq, Hkv, d, dg, block, nb)
+    logits = torch.empty((B, Hkv, nb), dtype=torch.float32, device="cuda")
+    cnt = torch.empty((B, Hkv), dtype=torch.int32, device="cuda")
+    k_blocks = nb // 10
+    cap = k_blocks + 1 if mode == "topk" else nb
+    idx = torch.full((B, Hkv, cap), -7, dtype=torch.int32, device="cuda")
+    x = {"topk": 0.0, "threshold": float(np.float32(0.5 / nb)), "topp": float(np.float32(0.9))}[mode]
+    m = {"topk": S.SELECT_TOPK, "threshold": S.SELECT_THRESHOLD, "topp": S.SELECT_TOPP}[mode]
+    S.decode_plan(sh, torch.from_numpy(seqlens).cuda(), to_dev_bf16(kc), to_dev_bf16(q), to_dev_bf16(w_q), m, idx,
+                  cnt, token_budget=k_blocks * block, tau=x, logits=logits)
+    lg = logits.cpu().numpy()
+    idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
+    for b in range(B):
+        L = int(seqlens[b])
+        nfull = L // block
+        for h in range(Hkv):
+            qg = O.q_gate(f64(q[b, h * g:(h + 1) * g]), f64(w_q[h]), L, sh.rope_base)
+            check_logits(lg[b, h, :nfull], O.gate_logits(qg, f64(kc[b, h]), L, block), f"nb {nb} b{b} h{h}")
+            assert np.all(lg[b, h, nfull:] == -np.inf)
+            z = lg[b, h].astype(np.float64)
+            got = gpu_list(idx_h[b, h], cnt_h[b, h])
+            assert np.all(idx_h[b, h, cnt_h[b, h]:] == -1)
+            if mode == "topk":
+                assert got == O.select_topk(z, k_blocks, L, block), f"nb {nb} b{b} h{h}"
+            elif mode == "threshold":
+                check_selection(got, O.select_threshold(z, x, L, block), O.gate_scores(z[:nfull]), x,
+                                f"nb {nb} b{b} h{h}")
+            else:
+                assert got == O.select_topp(z, x, L, block), f"nb {nb} b{b} h{h}"
 
 
 # ------------------------------------------------------------------ gate score / kcomp
