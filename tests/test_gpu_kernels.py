@@ -265,7 +265,8 @@ def test_kcomp_incremental_freeze_and_rebuild():
 
 # ------------------------------------------------------------------ sparse decode on oracle block lists
 
-@pytest.mark.parametrize("d,blk,g", [(128, 64, 4), (128, 128, 5), (64, 64, 8), (64, 128, 1), (128, 64, 2)])
+@pytest.mark.parametrize("d,blk,g", [(128, 64, 4), (128, 128, 5), (64, 64, 8), (64, 128, 1), (128, 64, 2),
+                                     (128, 64, 8)])
 @pytest.mark.parametrize("ns", [1, 2, 3, 0, -1])
 def test_sparse_decode_vs_oracle(d, blk, g, ns):
     Hkv = 2

@@ -72,7 +72,7 @@ def _check_case(d, blk, g, Hkv, nan_tail):
 
 
 @pytest.mark.parametrize("d,blk,g,Hkv", [(128, 64, 4, 2), (128, 128, 2, 2), (64, 64, 8, 1), (64, 128, 1, 3),
-                                         (128, 64, 5, 1)])
+                                         (128, 64, 5, 1), (128, 64, 8, 1)])
 def test_prefill_gt_vs_oracle(d, blk, g, Hkv):
     _check_case(d, blk, g, Hkv, nan_tail=False)
 

@@ -53,7 +53,8 @@ def _check_row(got, ref, what):
     assert not bad.any(), f"{what}: {int(bad.sum())} scores off, worst rel {float(np.max(np.abs(g - ref) / ref)):.2e}"
 
 
-@pytest.mark.parametrize("d,blk,g", [(128, 64, 4), (128, 128, 5), (64, 64, 8), (64, 128, 1), (128, 64, 2)])
+@pytest.mark.parametrize("d,blk,g", [(128, 64, 4), (128, 128, 5), (64, 64, 8), (64, 128, 1), (128, 64, 2),
+                                     (128, 64, 8)])
 def test_gate_truth_vs_oracle(d, blk, g):
     Hkv = 2
     cfg = config(1, B=3, Hq=g * Hkv, Hkv=Hkv, head_dim=d, gate_dim=64, block=blk, seed=700 + d + blk + g)
