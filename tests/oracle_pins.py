@@ -350,11 +350,18 @@ def check_ground_truth():
 
 
 def check_prefill_ground_truth():
-    """Prefill target vs three other things: every row i is the (pinned) decode target of query
+    """Prefill output, LSE and targets against a hand-derived two-head case; then the target vs
+    three other things: every row i is the (pinned) decode target of query
     i over keys 0..i; the output is torch's float64 causal attention; and the pages' tile
     recurrence (per-tile row maxima r, running max m and normaliser l, then exp(r - m) / l)
     reproduces each head's pooled probabilities before the group max."""
     import torch
+    fx = _fx_att("prefill_ground_truth")
+    o, lse, gt = O.prefill_ground_truth(np.array(fx["q"], float), np.array(fx["k"], float),
+                                        np.array(fx["v"], float), fx["block"], fx["scale"])
+    _close(o, fx["expected_o"], 1e-12, "prefill fixture o")
+    _close(lse, fx["expected_lse"], 1e-12, "prefill fixture lse")
+    _close(gt, fx["expected_gt"], 1e-12, "prefill fixture targets")
     rng = np.random.default_rng(16)
     g, L, d, b = 3, 37, 8, 8
     q = rng.standard_normal((g, L, d))
