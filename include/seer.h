@@ -125,8 +125,8 @@ seer_status seer_kcomp_update(const seer_dims_t* dims, const seer_kv_t* k_nope,
 
 /*
  * seer_kcomp_append -- the same cache update from running block statistics, one appended
- * token per sequence and call [CP Knowl 2, Knowl 5: the cache updates once every b generated
- * tokens from the latest b keys, so their per-channel max, min and sum are all it needs].
+ * token per sequence and call [CP Knowl 2, Knowl 5: an entry is built from the b keys of one
+ * finished block, so their per-channel max, min and sum are all it needs].
  *
  * Each sequence b has just appended token t = seqlens[b] - 1 (seqlens after the append;
  * seqlens[b] <= 0: nothing appended, nothing done).  With n = floor(t / b), i = t mod b and

@@ -119,8 +119,8 @@ def kcomp_update(k_nope: np.ndarray, length: int, valid: int, w_k: np.ndarray,
     """Bring one (b, kv-head) K Compression Cache up to date; return the new valid count.
 
     Entries n in [valid, floor(length/b)) are computed from their b keys;
-    entries below `valid` are left untouched [CP Knowl 5: the cache updates
-    once every b generated tokens from the latest b keys].
+    entries below `valid` are left untouched [CP Knowl 5: each time b new tokens
+    exist, one entry is built from those b keys].
     k_nope: [>= length, d] pre-RoPE keys; kcomp: [max_blocks, d_gate] (written in place).
     """
     nfull = length // block
@@ -133,9 +133,8 @@ def kcomp_append(state: np.ndarray, k_new: np.ndarray, length: int, valid: int, 
                  kcomp: np.ndarray, block: int, base: float) -> int:
     """The same cache update, one appended token at a time, from running block statistics.
 
-    The cache is updated once every b generated tokens from the latest b keys [CP Knowl 5], so a
-    decoder only needs those keys' per-channel max, min and sum, not a pre-RoPE copy of the whole
-    context.  `k_new` [d] is the pre-RoPE key of token length-1; `state` [3, d] holds the running
+    Each entry is built from the b keys of one finished block [CP Knowl 5], so a decoder only
+    needs those keys' per-channel max, min and sum, not a pre-RoPE copy of the whole context.  `k_new` [d] is the pre-RoPE key of token length-1; `state` [3, d] holds the running
     max / min / sum of the current block's keys (restarted at a block's first token).  When the
     token completes block n, kcomp[n] = bf16(RoPE_{n*b}(W_k . [max | min | sum/b])) and the fill
     count becomes n+1 (the block's earlier entries must already be there: valid == n).
