@@ -664,7 +664,7 @@ seer_status seer_sparse_decode(const seer_dims_t* dims, const void* q, const see
 // ---------------------------------------------------------------- decode ground truth
 
 namespace {
-// counters [BH] | per-chunk (max, sum) [BH][nchunk][warps][8][2] | block maxima [BH][NB][warps][8]
+// counters [BH] | per-chunk (max, sum) [BH][nchunk][8][2] | block maxima [BH][NB][8] (8 = the largest group)
 size_t truth_layout(const seer_dims_t* d, int* nchunk, size_t* off_part, size_t* off_bmax) {
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
   const size_t bh = (size_t)d->batch * d->num_kv_heads;

@@ -200,6 +200,22 @@ def test_prefill_gt_validation(lib, S):
                                1 << 30, None, None) == 2     # paged caches: unsupported
 
 
+def test_gate_truth_validation(lib, S):
+    d = _dims(S)
+    k = _kv(S)
+    up = lambda x: (x + 255) // 256 * 256
+    bh, nchunk = 8 * 8, 512 // 16                   # 16 blocks per chunk
+    # arrival counters | per-chunk (max, sum) of each of 8 group rows | block maxima of 8 group rows
+    n = up(bh * 4) + up(bh * nchunk * 8 * 2 * 4) + bh * 512 * 8 * 4
+    assert lib.seer_gate_truth_workspace_bytes(ctypes.byref(d)) == n
+    assert lib.seer_gate_truth_workspace_bytes(ctypes.byref(_dims(S, head_dim=80))) == 0
+    assert lib.seer_gate_truth(ctypes.byref(d), None, ctypes.byref(k), P, P, None, P, n, None, None) == 1
+    assert lib.seer_gate_truth(ctypes.byref(d), P, ctypes.byref(k), P, ctypes.c_void_p(4100), None, P, n, None,
+                               None) == 1             # scores not 16-byte aligned
+    assert lib.seer_gate_truth(ctypes.byref(d), P, ctypes.byref(k), P, P, None, P, n - 1, None, None) == 1
+    assert "workspace" in lib.seer_last_error().decode()
+
+
 def test_missing_library_fails_loudly(tmp_path):
     from block_sparse_attention_attngate_b200 import seer
     with pytest.raises(ImportError):
