@@ -353,7 +353,8 @@ seer_status seer_gate_truth(const seer_dims_t* dims, const void* q, const seer_k
  *   gt[b, h, t, n] = G[n] / sum_n' G[n'],   G[n] = max_j max_{u in block n, u <= t} softmax_u(...)
  *                    for n <= t / b, and 0 for t / b < n < max_blocks
  * i.e. row t of gt is the decode target (seer_gate_truth) of query position t.  Rows t >= L_b
- * are not written.
+ * are not written, and q, K and V rows at positions >= L_b are never used (they may hold
+ * anything, NaN included).
  *
  *   q          device bf16 [B, Hq, max_len, d]
  *   max_len    row capacity of q / out / lse_out / gt (>= every seqlens[b]; max_blocks*b >= max_len)
