@@ -73,7 +73,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
             print(r.stdout + r.stderr, flush=True)
         objs.append(obj)
     tmp = LIB + ".tmp"
-    cmd = [nvcc, *ARCH, "-shared", "-o", tmp, *objs, "-lcuda" if False else "-ldl"]
+    cmd = [nvcc, *ARCH, "-shared", "-o", tmp, *objs, "-ldl"]   # the static CUDA runtime (nvcc default) needs libdl
     if verbose:
         print(" ".join(cmd), flush=True)
     r = subprocess.run(cmd, capture_output=True, text=True)
