@@ -34,6 +34,37 @@ Readings taken where the pages are silent (each is pinned by a test):
   * Selected indices are returned ascending.
   * Attention scale defaults to 1/sqrt(d) [SK]; query head i reads KV head
     floor(i / g).
+  * Top-p takes blocks in descending S (ties to the lower index) until their
+    S-sum reaches p [CP K14].
+  * The decode ground truth pools every block the length reaches, the partial
+    one included; the prefill target of position t is the decode target of a
+    query at t over keys 0..t, with the group max and normalisation applied
+    [CP K3, K4].
+  * The running-statistics cache keeps per-channel max, min and sum of the
+    current block's keys, restarted at a block's first token [CP K5].
+
+Pins (tests/oracle_pins.py; each compares against something other than this
+module: hand-derived fixtures under tests/golden/, closed forms, brute force,
+torch routines, or invariants), by function:
+  bf16_to_f64, round_to_bf16     check_bf16_fixture, check_bf16_vs_torch
+  rope                           check_rope_fixture, check_rope_identity_norm_composition,
+                                 check_rope_relative_invariance
+  pool_block                     check_pool_fixture, check_pool_bruteforce
+  k_gate_entry, q_gate,          check_k_gate_fixture, check_q_gate_fixture,
+  gate_logits                    check_gate_logits_fixture, check_gate_linear_bruteforce
+  kcomp_update                   check_kcomp_incremental, check_memory_ratio
+  kcomp_append                   check_kcomp_append_matches_rebuild
+  gate_scores, select_threshold  check_threshold_fixture, check_threshold_extremes
+  select_topk                    check_topk_fixture, check_topk_definition_random
+  select_topp                    check_topp_fixture, check_topp_minimal
+  block_tokens, attend,          check_attention_fixture, check_attention_dense_equivalence,
+  sparse_decode                  check_attention_single_block_and_mask
+  combine, split_list            check_combine_fixture, check_combine_partitions
+  decode_ground_truth            check_ground_truth
+  prefill_ground_truth           check_prefill_ground_truth (hand-derived fixture, torch causal
+                                 attention, the decode target row by row, the tile recurrence)
+  decode_step_bh                 check_gqa_shared_selection
+No function here is left without a pin.
 """
 
 from __future__ import annotations

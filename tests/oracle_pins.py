@@ -56,6 +56,13 @@ def check_bf16_vs_torch():
     ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
     got = O.round_to_bf16(x.astype(np.float64))
     assert np.array_equal(got, ref), "round_to_bf16 disagrees with torch on float32 inputs"
+    # decoding bf16 bit patterns: every pattern that is not a NaN, against torch's own widening
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    wide = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    with np.errstate(invalid="ignore"):      # signalling-NaN patterns widen to NaN
+        dec = O.bf16_to_f64(bits)
+    keep = ~np.isnan(wide)
+    assert np.array_equal(dec[keep], wide[keep]) and np.all(np.isnan(dec[~keep])), "bf16_to_f64"
 
 
 # ---------------------------------------------------------------- RoPE
