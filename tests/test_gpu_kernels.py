@@ -7,6 +7,7 @@ layouts, out-of-range indices and selection rows up to the largest accepted
 max_blocks (8192).
 """
 
+import functools
 import math
 
 import numpy as np
@@ -264,6 +265,44 @@ def test_kcomp_incremental_freeze_and_rebuild():
 
 
 # ------------------------------------------------------------------ sparse decode on oracle block lists
+
+@functools.lru_cache(maxsize=1)
+def _longest_problem():
+    blk, d, g, nb = 64, 64, 4, 8192
+    cfg = config(1, B=1, Hq=g, Hkv=1, head_dim=d, gate_dim=64, block=blk, seed=3131)
+    return cfg, make_inputs(cfg, lengths=[nb * blk - 5], tail="nan")
+
+
+@pytest.mark.parametrize("ns", [0, -1, 16])
+def test_sparse_decode_longest_lists(ns):
+    """The longest lists accepted: max_blocks = 8192 (524,288 tokens at b = 64) with a ragged last
+    block (NaN past the length), half of the full blocks plus the partial one (4097 entries), then
+    every block; the balanced, capacity and (split, kv head, batch) schedules."""
+    blk, d, g, nb = 64, 64, 4, 8192
+    L = nb * blk - 5
+    cfg, inp = _longest_problem()
+    assert inp.max_blocks == nb
+    dv = _dev(inp)
+    sh = _shape(cfg, inp)
+    kv_k, kv_v = S.KVCache.contiguous(dv["k"]), S.KVCache.contiguous(dv["v"])
+    rng = np.random.default_rng(77)
+    half = sorted(int(x) for x in rng.choice(nb - 1, size=(nb - 1) // 2, replace=False)) + [nb - 1]
+    kk, vv, q = f64(inp.k[0, 0]), f64(inp.v[0, 0]), f64(inp.q[0])
+    for blocks in (half, list(range(nb))):
+        idx = np.full((1, 1, nb), -1, np.int32)
+        idx[0, 0, :len(blocks)] = blocks
+        cnt = np.array([[len(blocks)]], np.int32)
+        out = torch.empty((1, g, d), dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty((1, g), dtype=torch.float32, device="cuda")
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        S.sparse_decode(sh, dv["q"], kv_k, kv_v, torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda(),
+                        dv["seqlens"], out, S.alloc_workspace(sh, nb, ns), num_split=ns, lse=lse, err=err)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        ro, rl = O.sparse_decode(q, kk, vv, blocks, L, blk, 1.0 / math.sqrt(d))
+        check_attention(f64(bf16_bits(out))[0], ro, f"{len(blocks)} blocks ns {ns}")
+        check_lse(lse.cpu().numpy()[0].astype(np.float64), rl, f"{len(blocks)} blocks ns {ns}")
+
 
 @pytest.mark.parametrize("d,blk,g", [(128, 64, 4), (128, 128, 5), (64, 64, 8), (64, 128, 1), (128, 64, 2),
                                      (128, 64, 8)])
