@@ -478,6 +478,59 @@ def test_sparse_decode_edges_and_device_errors():
     check_attention(f64(bf16_bits(out))[3], ro, "skipped bad index")
 
 
+def test_repeat_runs_are_bitwise_identical():
+    """Every kernel is deterministic (integer atomics only; split pieces merged in a fixed order):
+    two runs on fresh buffers agree bit for bit -- the decode step fused and unfused, the ground
+    truth scorer and the prefill forward."""
+    blk, d, dg, g, Hkv = 64, 128, 128, 4, 2
+    cfg = config(1, B=2, Hq=g * Hkv, Hkv=Hkv, head_dim=d, gate_dim=dg, block=blk, seed=4242)
+    lengths = [20 * blk + 7, 16 * blk]
+    inp = make_inputs(cfg, lengths=lengths)
+    dv = _dev(inp)
+    sh = _shape(cfg, inp)
+    nb = inp.max_blocks
+    kv_k, kv_v = S.KVCache.contiguous(dv["k"]), S.KVCache.contiguous(dv["v"])
+
+    def bits(t):
+        return t.contiguous().view(torch.int32 if t.element_size() == 4 else torch.int16).cpu()
+
+    for fused in (True, False):
+        runs = []
+        for _ in range(2):
+            kc = torch.zeros((cfg.B, Hkv, nb, dg), dtype=torch.bfloat16, device="cuda")
+            valid = torch.zeros(cfg.B, Hkv, dtype=torch.int32, device="cuda")
+            st = S.DecodeStep(sh, kv_k, kv_v, dv["w_q"], dv["w_k"], kc, valid, mode=S.SELECT_TOPK,
+                              token_budget=4 * blk, num_split=2)
+            st.run(dv["q"], dv["seqlens"], fused=fused)
+            torch.cuda.synchronize()
+            assert int(st.err.item()) == 0
+            runs.append(st)
+        a, b = runs
+        for name in ("kcomp", "valid_blocks", "block_idx", "block_cnt", "out", "lse"):
+            assert torch.equal(bits(getattr(a, name)), bits(getattr(b, name))), f"fused={fused}: {name}"
+        for bb, L in enumerate(lengths):
+            n = L // blk
+            assert torch.equal(bits(a.logits[bb, :, :n]), bits(b.logits[bb, :, :n])), f"fused={fused}: logits"
+    scores = []
+    for _ in range(2):
+        sc = torch.empty((cfg.B, Hkv, nb), dtype=torch.float32, device="cuda")
+        S.gate_truth(sh, dv["q"], kv_k, dv["seqlens"], sc, S.alloc_truth_workspace(sh))
+        scores.append(bits(sc))
+    assert torch.equal(scores[0], scores[1]), "ground truth"
+    T = int(inp.k.shape[2])
+    q4 = torch.randn(cfg.B, cfg.Hq, T, d, generator=torch.Generator().manual_seed(5)).to(torch.bfloat16).cuda()
+    outs = []
+    for _ in range(2):
+        o = torch.full((cfg.B, cfg.Hq, T, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+        ls = torch.full((cfg.B, cfg.Hq, T), 7.0, dtype=torch.float32, device="cuda")
+        gt = torch.full((cfg.B, Hkv, T, nb), 7.0, dtype=torch.float32, device="cuda")
+        ws = torch.empty(S.prefill_gt_workspace_bytes(sh, T), dtype=torch.uint8, device="cuda")
+        S.prefill_gt(sh, q4, kv_k, kv_v, dv["seqlens"], o, gt, ws, lse=ls)
+        outs.append((bits(o), bits(ls), bits(gt)))
+    for x, y in zip(*outs):
+        assert torch.equal(x, y), "prefill"
+
+
 def test_host_argument_errors():
     sh = S.Shape(2, 8, 2, 128, 128, 64, 16)
     t = torch.zeros(2, 2, 1024, 128, dtype=torch.bfloat16, device="cuda")
