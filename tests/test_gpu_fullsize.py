@@ -1,6 +1,7 @@
 """Full-size parity on sampled outputs, in the launch configurations bench.py times:
-the ground-truth scorer on the Qwen3-8B-shaped 32k step, and the prefill forward with targets on
-one 8k sequence (B=1, Hq=32, Hkv=8, d=128, b=64).  The oracle computes each sampled row on its
+the ground-truth scorer and the block-completing running-statistics cache launch on the
+Qwen3-8B-shaped 32k step, and the prefill forward with targets on one 8k sequence (B=1, Hq=32,
+Hkv=8, d=128, b=64).  The oracle computes each sampled row on its
 own: the decode target of a (b, kv-head) from its whole K, and a prefill row i as the attention
 and decode target of query position i over keys 0..i (the prefill target rows are pinned to the
 decode target in the oracle's own checks).  Tolerances as the small-size tests."""
