@@ -29,9 +29,9 @@ def _bf16_bits(x):
             .view(np.uint16))
 
 
-def _check_case(d, blk, g, Hkv, nan_tail):
+def _check_case(d, blk, g, Hkv, nan_tail, lengths=None):
     rng = np.random.default_rng(1300 + d + blk + g)
-    lengths = [300, 2 * blk + 7, 5]
+    lengths = lengths or [300, 2 * blk + 7, 5]
     B, Hq, T = len(lengths), g * Hkv, 320
     NB = -(-T // blk)
     q = _bf16_bits(rng.standard_normal((B, Hq, T, d)))
@@ -56,6 +56,9 @@ def _check_case(d, blk, g, Hkv, nan_tail):
     lse_h, gt_h = lse.cpu().numpy().astype(np.float64), gt.cpu().numpy().astype(np.float64)
     scale = 1.0 / math.sqrt(d)
     for b, L in enumerate(lengths):
+        if L == 0:                                       # an empty sequence: nothing written
+            assert np.all(gt_h[b] == 7.0) and np.all(lse_h[b] == 7.0) and np.all(np.isnan(o_h[b]))
+            continue
         for h in range(Hkv):
             ro, rl, rg = O.prefill_ground_truth(f64(q[b, h * g:(h + 1) * g, :L]), f64(k[b, h, :L]),
                                                 f64(v[b, h, :L]), blk, scale)
@@ -82,3 +85,8 @@ def test_prefill_gt_nan_past_length(d, blk, g, Hkv):
     """q, K and V rows past each sequence's length hold NaN (a cache's unused tail): none of it
     reaches the outputs, the LSEs or the targets of the positions that exist."""
     _check_case(d, blk, g, Hkv, nan_tail=True)
+
+
+def test_prefill_gt_empty_and_one_token_sequences():
+    """Sequences of 0 and 1 tokens beside a ragged one: the empty one is left untouched."""
+    _check_case(128, 64, 4, 2, nan_tail=True, lengths=[0, 1, 2 * 64 + 7])
