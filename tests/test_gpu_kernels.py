@@ -478,6 +478,38 @@ def test_sparse_decode_edges_and_device_errors():
     check_attention(f64(bf16_bits(out))[3], ro, "skipped bad index")
 
 
+def test_decode_step_with_an_empty_sequence():
+    """A sequence of length 0 in the batch gets no blocks, a fill count of 0, a zero output and
+    lse = -inf; the other sequence's cache rows and lists are bit-identical to a run in which the
+    first sequence is not empty, and its outputs agree within the attention bar."""
+    blk, d, dg, g, Hkv = 64, 128, 128, 4, 2
+    L1 = 9 * blk + 17
+    cfg = config(1, B=2, Hq=g * Hkv, Hkv=Hkv, head_dim=d, gate_dim=dg, block=blk, seed=5353)
+    inp = make_inputs(cfg, lengths=[3 * blk + 1, L1])
+    dv = _dev(inp)
+    sh = _shape(cfg, inp)
+    kv_k, kv_v = S.KVCache.contiguous(dv["k"]), S.KVCache.contiguous(dv["v"])
+    steps = []
+    for L0 in (0, 3 * blk + 1):
+        kc = torch.zeros((cfg.B, Hkv, inp.max_blocks, dg), dtype=torch.bfloat16, device="cuda")
+        valid = torch.zeros(cfg.B, Hkv, dtype=torch.int32, device="cuda")
+        st = S.DecodeStep(sh, kv_k, kv_v, dv["w_q"], dv["w_k"], kc, valid, mode=S.SELECT_TOPK,
+                          token_budget=4 * blk)
+        st.run(dv["q"], torch.tensor([L0, L1], dtype=torch.int32, device="cuda"))
+        torch.cuda.synchronize()
+        assert int(st.err.item()) == 0
+        steps.append(st)
+    e, f = steps
+    assert e.block_cnt[0].cpu().tolist() == [0] * Hkv and e.valid_blocks[0].cpu().tolist() == [0] * Hkv
+    assert torch.all(e.out[0].float() == 0.0) and torch.all(torch.isneginf(e.lse[0]))
+    for name in ("kcomp", "block_idx", "block_cnt", "valid_blocks"):
+        x, y = getattr(e, name)[1], getattr(f, name)[1]
+        assert torch.equal(x.view(torch.int16) if x.dtype == torch.bfloat16 else x,
+                           y.view(torch.int16) if y.dtype == torch.bfloat16 else y), name
+    check_attention(f64(bf16_bits(e.out[1])), f64(bf16_bits(f.out[1])), "out of the other sequence")
+    check_lse(e.lse[1].cpu().numpy().astype(np.float64), f.lse[1].cpu().numpy().astype(np.float64), "its lse")
+
+
 def test_repeat_runs_are_bitwise_identical():
     """Every kernel is deterministic (integer atomics only; split pieces merged in a fixed order):
     two runs on fresh buffers agree bit for bit -- the decode step fused and unfused, the ground
