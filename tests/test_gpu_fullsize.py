@@ -1,7 +1,6 @@
 """Full-size parity on sampled outputs, in the launch configurations bench.py times:
-the ground-truth scorer and the block-completing running-statistics cache launch on the
-Qwen3-8B-shaped 32k step, and the prefill forward with targets on one 8k sequence (B=1, Hq=32,
-Hkv=8, d=128, b=64).  The oracle computes each sampled row on its
+the ground-truth scorer on the Qwen3-8B-shaped 32k step, and the prefill forward with targets on
+one 8k sequence (B=1, Hq=32, Hkv=8, d=128, b=64).  The oracle computes each sampled row on its
 own: the decode target of a (b, kv-head) from its whole K, and a prefill row i as the attention
 and decode target of query position i over keys 0..i (the prefill target rows are pinned to the
 decode target in the oracle's own checks).  Tolerances as the small-size tests."""
@@ -14,7 +13,7 @@ import pytest
 import torch
 
 from oracle import seer_oracle as O
-from seer_harness import OracleBH, bf16_bits, check_attention, check_kcomp_rows, check_lse, f64, to_dev_bf16
+from seer_harness import OracleBH, bf16_bits, check_attention, check_lse, f64, to_dev_bf16
 from synthetic import config, make_inputs
 
 pytestmark = pytest.mark.gpu
@@ -89,30 +88,3 @@ def test_prefill_8k_sampled():
             bad = np.abs(row[:len(ref)] - ref) > GT_REL_PREFILL * ref + 1e-7
             assert not bad.any(), f"h{h} i{i}: {int(bad.sum())} target entries off"
             assert np.all(row[len(ref):] == 0.0)
-
-
-def test_kcomp_append_32k_sampled():
-    """The cache from running block statistics at the 32k step's shapes (B=8, Hkv=8, 512 blocks of
-    64), in the launch that completes a block: statistics primed from the key cache 63 tokens into
-    block 511, then the token that completes it writes entry 511 of every (b, kv-head)."""
-    cfg, inp = _step_32k()
-    B, Hkv, d, dg, blk, nb = cfg.B, cfg.Hkv, cfg.head_dim, cfg.gate_dim, cfg.block, inp.max_blocks
-    L = nb * blk
-    assert np.all(inp.seqlens == L)
-    sh = S.Shape(B, cfg.Hq, Hkv, d, dg, blk, nb, rope_base=cfg.rope_base)
-    kv = S.KVCache.contiguous(to_dev_bf16(inp.k))
-    state = S.alloc_kcomp_state(sh)
-    err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    S.kcomp_state_init(sh, kv, torch.full((B,), L - 1, dtype=torch.int32, device="cuda"), state, err=err)
-    valid = torch.full((B, Hkv), nb - 1, dtype=torch.int32, device="cuda")
-    kc = torch.zeros((B, Hkv, nb, dg), dtype=torch.bfloat16, device="cuda")
-    S.kcomp_append(sh, to_dev_bf16(np.ascontiguousarray(inp.k[:, :, L - 1])), torch.full((B,), L, dtype=torch.int32,
-                   device="cuda"), state, valid, to_dev_bf16(inp.w_k), kc, err=err)
-    torch.cuda.synchronize()
-    assert int(err.item()) == 0
-    assert np.all(valid.cpu().numpy() == nb)
-    got = bf16_bits(kc)
-    assert np.all(got[:, :, :nb - 1] == 0), "entries below the fill count were written"
-    for b, h in ((0, 0), (2, 7), (5, 3), (7, 6)):
-        ref = O.k_gate_entry(f64(inp.k[b, h, L - blk:L]), f64(inp.w_k[h]), nb - 1, blk, cfg.rope_base)
-        check_kcomp_rows(got[b, h, nb - 1:nb], ref[None], f"b{b} h{h}")

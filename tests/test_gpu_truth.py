@@ -53,8 +53,7 @@ def _check_row(got, ref, what):
     assert not bad.any(), f"{what}: {int(bad.sum())} scores off, worst rel {float(np.max(np.abs(g - ref) / ref)):.2e}"
 
 
-@pytest.mark.parametrize("d,blk,g", [(128, 64, 4), (128, 128, 5), (64, 64, 8), (64, 128, 1), (128, 64, 2),
-                                     (128, 64, 8)])
+@pytest.mark.parametrize("d,blk,g", [(128, 64, 4), (128, 128, 5), (64, 64, 8), (64, 128, 1), (128, 64, 2)])
 def test_gate_truth_vs_oracle(d, blk, g):
     Hkv = 2
     cfg = config(1, B=3, Hq=g * Hkv, Hkv=Hkv, head_dim=d, gate_dim=64, block=blk, seed=700 + d + blk + g)
@@ -132,18 +131,3 @@ def test_ground_truth_selection_pipeline():
             ro, _ = ob.attention(L, inp.q, sel)
             check_attention(o[b, h * g:(h + 1) * g], ro, f"b{b} h{h}")
     assert compared >= cfg.B * Hkv // 2
-
-
-def test_gate_truth_empty_sequence():
-    """A sequence of length 0 gets an all-zero row (log scores -inf); the other rows are unaffected."""
-    blk, d, g, Hkv = 64, 128, 4, 2
-    cfg = config(1, B=2, Hq=g * Hkv, Hkv=Hkv, head_dim=d, gate_dim=64, block=blk, seed=2929)
-    lengths = [0, 3 * blk + 5]
-    inp = make_inputs(cfg, lengths=lengths, tail="nan")
-    got, lg = _run_truth(cfg, inp)
-    assert np.all(got[0] == 0.0) and np.all(np.isneginf(lg[0]))
-    scale = 1.0 / math.sqrt(d)
-    for h in range(Hkv):
-        ob = OracleBH(inp, 1, h)
-        ref = O.decode_ground_truth(ob.q_group(inp.q), ob.k, lengths[1], blk, scale)
-        _check_row(got[1, h], ref, f"h{h}")
