@@ -29,7 +29,7 @@ keeps the plain 1e-3 bound.
 from __future__ import annotations
 
 import math
-from typing import Dict, List, Sequence, Tuple
+from typing import List, Sequence
 
 import numpy as np
 import torch

@@ -8,8 +8,6 @@ mis-weighted combine, an unnormalised target.  A mutant that
 no pin catches would mean the pins do not fix that part of the definition.
 """
 
-import math
-
 import numpy as np
 import pytest
 
