@@ -2,8 +2,8 @@
 // the cache update that needs no pre-RoPE copy of the whole context.
 //
 // "SeerAttention-R: Sparse Attention Adaptation for Long Reasoning"
-// (chapterpal.com summary), Knowl 2 and Knowl 5: the cache is updated once
-// every b generated tokens from the latest b keys, whose entry is
+// (chapterpal.com summary), Knowl 2 and Knowl 5: each finished block of b keys
+// gets one cache entry,
 //   RoPE_{n*b}( W_k[h] . [max | min | avg] of the block's pre-RoPE keys ).
 // max, min and avg over a block need only the running per-channel max, min and
 // sum of its keys so far, so each (b, kv-head) keeps those (fp32, 3 x d) and
