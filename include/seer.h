@@ -158,7 +158,7 @@ seer_status seer_kcomp_append(const seer_dims_t* dims, const void* k_new, const 
 
 /*
  * seer_kcomp_state_init -- prime the running block statistics of seer_kcomp_append from the
- * key cache: for every (b, h), the per-channel max, min and sum of the pre-RoPE keys of tokens
+ * key cache [CP Knowl 5: the entry of the block in progress is built once it is full]: for every (b, h), the per-channel max, min and sum of the pre-RoPE keys of tokens
  * [floor(L_b / b) * b, L_b) (the current, incomplete block; empty at a block boundary:
  * -inf, +inf, 0).  Reads at most b - 1 keys per (b, h).  Page or capacity errors set
  * SEER_DEVERR_PAGE_INDEX / SEER_DEVERR_COUNT in *err_word and leave the empty statistics.
@@ -218,7 +218,8 @@ seer_status seer_select_blocks(const seer_dims_t* dims, const float* logits,
                                int32_t capacity, void* stream);
 
 /*
- * seer_decode_plan -- seer_kcomp_update + seer_gate_score + seer_select_blocks in one launch.
+ * seer_decode_plan -- seer_kcomp_update + seer_gate_score + seer_select_blocks in one launch
+ * [CP Knowl 1-2, Knowl 5, as those three calls].
  *
  * Same arguments and results as the three calls made in that order, with these differences:
  *   valid_blocks  NULL skips the cache update (the cache must then be current already)
@@ -233,15 +234,15 @@ seer_status seer_decode_plan(const seer_dims_t* dims, const seer_kv_t* k_nope, c
                              int32_t capacity, void* stream);
 
 /*
- * A split count for the pages' (num_split, Hkv, B) grid that fills one wave of the SMs (host
- * heuristic, no device reads).  seer_sparse_decode uses its own one-wave schedules when given
+ * A split count for the pages' (num_split, Hkv, B) grid [CP Knowl 6] that fills one wave of the
+ * SMs (host heuristic, no device reads).  seer_sparse_decode uses its own one-wave schedules when given
  * num_split == 0 or -1; pass this value to get the grid schedule instead.
  */
 int32_t seer_sparse_decode_auto_split(const seer_dims_t* dims, int32_t capacity);
 
 /*
- * Workspace bytes seer_sparse_decode needs for `num_split`: one arrival counter per (b, h) plus
- * fp32 partial outputs and LSEs -- 2 slots per CTA of the one-wave schedules (num_split 0, -1),
+ * Workspace bytes seer_sparse_decode needs for `num_split` [CP Knowl 6: the split partials and
+ * their log-sum-exp combine]: one arrival counter per (b, h) plus fp32 partial outputs and LSEs -- 2 slots per CTA of the one-wave schedules (num_split 0, -1),
  * num_split slots per (b, h) for the grid schedule, none for num_split == 1.  The counters must
  * be zero before the first call (e.g. allocate zero-filled); every completed call leaves them
  * zero again.

@@ -216,6 +216,23 @@ def test_gate_truth_validation(lib, S):
     assert "workspace" in lib.seer_last_error().decode()
 
 
+def test_every_entry_point_cites_its_passage():
+    """Each entry point's comment block in the header cites the page section that defines the
+    operation, or says that the pages have no counterpart (utilities excepted)."""
+    import re
+    text = open(HEADER).read()
+    blocks = re.findall(r"/\*(.*?)\*/\s*((?:[\w\s\*]+?\s\**seer_\w+\s*\([^;]*\);\s*)+)", text, re.S)
+    seen = set()
+    for comment, decls in blocks:
+        for name in re.findall(r"(seer_\w+)\s*\(", decls):
+            seen.add(name)
+            if name in ("seer_last_error", "seer_version"):
+                continue
+            assert re.search(r"\[CP |\[PN |\[SK |no counterpart", comment), f"{name}: no citation"
+    assert {"seer_kcomp_update", "seer_gate_score", "seer_select_blocks", "seer_sparse_decode",
+            "seer_decode_plan", "seer_gate_truth", "seer_prefill_gt", "seer_kcomp_append"} <= seen
+
+
 def test_missing_library_fails_loudly(tmp_path):
     from block_sparse_attention_attngate_b200 import seer
     with pytest.raises(ImportError):
