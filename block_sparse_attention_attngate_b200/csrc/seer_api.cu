@@ -591,10 +591,14 @@ size_t seer_sparse_decode_workspace_bytes(const seer_dims_t* dims, int32_t capac
   return ws_layout(dims, ns, ctas, &a, &b);
 }
 
-seer_status seer_sparse_decode(const seer_dims_t* dims, const void* q, const seer_kv_t* k, const seer_kv_t* v,
-                               const int32_t* block_idx, const int32_t* block_cnt, const int32_t* seqlens,
-                               int32_t capacity, int32_t num_split, void* workspace, size_t workspace_bytes,
-                               void* out, float* lse_out, int32_t* err_word, void* stream) {
+}  // extern "C"
+
+namespace seer {
+
+seer_status prepare_sparse_decode(const seer_dims_t* dims, const void* q, const seer_kv_t* k, const seer_kv_t* v,
+                                  const int32_t* block_idx, const int32_t* block_cnt, const int32_t* seqlens,
+                                  int32_t capacity, int32_t num_split, void* workspace, size_t workspace_bytes,
+                                  void* out, float* lse_out, int32_t* err_word, DecodeLaunch* L) {
   seer_status st = check_dims(dims);
   if (st != SEER_OK) return st;
   if ((st = check_kv(dims, k, "k")) != SEER_OK) return st;
@@ -622,10 +626,9 @@ seer_status seer_sparse_decode(const seer_dims_t* dims, const void* q, const see
       return fail(SEER_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed for num_split %d", workspace_bytes, need, ns);
     if (!aligned16(workspace)) return fail(SEER_ERR_INVALID_ARG, "workspace not 16-byte aligned");
   }
-  CUtensorMap tk, tv;
-  seer::DecodeParams p;
-  if ((st = tensor_map(dims, k, "k", &tk, p.k_perm)) != SEER_OK) return st;
-  if ((st = tensor_map(dims, v, "v", &tv, p.v_perm)) != SEER_OK) return st;
+  DecodeParams& p = L->p;
+  if ((st = tensor_map(dims, k, "k", &L->tk, p.k_perm)) != SEER_OK) return st;
+  if ((st = tensor_map(dims, v, "v", &L->tv, p.v_perm)) != SEER_OK) return st;
   p.q = static_cast<const uint16_t*>(q);
   p.idx = block_idx;
   p.cnt = block_cnt;
@@ -655,10 +658,32 @@ seer_status seer_sparse_decode(const seer_dims_t* dims, const void* q, const see
   p.out = static_cast<uint16_t*>(out);
   p.lse_out = lse_out;
   p.err = err_word;
-  cudaError_t e = seer::launch_sparse_decode(tk, tv, p, dims->head_dim, dims->block_size, ctas,
-                                             static_cast<cudaStream_t>(stream));
+  L->D = dims->head_dim;
+  L->BLK = dims->block_size;
+  L->ctas = ctas;
+  L->need = need;
+  return SEER_OK;
+}
+
+seer_status launch_prepared_decode(const DecodeLaunch& L, cudaStream_t s) {
+  cudaError_t e = launch_sparse_decode(L.tk, L.tv, L.p, L.D, L.BLK, L.ctas, s);
   if (e != cudaSuccess) return cuda_fail(e, "sparse_decode launch");
   return SEER_OK;
+}
+
+}  // namespace seer
+
+extern "C" {
+
+seer_status seer_sparse_decode(const seer_dims_t* dims, const void* q, const seer_kv_t* k, const seer_kv_t* v,
+                               const int32_t* block_idx, const int32_t* block_cnt, const int32_t* seqlens,
+                               int32_t capacity, int32_t num_split, void* workspace, size_t workspace_bytes,
+                               void* out, float* lse_out, int32_t* err_word, void* stream) {
+  seer::DecodeLaunch L;
+  const seer_status st = seer::prepare_sparse_decode(dims, q, k, v, block_idx, block_cnt, seqlens, capacity, num_split,
+                                                     workspace, workspace_bytes, out, lse_out, err_word, &L);
+  if (st != SEER_OK) return st;
+  return seer::launch_prepared_decode(L, static_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------- decode ground truth

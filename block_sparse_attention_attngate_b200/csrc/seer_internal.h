@@ -8,6 +8,8 @@
 
 #include <atomic>
 
+#include "seer.h"
+
 namespace seer {
 
 // Launch `kern` on `s` with programmatic stream serialization (see pdl_wait /
@@ -173,6 +175,20 @@ struct DecodeParams {
 cudaError_t launch_sparse_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                                  int D, int BLK, int grid_flat, cudaStream_t s);
 int decode_ctas_per_sm(int D, int BLK);
+
+// seer_sparse_decode in two stages: every argument check and the launch set-up (tensor maps,
+// parameters), which enqueues nothing, then the launch itself.
+struct DecodeLaunch {
+  CUtensorMap tk, tv;
+  DecodeParams p;
+  int D, BLK, ctas;
+  size_t need;   // workspace bytes the launch uses
+};
+seer_status prepare_sparse_decode(const seer_dims_t* dims, const void* q, const seer_kv_t* k, const seer_kv_t* v,
+                                  const int32_t* block_idx, const int32_t* block_cnt, const int32_t* seqlens,
+                                  int32_t capacity, int32_t num_split, void* workspace, size_t workspace_bytes,
+                                  void* out, float* lse_out, int32_t* err_word, DecodeLaunch* launch);
+seer_status launch_prepared_decode(const DecodeLaunch& launch, cudaStream_t s);
 
 // ---------------------------------------------------------------- decode ground truth
 struct TruthParams {

@@ -18,8 +18,12 @@
 // device address (on the host it names a stand-in object): the device address
 // is looked up with cudaGetSymbolAddress, once per device, by the first call
 // made while that device is current; make that first call before any stream
-// capture.  Each call clears the counters it relies on (an async memset on
-// the caller's stream) because the array keeps whatever the previous call left.
+// capture.  The looked-up address is kept for the life of the process, so
+// calls after cudaDeviceReset (which unloads the library's device image) are
+// not supported.  Each call clears the counters it relies on (an async memset
+// on the caller's stream) because the array keeps whatever the previous call
+// left; a call rejected by its argument checks enqueues nothing, not even that
+// memset.
 #include <stdio.h>
 
 #include <mutex>
@@ -83,11 +87,18 @@ extern "C" seer_status seer_sparse_decode_noalloc(const seer_dims_t* dims, const
   if (need > 0) {
     cudaError_t e = noalloc_scratch(&scratch);
     if (e != cudaSuccess) return cuda_error(e, "cudaGetSymbolAddress");
+  }
+  // every argument check of seer_sparse_decode runs before anything is enqueued
+  seer::DecodeLaunch L;
+  const seer_status st = seer::prepare_sparse_decode(dims, q, k, v, block_idx, block_cnt, seqlens, capacity, ns,
+                                                     scratch, need > 0 ? kNoAllocScratchBytes : 0, out, lse_out,
+                                                     err_word, &L);
+  if (st != SEER_OK) return st;
+  if (L.need > 0) {
     // the arrival counters open the workspace layout (B * Hkv int32) and must start at zero
     const size_t counters = (size_t)dims->batch * dims->num_kv_heads * sizeof(int32_t);
-    e = cudaMemsetAsync(scratch, 0, counters, static_cast<cudaStream_t>(stream));
+    cudaError_t e = cudaMemsetAsync(scratch, 0, counters, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_error(e, "clearing the arrival counters");
   }
-  return seer_sparse_decode(dims, q, k, v, block_idx, block_cnt, seqlens, capacity, ns, scratch,
-                            need > 0 ? kNoAllocScratchBytes : 0, out, lse_out, err_word, stream);
+  return seer::launch_prepared_decode(L, static_cast<cudaStream_t>(stream));
 }

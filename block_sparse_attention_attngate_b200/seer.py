@@ -128,9 +128,20 @@ def _need_err(err):
         _need(err, torch.int32, "err")
 
 
+def _need_current_device(t, name: str):
+    """The C calls take bare pointers and launch on the current device: a tensor on another GPU
+    would be read through the wrong device's address space (and the no-allocation call would
+    pick the current device's scratch)."""
+    cur = torch.cuda.current_device()
+    if t.get_device() != cur:
+        raise ValueError(f"{name} is on cuda:{t.get_device()} but the current device is cuda:{cur}; "
+                         f"call under torch.cuda.device({t.get_device()})")
+
+
 def _need(t: torch.Tensor, dtype: torch.dtype, name: str, contiguous: bool = True):
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise TypeError(f"{name} must be a CUDA tensor")
+    _need_current_device(t, name)
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if contiguous and not t.is_contiguous():

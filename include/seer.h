@@ -302,11 +302,13 @@ seer_status seer_sparse_decode(const seer_dims_t* dims, const void* q, const see
  *
  * Arguments and results are those of seer_sparse_decode without workspace/workspace_bytes.
  * Returns SEER_ERR_CAPACITY when the chosen split count needs more scratch than 8 MiB
- * (seer_sparse_decode_workspace_bytes > 8388608); nothing is enqueued then.
+ * (seer_sparse_decode_workspace_bytes > 8388608).  Every argument check of seer_sparse_decode
+ * runs first: on any non-OK status nothing at all is enqueued.
  * The first call on a device looks up the scratch's device address (cudaGetSymbolAddress) with
- * that device current; make that first call before any stream capture.  Each call clears the
- * arrival counters with an async memset on `stream`.  All calls on a device share the scratch:
- * calls that overlap on the GPU race and must be serialised by the caller.  Allocates nothing.
+ * that device current and keeps it for the life of the process; make that first call before any
+ * stream capture, and make no call after cudaDeviceReset.  Each call clears the arrival counters
+ * with an async memset on `stream`.  All calls on a device share the scratch: calls that overlap
+ * on the GPU race and must be serialised by the caller.  Allocates nothing.
  */
 seer_status seer_sparse_decode_noalloc(const seer_dims_t* dims, const void* q, const seer_kv_t* k,
                                        const seer_kv_t* v, const int32_t* block_idx,

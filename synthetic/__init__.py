@@ -16,6 +16,7 @@ from .inputs import (  # noqa: F401
     make_block_lists,
     make_inputs,
     make_logits,
+    make_pair_inputs,
     make_step_query,
     paged_view,
     scale_gate_weights,

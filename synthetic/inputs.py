@@ -149,6 +149,56 @@ def make_step_query(cfg: DecodeConfig, step: int) -> np.ndarray:
     return q
 
 
+def _kv_slice(cfg: DecodeConfig, b: int, h: int, length: int, final: int, lcap: int, q32: np.ndarray,
+              tail: str):
+    """The K and V rows (bf16 bits, [lcap, d]) of one (b, kv-head), and its planted blocks (or None)."""
+    d, blk, g = cfg.head_dim, cfg.block, cfg.g
+    kf = _rng(cfg.seed, _T_K, b, h).standard_normal((lcap, d), dtype=np.float32)
+    vf = _rng(cfg.seed, _T_V, b, h).standard_normal((lcap, d), dtype=np.float32)
+    nfull0 = length // blk
+    chosen = None
+    if cfg.hot_blocks and nfull0 > 0:
+        qs = q32[b, h * g:(h + 1) * g].astype(np.float64).sum(axis=0)
+        qhat = (qs / np.linalg.norm(qs)).astype(np.float32)
+        chosen = sorted(int(x) for x in _rng(cfg.seed, _T_HOT, b, h).choice(
+            nfull0, size=min(cfg.hot_blocks, nfull0), replace=False))
+        for n in chosen:
+            kf[n * blk:(n + 1) * blk] += np.float32(3.0) * qhat
+    k = bf16_bits_from_f32(kf)
+    v = bf16_bits_from_f32(vf)
+    if tail == "nan":
+        k[final:] = BF16_NAN_BITS
+        v[final:] = BF16_NAN_BITS
+    return k, v, chosen
+
+
+@dataclass
+class PairInputs:
+    """The inputs of one (b, kv-head) of a decode problem, as make_inputs draws them."""
+    length: int
+    q: np.ndarray       # uint16 [g, d]  the group's query rows
+    k: np.ndarray       # uint16 [lcap, d]
+    v: np.ndarray       # uint16 [lcap, d]
+    w_q: np.ndarray     # uint16 [d_gate, g*d]
+    w_k: np.ndarray     # uint16 [d_gate, 3*d]
+
+
+def make_pair_inputs(cfg: DecodeConfig, b: int, h: int) -> PairInputs:
+    """One (b, kv-head)'s slices of make_inputs(cfg) (default lengths and tail), drawn from the same
+    streams without drawing the rest of the batch."""
+    d, dg, blk, g = cfg.head_dim, cfg.gate_dim, cfg.block, cfg.g
+    seqlens = _lengths(cfg)
+    final = seqlens + (cfg.steps - 1 if cfg.steps > 1 else 0)
+    lcap = int(-(-int(final.max()) // blk) * blk) if final.max() > 0 else blk
+    q = make_step_query(cfg, 0)
+    k, v, _ = _kv_slice(cfg, b, h, int(seqlens[b]), int(final[b]), lcap, bf16_bits_to_f32(q), "random")
+    w_q = bf16_bits_from_f32(_rng(cfg.seed, _T_WQ, h).standard_normal((dg, g * d), dtype=np.float32)
+                             / np.float32(math.sqrt(g * d)))
+    w_k = bf16_bits_from_f32(_rng(cfg.seed, _T_WK, h).standard_normal((dg, 3 * d), dtype=np.float32)
+                             / np.float32(math.sqrt(3 * d)))
+    return PairInputs(length=int(seqlens[b]), q=q[b, h * g:(h + 1) * g], k=k, v=v, w_q=w_q, w_k=w_k)
+
+
 def make_inputs(cfg: DecodeConfig, *, tail: str = "random",
                 lengths: Optional[Sequence[int]] = None) -> DecodeInputs:
     """Draw one decode problem.
@@ -178,22 +228,9 @@ def make_inputs(cfg: DecodeConfig, *, tail: str = "random",
     hot: Dict[Tuple[int, int], List[int]] = {}
     for b in range(B):
         for h in range(Hkv):
-            kf = _rng(cfg.seed, _T_K, b, h).standard_normal((lcap, d), dtype=np.float32)
-            vf = _rng(cfg.seed, _T_V, b, h).standard_normal((lcap, d), dtype=np.float32)
-            nfull0 = int(seqlens[b]) // blk
-            if cfg.hot_blocks and nfull0 > 0:
-                qs = q32[b, h * g:(h + 1) * g].astype(np.float64).sum(axis=0)
-                qhat = (qs / np.linalg.norm(qs)).astype(np.float32)
-                chosen = sorted(int(x) for x in _rng(cfg.seed, _T_HOT, b, h).choice(
-                    nfull0, size=min(cfg.hot_blocks, nfull0), replace=False))
+            k[b, h], v[b, h], chosen = _kv_slice(cfg, b, h, int(seqlens[b]), int(final[b]), lcap, q32, tail)
+            if chosen is not None:
                 hot[(b, h)] = chosen
-                for n in chosen:
-                    kf[n * blk:(n + 1) * blk] += np.float32(3.0) * qhat
-            k[b, h] = bf16_bits_from_f32(kf)
-            v[b, h] = bf16_bits_from_f32(vf)
-            if tail == "nan":
-                k[b, h, int(final[b]):] = BF16_NAN_BITS
-                v[b, h, int(final[b]):] = BF16_NAN_BITS
     return DecodeInputs(cfg=cfg, seqlens=seqlens, final_lens=final.astype(np.int32), q=q, k=k, v=v,
                         w_q=w_q, w_k=w_k, hot=hot)
 

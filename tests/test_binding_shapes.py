@@ -132,3 +132,22 @@ def test_prefill_gt_shapes():
                       ("lse", torch.zeros(B, HQ, T + 1)), ("q", torch.zeros(B, 4, T, D)),
                       ("k", _cache(torch.zeros(B, 1, NB * BLK, D)))):
         _rejects(S.prefill_gt, good, name, bad)
+
+
+def test_tensors_must_be_on_the_current_device(monkeypatch):
+    """The C calls launch on the current device with bare pointers: a tensor on another GPU is
+    refused before any call (checked here with a stand-in device index, no GPU needed)."""
+
+    class OnDevice1:
+        def get_device(self):
+            return 1
+
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    with pytest.raises(ValueError, match="cuda:1 but the current device is cuda:0"):
+        S.seer._need_current_device(OnDevice1(), "q")
+
+    class OnDevice0:
+        def get_device(self):
+            return 0
+
+    S.seer._need_current_device(OnDevice0(), "q")

@@ -19,8 +19,8 @@ import pytest
 import torch
 
 from oracle import seer_oracle as O
-from seer_harness import (OracleBH, bf16_bits, check_attention, check_kcomp_rows, check_logits, check_logits_e2e,
-                          check_lse, check_selection, e2e_logit_bound, f64, gpu_list, to_dev_bf16)
+from seer_harness import (LOGIT_RTOL, OracleBH, bf16_bits, check_attention, check_kcomp_rows, check_logits,
+                          check_logits_e2e, check_lse, check_selection, e2e_logit_bound, f64, gpu_list, to_dev_bf16)
 from synthetic import (SWEEP_SPARSITIES, bf16_bits_from_f32, config, make_inputs, make_step_query,
                        scale_gate_weights)
 from synthetic.inputs import sweep_budget
@@ -69,7 +69,18 @@ def _boundary_ok(z, gpu, ref, mode, bound, k_blocks=0, tau=0.0):
 
 
 def _run_and_check(P, step, q_bits, lengths, mode, k_blocks=0, tau=0.0, pairs=None, attn_pairs=None, label=""):
-    """One GPU step vs the oracle; returns (selection mismatches, pairs compared)."""
+    """One GPU step vs the oracle; returns (selection mismatches against the all-oracle step,
+    pairs compared, the oracle's lists).
+
+    Per (b, h):
+      * the GPU logits against the oracle's logits evaluated on the cache rows the GPU step
+        itself read (widened exactly from bf16), at the plain logit tolerance;
+      * the GPU list against the oracle's selection on those same logits: identical, except a
+        block whose logit sits within twice the logit tolerance of the cut-off;
+      * the GPU list against the all-oracle step (oracle cache): identical except at the
+        cut-off (the two caches may round an entry one ulp apart);
+      * the GPU output and LSE against the oracle's attention over the GPU's own list.
+    """
     c = P.cfg
     seq = torch.from_numpy(np.asarray(lengths, np.int32)).cuda()
     q = to_dev_bf16(q_bits)
@@ -78,6 +89,7 @@ def _run_and_check(P, step, q_bits, lengths, mode, k_blocks=0, tau=0.0, pairs=No
     assert int(step.err.item()) == 0, f"{label}: device error word {int(step.err.item())}"
     idx, cnt = step.block_idx.cpu().numpy(), step.block_cnt.cpu().numpy()
     lg = step.logits.cpu().numpy()
+    kc_gpu = f64(bf16_bits(step.kcomp))   # the cache rows this step's gate read
     o = f64(bf16_bits(out))
     lse = step.lse.cpu().numpy()
     pairs = pairs or sorted(P.obh)
@@ -89,18 +101,32 @@ def _run_and_check(P, step, q_bits, lengths, mode, k_blocks=0, tau=0.0, pairs=No
         ob = P.obh[(b, h)]
         ref = ob.step(L, q_bits, mode, k_blocks=k_blocks, tau=tau, w_q_bits=P.w_q_bits)
         nfull = L // c.block
+        got = gpu_list(idx[b, h], cnt[b, h])
+        # logits and selection on the GPU's own cache rows
+        z_own = O.gate_logits(ref["q_gate"], kc_gpu[b, h], L, c.block)
+        check_logits(lg[b, h, :nfull], z_own, f"{label} logits on the GPU cache b{b} h{h}")
+        own = O.select_topk(z_own, k_blocks, L, c.block) if mode == "topk" else O.select_threshold(z_own, tau, L, c.block)
+        if nfull:
+            rms = math.sqrt(float(np.mean(z_own ** 2)))
+            own_bound = LOGIT_RTOL * np.maximum(np.abs(z_own), rms)
+            assert _boundary_ok(z_own, got, own, mode, own_bound, k_blocks, tau), \
+                f"{label} b{b} h{h}: list differs from the selection on the GPU cache away from the cut-off: " \
+                f"{sorted(set(got) ^ set(own))}"
+        else:
+            assert got == own, f"{label} b{b} h{h}: {got} vs {own}"
+        # against the all-oracle step
         bound = e2e_logit_bound(ref["q_gate"], ob.kcomp(L)[:nfull], ref["logits"])
         check_logits_e2e(lg[b, h, :nfull], ref["logits"], bound, f"{label} e2e logits b{b} h{h}")
-        got = gpu_list(idx[b, h], cnt[b, h])
         oracle_lists[(b, h)] = ref["blocks"]
         if got != ref["blocks"]:
             mism += 1
             assert _boundary_ok(ref["logits"], got, ref["blocks"], mode, bound, k_blocks, tau), \
                 f"{label} b{b} h{h}: lists differ away from the cutoff: {sorted(set(got) ^ set(ref['blocks']))}"
-        elif (b, h) in attn_pairs:
+        if (b, h) in attn_pairs:
             g = c.g
-            check_attention(o[b, h * g:(h + 1) * g], ref["o"], f"{label} e2e out b{b} h{h}")
-            check_lse(lse[b, h * g:(h + 1) * g], ref["lse"], f"{label} e2e lse b{b} h{h}")
+            ro, rl = (ref["o"], ref["lse"]) if got == ref["blocks"] else ob.attention(L, q_bits, got)
+            check_attention(o[b, h * g:(h + 1) * g], ro, f"{label} e2e out b{b} h{h}")
+            check_lse(lse[b, h * g:(h + 1) * g], rl, f"{label} e2e lse b{b} h{h}")
     return mism, len(pairs), oracle_lists
 
 
@@ -201,6 +227,32 @@ def test_topk_workload(cid):
                    for (b, h) in inp.hot)
         total = sum(len(v) for v in inp.hot.values())
         print(f"cfg{cid}: planted blocks selected {hits}/{total}")
+
+
+def test_paged_ragged_workload():
+    """The Qwen3-14B-shaped ragged batch (g = 5, block 128, lengths never a multiple of 128, so the
+    partial block is forced on; four of its sequences) on a paged cache: pages shuffled by a seeded
+    permutation, NaN in every unused page and past each length.  Cache rebuild, logits, lists and
+    outputs through DecodeStep against the oracle, as for the contiguous workloads."""
+    from synthetic import paged_view
+    cfg = config(3, B=4)
+    inp = make_inputs(cfg, tail="nan")
+    P = Problem(inp)
+    L = inp.seqlens
+    assert np.all(L % cfg.block != 0)
+    pool_k, table = paged_view(inp.k, cfg.block, seed=31)
+    pool_v, _ = paged_view(inp.v, cfg.block, seed=31)
+    tbl = torch.from_numpy(table).cuda()
+    kk = S.KVCache.paged(to_dev_bf16(pool_k), tbl)
+    vv = S.KVCache.paged(to_dev_bf16(pool_v), tbl)
+    S.kcomp_update(P.sh, kk, torch.from_numpy(L).cuda(), P.valid, P.w_k, P.kc)
+    torch.cuda.synchronize()
+    _check_kcomp(P, L)
+    step = S.DecodeStep(P.sh, kk, vv, P.w_q, P.w_k, P.kc, P.valid, mode=S.SELECT_TOPK, token_budget=cfg.budget)
+    mism, n, _ = _run_and_check(P, step, inp.q, L, "topk", k_blocks=cfg.topk_blocks, label="paged cfg3")
+    assert mism <= max(1, n // 20), f"paged cfg3: {mism}/{n} lists differ (all at the cutoff)"
+    cnt = step.block_cnt.cpu().numpy()
+    assert np.all(cnt == cfg.topk_blocks + 1), "every list holds k blocks plus the forced partial block"
 
 
 def test_sparsity_sweep_and_dense_path():

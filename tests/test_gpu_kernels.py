@@ -244,7 +244,10 @@ def test_sparse_decode_many_short_lists(ns):
             check_lse(lh[b, h * g:(h + 1) * g], rl, f"b{b} h{h}")
 
 
-def test_sparse_decode_paged_matches_contiguous():
+@pytest.mark.parametrize("ns", [3, 0, -1])
+def test_sparse_decode_paged_matches_contiguous(ns):
+    """A paged cache (shuffled pages, NaN in every unused page) against the oracle, under each
+    schedule; the paged and contiguous results are also bit-identical (same tiles, same order)."""
     blk, d, g, Hkv = 64, 128, 4, 2
     cfg = config(1, B=2, Hq=g * Hkv, Hkv=Hkv, head_dim=d, gate_dim=64, block=blk, seed=1313)
     lengths = [10 * blk + 5, 7 * blk]
@@ -265,21 +268,37 @@ def test_sparse_decode_paged_matches_contiguous():
         else:
             kk, vv = S.KVCache.contiguous(dv["k"]), S.KVCache.contiguous(dv["v"])
         out = torch.empty((cfg.B, cfg.Hq, d), dtype=torch.bfloat16, device="cuda")
-        ws = S.alloc_workspace(sh, cap, 3)
-        S.sparse_decode(sh, dv["q"], kk, vv, idx_d, cnt_d, dv["seqlens"], out, ws, num_split=3)
+        lse = torch.empty((cfg.B, cfg.Hq), dtype=torch.float32, device="cuda")
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        ws = S.alloc_workspace(sh, cap, ns)
+        S.sparse_decode(sh, dv["q"], kk, vv, idx_d, cnt_d, dv["seqlens"], out, ws, num_split=ns, lse=lse, err=err)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0, f"{layout}: device error word {int(err.item())}"
+        o, lh = f64(bf16_bits(out)), lse.cpu().numpy()
+        for b in range(cfg.B):
+            for h in range(Hkv):
+                ro, rl = OracleBH(inp, b, h).attention(lengths[b], inp.q, gpu_list(idx[b, h], cnt[b, h]))
+                check_attention(o[b, h * g:(h + 1) * g], ro, f"{layout} ns={ns} b{b} h{h}")
+                check_lse(lh[b, h * g:(h + 1) * g], rl, f"{layout} ns={ns} b{b} h{h}")
         outs.append(out)
     assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16)), "paged != contiguous"
-    # paged kcomp equals contiguous kcomp
+    # the paged cache rebuild against the oracle's cache, and bit-identical to the contiguous one
     kcs = []
     for kk in (S.KVCache.contiguous(dv["k"]), S.KVCache.paged(to_dev_bf16(pool_k), tbl)):
         kc = torch.zeros((cfg.B, Hkv, inp.max_blocks, 64), dtype=torch.bfloat16, device="cuda")
         S.kcomp_update(sh, kk, dv["seqlens"], torch.zeros(cfg.B, Hkv, dtype=torch.int32, device="cuda"), dv["w_k"], kc)
         kcs.append(kc)
+    got = bf16_bits(kcs[1])
+    for b in range(cfg.B):
+        for h in range(Hkv):
+            nfull = lengths[b] // blk
+            check_kcomp_rows(got[b, h, :nfull], OracleBH(inp, b, h).kcomp(lengths[b])[:nfull], f"paged kcomp b{b} h{h}")
     assert torch.equal(kcs[0].view(torch.int16), kcs[1].view(torch.int16)), "paged kcomp != contiguous"
 
 
 def test_sparse_decode_token_major_layout():
-    """A [B, T, Hkv, d] cache (token-major, vLLM-style strides) gives the same result."""
+    """A [B, T, Hkv, d] cache (token-major, vLLM-style strides) against the oracle; it also
+    gives the same bits as the head-major layout."""
     blk, d, g, Hkv = 64, 128, 4, 2
     cfg = config(1, B=2, Hq=g * Hkv, Hkv=Hkv, head_dim=d, gate_dim=64, block=blk, seed=1414)
     lengths = [6 * blk + 9, 4 * blk]
@@ -297,8 +316,16 @@ def test_sparse_decode_token_major_layout():
         else:
             k4, v4 = dv["k"], dv["v"]
         out = torch.empty((cfg.B, cfg.Hq, d), dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty((cfg.B, cfg.Hq), dtype=torch.float32, device="cuda")
         S.sparse_decode(sh, dv["q"], S.KVCache.contiguous(k4), S.KVCache.contiguous(v4), idx_d, cnt_d,
-                        dv["seqlens"], out, S.alloc_workspace(sh, cap, 2), num_split=2)
+                        dv["seqlens"], out, S.alloc_workspace(sh, cap, 2), num_split=2, lse=lse)
+        torch.cuda.synchronize()
+        o, lh = f64(bf16_bits(out)), lse.cpu().numpy()
+        for b in range(cfg.B):
+            for h in range(Hkv):
+                ro, rl = OracleBH(inp, b, h).attention(lengths[b], inp.q, gpu_list(idx[b, h], cnt[b, h]))
+                check_attention(o[b, h * g:(h + 1) * g], ro, f"token-major={tm} b{b} h{h}")
+                check_lse(lh[b, h * g:(h + 1) * g], rl, f"token-major={tm} b{b} h{h}")
         outs.append(out)
     assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
 

@@ -7,7 +7,7 @@ import math
 
 import numpy as np
 
-from synthetic import CONFIGS, bf16_bits_to_f32, config, make_inputs
+from synthetic import CONFIGS, bf16_bits_to_f32, config, make_inputs, make_pair_inputs
 from synthetic.inputs import BF16_NAN_BITS, _lengths
 
 
@@ -75,3 +75,18 @@ def test_hot_blocks_and_nan_tail():
             assert abs(m) < 0.5, f"block {n}: mean projection {m:.2f}"
     assert np.all(inp.k[0, 0, L:] == BF16_NAN_BITS) and np.all(inp.v[0, 0, L:] == BF16_NAN_BITS)
     assert not np.any(inp.k[0, 0, :L] == BF16_NAN_BITS)
+
+
+def test_pair_inputs_are_the_batch_slices():
+    """One (b, kv-head) drawn on its own equals the same slice of the whole batch (planted blocks
+    and ragged lengths included)."""
+    for cid, over in ((2, dict(B=2, Hkv=2, Hq=8, length=1000)), (3, dict(B=3, Hkv=2, Hq=10))):
+        cfg = config(cid, **over)
+        inp = make_inputs(cfg)
+        for b in range(cfg.B):
+            for h in range(cfg.Hkv):
+                pi = make_pair_inputs(cfg, b, h)
+                assert pi.length == int(inp.seqlens[b])
+                assert np.array_equal(pi.k, inp.k[b, h]) and np.array_equal(pi.v, inp.v[b, h])
+                assert np.array_equal(pi.q, inp.q[b, h * cfg.g:(h + 1) * cfg.g])
+                assert np.array_equal(pi.w_q, inp.w_q[h]) and np.array_equal(pi.w_k, inp.w_k[h])
