@@ -57,9 +57,9 @@ def parse():
     ap.add_argument("--budget", type=int, default=0, help="override the token budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="skip the sparsity sweep rows")
-    ap.add_argument("--only", default="all", choices=["all", "decode", "truth", "prefill"],
-                    help="decode / truth / prefill: run just the sparse-decode / ground-truth / prefill-with-targets "
-                         "launches (small targets for profilers)")
+    ap.add_argument("--only", default="all", choices=["all", "step", "decode", "truth", "prefill"],
+                    help="step / decode / truth / prefill: run just the one-launch step / sparse-decode / "
+                         "ground-truth / prefill-with-targets launches (small targets for profilers)")
     return ap.parse_args()
 
 
@@ -97,17 +97,25 @@ def _peaks():
         return 6650.0, "fallback"
 
 
-def _profiled_traffic(summary="sparse_decode_kernel.qwen3-8b-32k-decode.md", source="sparse_decode.cu"):
+STEP_SOURCES = ["sparse_decode.cu", "step_plan.cuh", "gate_device.cuh", "select_device.cuh", "kcomp_device.cuh",
+                "seer_device.cuh"]
+
+
+def _profiled_traffic(summary="decode_step_kernel.qwen3-8b-32k-decode-step.md", sources=None):
     """DRAM bytes (read + write) per launch of a kernel from its committed ncu summary, or None
-    when the kernel source has changed since those counters were taken."""
+    when the kernel's sources have changed since those counters were taken (sha256 of the sources'
+    bytes, concatenated in the order given)."""
     import hashlib
+    sources = sources or STEP_SOURCES
     try:
         with open(os.path.join(ROOT, "profiles", summary)) as f:
             fields = dict(line.split(": ", 1) for line in f.read().splitlines() if ": " in line
                           and line.split(": ", 1)[0] in ("source_sha256", "traffic_bytes_per_launch"))
-        with open(os.path.join(ROOT, "block_sparse_attention_attngate_b200", "csrc", source), "rb") as f:
-            current = hashlib.sha256(f.read()).hexdigest()
-        if fields.get("source_sha256", "").strip() != current:
+        h = hashlib.sha256()
+        for src in sources:
+            with open(os.path.join(ROOT, "block_sparse_attention_attngate_b200", "csrc", src), "rb") as f:
+                h.update(f.read())
+        if fields.get("source_sha256", "").strip() != h.hexdigest():
             return None
         return int(fields["traffic_bytes_per_launch"])
     except Exception:
@@ -279,63 +287,108 @@ def run_reference(args):
 
 # ---------------------------------------------------------------------------- GPU arm
 
-def sweep_rows(S, dev, stream, peak, shape2, reps2, seqlens2, cfg2, inp2, iters=60, warm=5):
-    """The roofline rows besides the headline step: config 2 at k = 52 (89.8 % sparse) and the
-    64k sweep (config 4) at 50/75/90/95 % sparsity plus its all-blocks dense path.  Block lists
-    come from the plan kernel; the sparse decode alone is timed (eager launches rotating over
-    three replicas of the K/V cache, CUDA events)."""
+def _up(bits, dev):
     import torch
-    from synthetic import SWEEP_SPARSITIES, config, make_inputs, sweep_budget
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
 
-    def time_decode(steps_, q_list, seql):
-        R = len(steps_)
 
-        def one(i):
-            st = steps_[i % R]
-            S.sparse_decode(st.shape, q_list[i % R], st.k, st.v, st.block_idx, st.block_cnt, seql, st.out,
-                            st.workspace, st.num_split, st.lse, st.err, stream=stream)
-        with torch.cuda.stream(stream):
-            for i in range(warm):
-                one(i)
-        stream.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for i in range(iters):
-                one(i)
-            e1.record(stream)
-        e1.synchronize()
-        return e0.elapsed_time(e1) / iters * 1e3
+def time_decode_alone(S, steps_, q_list, seql, stream, iters=60, warm=5):
+    """Mean device time of the sparse decode alone (eager launches rotating over the replicas)."""
+    import torch
+    R = len(steps_)
 
-    def row(cfg, inp, steps_, q_list, seql, extra):
-        st = steps_[0]
-        with torch.cuda.stream(stream):
-            for r, s_ in enumerate(steps_):
-                s_.run(q_list[r], seql, stream=stream)
-        stream.synchronize()
-        cnt_h, idx_h = st.block_cnt.cpu().numpy(), st.block_idx.cpu().numpy()
-        nb = algorithmic_bytes(cfg, inp.seqlens, cnt_h, idx_h, st.capacity, inp.max_blocks)
-        us = time_decode(steps_, q_list, seql)
-        gbs = nb["decode"] / (us * 1e-6) / 1e9
-        out = {"decode_us": us, "achieved_gbs": gbs, "frac": gbs / peak, "bytes": nb["decode"],
-               "sparsity": 1.0 - float(cnt_h.mean()) / inp.max_blocks, "num_split": st.num_split}
-        out.update(extra)
-        return out
+    def one(i):
+        st = steps_[i % R]
+        S.sparse_decode(st.shape, q_list[i % R], st.k, st.v, st.block_idx, st.block_cnt, seql, st.out, st.workspace,
+                        st.num_split, st.lse, st.err, stream=stream)
+    with torch.cuda.stream(stream):
+        for i in range(warm):
+            one(i)
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(iters):
+            one(i)
+        e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / iters * 1e3
 
-    def steps_for(shape, reps_kv, w_q, w_k, kcs, valids, budget):
-        return [S.DecodeStep(shape, S.KVCache.contiguous(k), S.KVCache.contiguous(v), w_q, w_k, kc, valid,
-                             mode=S.SELECT_TOPK, token_budget=budget)
-                for (k, v), kc, valid in zip(reps_kv, kcs, valids)]
 
-    res = {}
-    # decode ground truth (full attention scores of every block) on the 32k step: reads all of K
-    sh_t = shape2
-    ws_t = S.alloc_truth_workspace(sh_t, dev)
+def time_step_graph(steps_, q_list, seql, stream, per_graph=30, replays=8, warm=2):
+    """Mean device time of one whole step: a CUDA graph of `per_graph` consecutive steps rotating over
+    the replicas (no host work between launches), replayed `replays` times."""
+    import torch
+    R = len(steps_)
+    with torch.cuda.stream(stream):
+        for r in range(R):
+            steps_[r].run(q_list[r], seql, stream=stream)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(per_graph):
+            steps_[i % R].run(q_list[i % R], seql, stream=stream)
+    with torch.cuda.stream(stream):
+        for _ in range(warm):
+            g.replay()
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(replays):
+            g.replay()
+        e1.record(stream)
+    e1.synchronize()
+    us = e0.elapsed_time(e1) / (replays * per_graph) * 1e3
+    del g
+    return us
+
+
+def measure_row(S, cfg, inp, steps_, q_list, seql, stream, peak, extra=None):
+    """One roofline row: the whole step as the product runs it (one launch where the shape allows)
+    against the step's algorithmic bytes, and the sparse decode alone against its own."""
+    import torch
+    st = steps_[0]
+    with torch.cuda.stream(stream):
+        for r, s_ in enumerate(steps_):
+            s_.run(q_list[r], seql, stream=stream)
+    stream.synchronize()
+    assert all(int(s_.err.item()) == 0 for s_ in steps_), "device error word set"
+    cnt_h, idx_h = st.block_cnt.cpu().numpy(), st.block_idx.cpu().numpy()
+    nb = algorithmic_bytes(cfg, inp.seqlens, cnt_h, idx_h, st.capacity, inp.max_blocks)
+    step_us = time_step_graph(steps_, q_list, seql, stream)
+    dec_us = time_decode_alone(S, steps_, q_list, seql, stream)
+    one_us = None
+    if st.num_split == -1 and S.decode_step_supported(st.shape, st.mode, st.capacity):
+        one = [S.DecodeStep(s_.shape, s_.k, s_.v, s_.w_q, s_.w_k, s_.kcomp, s_.valid_blocks, mode=s_.mode,
+                            token_budget=s_.token_budget, tau=s_.tau, num_split=-1, single_launch=True) for s_ in steps_]
+        one_us = time_step_graph(one, q_list, seql, stream)
+        del one
+    out = {"step_us": step_us, "step_bytes": nb["step"], "step_gbs": nb["step"] / (step_us * 1e-6) / 1e9,
+           "step_frac": nb["step"] / (step_us * 1e-6) / 1e9 / peak, "step_launches": st.kernels_per_step,
+           "one_launch_step_us": one_us,
+           "decode_us": dec_us, "bytes": nb["decode"], "achieved_gbs": nb["decode"] / (dec_us * 1e-6) / 1e9,
+           "frac": nb["decode"] / (dec_us * 1e-6) / 1e9 / peak,
+           "sparsity": 1.0 - float(cnt_h.mean()) / inp.max_blocks, "num_split": st.num_split}
+    out.update(extra or {})
+    return out
+
+
+def make_steps(S, shape, reps_kv, w_q, w_k, kcs, valids, budget, **kw):
+    return [S.DecodeStep(shape, kv_k, kv_v, w_q, w_k, kc, valid, mode=S.SELECT_TOPK, token_budget=budget, **kw)
+            for (kv_k, kv_v), kc, valid in zip(reps_kv, kcs, valids)]
+
+
+def truth_row(S, stream, peak, shape2, reps2, seqlens2, cfg2, inp2, iters=60, warm=5):
+    """The decode ground truth (full attention scores of every block) on the 32k step: reads all of K."""
+    import torch
+    dev = seqlens2.device
+    ws_t = S.alloc_truth_workspace(shape2, dev)
     sc_t = torch.empty(cfg2.B, cfg2.Hkv, inp2.max_blocks, dtype=torch.float32, device=dev)
     kvs_t = [S.KVCache.contiguous(rp["k"]) for rp in reps2]
 
     def truth(i):
-        S.gate_truth(sh_t, reps2[i % len(reps2)]["q"], kvs_t[i % len(reps2)], seqlens2, sc_t, ws_t, stream=stream)
+        S.gate_truth(shape2, reps2[i % len(reps2)]["q"], kvs_t[i % len(reps2)], seqlens2, sc_t, ws_t, stream=stream)
     with torch.cuda.stream(stream):
         for i in range(warm):
             truth(i)
@@ -350,54 +403,206 @@ def sweep_rows(S, dev, stream, peak, shape2, reps2, seqlens2, cfg2, inp2, iters=
     us_t = e0.elapsed_time(e1) / iters * 1e3
     k_bytes = int(sum(int(L) for L in inp2.seqlens)) * cfg2.Hkv * cfg2.head_dim * 2
     t_bytes = k_bytes + cfg2.B * cfg2.Hq * cfg2.head_dim * 2 + cfg2.B * cfg2.Hkv * inp2.max_blocks * 4
-    res["ground-truth-32k"] = {"us": us_t, "bytes": t_bytes, "achieved_gbs": t_bytes / (us_t * 1e-6) / 1e9,
-                               "frac": t_bytes / (us_t * 1e-6) / 1e9 / peak,
-                               "traffic": _profiled_traffic("truth_kernel.qwen3-8b-32k-ground-truth.md", "gate_truth.cu"),
-                               "what": "seer_gate_truth: all of K read once (K bytes + q + scores)"}
-    del ws_t, sc_t
-    # config 2 at k = 52
-    b52 = 3277
-    st2 = steps_for(shape2, [(rp["k"], rp["v"]) for rp in reps2], reps2[0]["step"].w_q, reps2[0]["step"].w_k,
-                    [rp["step"].kcomp for rp in reps2], [rp["step"].valid_blocks for rp in reps2], b52)
-    res["qwen3-8b-32k-k52"] = row(cfg2, inp2, st2, [rp["q"] for rp in reps2], seqlens2,
-                                  {"token_budget": b52, "k": -(-b52 // cfg2.block)})
-    del st2
-    # config 4: 64k context, sparsity sweep and the dense path
-    cfg4 = config(4)
-    inp4 = make_inputs(cfg4)
+    return {"us": us_t, "bytes": t_bytes, "achieved_gbs": t_bytes / (us_t * 1e-6) / 1e9,
+            "frac": t_bytes / (us_t * 1e-6) / 1e9 / peak,
+            "traffic": _profiled_traffic("truth_kernel.qwen3-8b-32k-ground-truth.md", ["gate_truth.cu"]),
+            "what": "seer_gate_truth: all of K read once (K bytes + q + scores)"}
 
-    def up(bits):
-        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+
+def _replicas(S, cfg, inp, shape, dev, R=3, paged_seed=None):
+    """R copies of a workload's K / V on the device (contiguous, or paged with the pages shuffled by a
+    seeded permutation), each with its own prefilled K Compression Cache."""
+    import torch
+    w_k = _up(inp.w_k, dev)
+    seq = torch.from_numpy(inp.seqlens).to(dev)
+    k0, v0 = _up(inp.k, dev), _up(inp.v, dev)
+    out = []
+    for r in range(R):
+        k = k0 if r == 0 else k0.clone()
+        v = v0 if r == 0 else v0.clone()
+        if paged_seed is None:
+            kv_k, kv_v = S.KVCache.contiguous(k), S.KVCache.contiguous(v)
+        else:
+            B, H, T, d = k.shape
+            blk = cfg.block
+            npb = T // blk
+            perm = torch.from_numpy(np.random.default_rng(paged_seed + r).permutation(B * npb).astype(np.int32)).to(dev)
+            table = perm.view(B, npb).contiguous()
+
+            def pool_of(x):
+                pages = x.view(B, H, npb, blk, d).permute(0, 2, 1, 3, 4).reshape(B * npb, H, blk, d)
+                pool = torch.empty_like(pages)
+                pool[perm.long()] = pages
+                return pool
+            kv_k, kv_v = S.KVCache.paged(pool_of(k), table), S.KVCache.paged(pool_of(v), table)
+            del k, v
+        kc = torch.zeros(cfg.B, cfg.Hkv, inp.max_blocks, cfg.gate_dim, dtype=torch.bfloat16, device=dev)
+        valid = torch.zeros(cfg.B, cfg.Hkv, dtype=torch.int32, device=dev)
+        S.kcomp_update(shape, kv_k, seq, valid, w_k, kc)
+        out.append(dict(kv=(kv_k, kv_v), kc=kc, valid=valid))
+    return out, seq, w_k
+
+
+def threshold_loop_row(S, dev, stream, peak, workers, steps=256):
+    """The 256-step decode loop with threshold selection (Qwen3-8B-shaped heads, B = 32, start
+    context 16384): one token per step, the K Compression Cache filling every 64 steps, per-head
+    gate temperatures set at step 0 so that the median sequence of head h selects f_h of the blocks
+    (f_h spaced 5 %..24 %), tau = 1/512.  The whole loop is one CUDA graph (the fill counts reset at
+    its start), so a step's time is the loop's over its steps; the realised spread of selected
+    fractions is recorded per step."""
+    import torch
+    from synthetic import config, make_inputs, make_step_query, scale_gate_weights
+    cfg = config(5)
+    inp = make_inputs(cfg, workers=workers)
+    B, Hq, Hkv, d, blk = cfg.B, cfg.Hq, cfg.Hkv, cfg.head_dim, cfg.block
+    NB = inp.max_blocks
+    shape = S.Shape(B, Hq, Hkv, d, cfg.gate_dim, blk, NB, cfg.rope_base)
+    reps, seq0, w_k = _replicas(S, cfg, inp, shape, dev, R=1)
+    kv_k, kv_v = reps[0]["kv"]
+    kc, valid = reps[0]["kc"], reps[0]["valid"]
+    # per-head temperatures from the step-0 logits of the unscaled gate (logits scale with c)
+    L1 = torch.from_numpy(inp.seqlens + 1).to(dev)
+    lg = torch.empty(B, Hkv, NB, dtype=torch.float32, device=dev)
+    S.gate_score(shape, _up(make_step_query(cfg, 0), dev), _up(inp.w_q, dev), kc, L1, lg)
+    nfull = (int(inp.seqlens[0]) + 1) // blk
+    z = lg[:, :, :nfull].double().cpu().numpy()
+    fr = np.linspace(0.05, 0.24, Hkv)
+
+    def count(c, zz):
+        e = np.exp(c * (zz - zz.max()))
+        return int((e / e.sum() > cfg.tau).sum())
+    temps = []
+    for h in range(Hkv):
+        lo, hi = 1e-3, 1e3
+        for _ in range(60):
+            mid = math.sqrt(lo * hi)
+            if np.median([count(mid, z[b, h]) for b in range(B)]) > fr[h] * nfull:
+                lo = mid
+            else:
+                hi = mid
+        temps.append(math.sqrt(lo * hi))
+    w_q = _up(scale_gate_weights(inp.w_q, temps), dev)
+    q_tab = torch.stack([_up(make_step_query(cfg, s_), dev) for s_ in range(steps)])
+    seq_tab = torch.from_numpy(np.stack([inp.seqlens + s_ + 1 for s_ in range(steps)]).astype(np.int32)).to(dev)
+    valid0 = valid.clone()
+    res = {"what": "256-step threshold loop, B=32, Hq=32, Hkv=8, d=128, b=64, L=16385..16640, tau=1/512",
+           "temperatures": temps}
+    for name, ns in (("balanced", 0), ("capacity", -1)):
+        st = S.DecodeStep(shape, kv_k, kv_v, w_q, w_k, kc, valid, mode=S.SELECT_THRESHOLD, tau=cfg.tau,
+                          num_split=ns)
+        # one eager pass recording the counts (and the bytes they imply)
+        valid.copy_(valid0)
+        cnts = []
+        with torch.cuda.stream(stream):
+            for s_ in range(steps):
+                st.run(q_tab[s_], seq_tab[s_], stream=stream)
+                cnts.append(st.block_cnt.clone())
+        stream.synchronize()
+        assert int(st.err.item()) == 0
+        cnt = torch.stack(cnts).cpu().numpy().astype(np.int64)            # [steps, B, Hkv]
+        Ls = seq_tab.cpu().numpy().astype(np.int64)[:, :, None]            # [steps, B, 1]
+        part = (Ls % blk != 0).astype(np.int64)
+        tok = (cnt - part) * blk + part * (Ls % blk)
+        kv_bytes = tok.sum(axis=(1, 2)) * d * 2 * 2
+        per_step_bytes = kv_bytes + 2 * B * Hq * d * 2 + B * Hkv * (st.capacity + 1) * 4
+        gate = B * Hkv * (Ls[:, :, 0] // blk).mean(axis=1) * cfg.gate_dim * 2 + Hkv * cfg.gate_dim * cfg.g * d * 2
+        step_bytes = per_step_bytes + gate + B * Hkv * NB * 4 * 2
+        frac_sel = cnt / np.ceil(Ls / blk)
+        g_ = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_, stream=stream):
+            valid.copy_(valid0)
+            for s_ in range(steps):
+                st.run(q_tab[s_], seq_tab[s_], stream=stream)
+        with torch.cuda.stream(stream):
+            g_.replay()
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(3):
+                g_.replay()
+            e1.record(stream)
+        e1.synchronize()
+        us = e0.elapsed_time(e1) / (3 * steps) * 1e3
+        del g_
+        sb = float(step_bytes.mean())
+        res[name] = {"step_us": us, "step_bytes_mean": sb, "step_gbs": sb / (us * 1e-6) / 1e9,
+                     "step_frac": sb / (us * 1e-6) / 1e9 / peak, "launches_per_step": st.kernels_per_step,
+                     "selected_fraction": {"min": float(frac_sel.min()), "median": float(np.median(frac_sel)),
+                                           "max": float(frac_sel.max()),
+                                           "within_2_30": float(((frac_sel >= 0.02) & (frac_sel <= 0.30)).mean()),
+                                           "per_step_median_min": float(np.median(frac_sel, axis=(1, 2)).min()),
+                                           "per_step_median_max": float(np.median(frac_sel, axis=(1, 2)).max())}}
+        del st
+    torch.cuda.synchronize()
+    return res
+
+
+def sweep_rows(S, dev, stream, peak, shape2, reps2, seqlens2, cfg2, inp2, workers):
+    """The roofline rows besides the headline step, each as the whole step (one launch where the
+    shape allows) and as the sparse decode alone: the 32k step at k = 52 (89.8 % sparse), the 64k
+    sweep at 50/75/90/95 % sparsity and its all-blocks dense path, the ragged Qwen3-14B-shaped batch,
+    the 32k step on a paged cache, the 256-step threshold loop; plus the ground-truth scorer and the
+    prefill forward with targets."""
+    import torch
+    from synthetic import SWEEP_SPARSITIES, config, make_inputs, sweep_budget
+    res = {"ground-truth-32k": truth_row(S, stream, peak, shape2, reps2, seqlens2, cfg2, inp2)}
+    q2 = [rp["q"] for rp in reps2]
+    kv2 = [(rp["step"].k, rp["step"].v) for rp in reps2]
+    w_q2, w_k2 = reps2[0]["step"].w_q, reps2[0]["step"].w_k
+    kcs2, valids2 = [rp["step"].kcomp for rp in reps2], [rp["step"].valid_blocks for rp in reps2]
+    b52 = 3277
+    st2 = make_steps(S, shape2, kv2, w_q2, w_k2, kcs2, valids2, b52)
+    res["qwen3-8b-32k-k52"] = measure_row(S, cfg2, inp2, st2, q2, seqlens2, stream, peak,
+                                          {"token_budget": b52, "k": -(-b52 // cfg2.block)})
+    del st2
+    # the 32k step on a paged cache (pages shuffled, one page per block)
+    reps_p, _, _ = _replicas(S, cfg2, inp2, shape2, dev, paged_seed=2024)
+    stp = make_steps(S, shape2, [r["kv"] for r in reps_p], w_q2, w_k2, [r["kc"] for r in reps_p],
+                     [r["valid"] for r in reps_p], cfg2.budget)
+    res["qwen3-8b-32k-paged"] = measure_row(S, cfg2, inp2, stp, q2, seqlens2, stream, peak,
+                                            {"token_budget": cfg2.budget, "layout": "paged, page = block"})
+    del stp, reps_p
+    torch.cuda.empty_cache()
+    # 64k context: sparsity sweep and the dense path
+    cfg4 = config(4)
+    inp4 = make_inputs(cfg4, workers=workers)
     NB4 = inp4.max_blocks
     shape4 = S.Shape(cfg4.B, cfg4.Hq, cfg4.Hkv, cfg4.head_dim, cfg4.gate_dim, cfg4.block, NB4, cfg4.rope_base)
-    w_q4, w_k4 = up(inp4.w_q), up(inp4.w_k)
-    seq4 = torch.from_numpy(inp4.seqlens).to(dev)
-    k4, v4 = up(inp4.k), up(inp4.v)
-    kv4 = [(k4, v4)] + [(k4.clone(), v4.clone()) for _ in range(2)]
-    q4 = [up(inp4.q) for _ in range(3)]
-    kcs4, valids4 = [], []
-    for k, _ in kv4:
-        kc = torch.zeros(cfg4.B, cfg4.Hkv, NB4, cfg4.gate_dim, dtype=torch.bfloat16, device=dev)
-        valid = torch.zeros(cfg4.B, cfg4.Hkv, dtype=torch.int32, device=dev)
-        S.kcomp_update(shape4, S.KVCache.contiguous(k), seq4, valid, w_k4, kc)
-        kcs4.append(kc)
-        valids4.append(valid)
+    reps4, seq4, w_k4 = _replicas(S, cfg4, inp4, shape4, dev)
+    w_q4 = _up(inp4.w_q, dev)
+    q4 = [_up(inp4.q, dev) for _ in range(3)]
+    args4 = ([r["kv"] for r in reps4], w_q4, w_k4, [r["kc"] for r in reps4], [r["valid"] for r in reps4])
     rows = []
     for sp in SWEEP_SPARSITIES:
         bud = sweep_budget(cfg4.length, sp)
-        st4 = steps_for(shape4, kv4, w_q4, w_k4, kcs4, valids4, bud)
-        rows.append(row(cfg4, inp4, st4, q4, seq4, {"target_sparsity": sp, "token_budget": bud,
-                                                      "k": -(-bud // cfg4.block)}))
+        st4 = make_steps(S, shape4, *args4, bud)
+        rows.append(measure_row(S, cfg4, inp4, st4, q4, seq4, stream, peak,
+                                {"target_sparsity": sp, "token_budget": bud, "k": -(-bud // cfg4.block)}))
         del st4
     res["sweep-64k"] = rows
-    # the all-blocks dense path on the same inputs (same kernel, every block selected)
-    st_d = steps_for(shape4, kv4, w_q4, w_k4, kcs4, valids4, cfg4.length)
-    dense = row(cfg4, inp4, st_d, q4, seq4, {"token_budget": cfg4.length, "k": NB4})
+    st_d = make_steps(S, shape4, *args4, cfg4.length)
+    dense = measure_row(S, cfg4, inp4, st_d, q4, seq4, stream, peak, {"token_budget": cfg4.length, "k": NB4})
     res["dense-64k"] = dense
     for r_ in rows:
         r_["speedup_vs_dense"] = dense["decode_us"] / r_["decode_us"]
-    del st_d, kv4, k4, v4
-    torch.cuda.synchronize()
+        r_["step_speedup_vs_dense"] = dense["step_us"] / r_["step_us"]
+    del st_d, reps4, args4, inp4
+    torch.cuda.empty_cache()
+    # the ragged Qwen3-14B-shaped batch (g = 5, block 128, every list with a forced partial block)
+    cfg3 = config(3)
+    inp3 = make_inputs(cfg3, workers=workers)
+    shape3 = S.Shape(cfg3.B, cfg3.Hq, cfg3.Hkv, cfg3.head_dim, cfg3.gate_dim, cfg3.block, inp3.max_blocks,
+                     cfg3.rope_base)
+    reps3, seq3, w_k3 = _replicas(S, cfg3, inp3, shape3, dev)
+    st3 = make_steps(S, shape3, [r["kv"] for r in reps3], _up(inp3.w_q, dev), w_k3, [r["kc"] for r in reps3],
+                     [r["valid"] for r in reps3], cfg3.budget)
+    res["qwen3-14b-ragged"] = measure_row(S, cfg3, inp3, st3, [_up(inp3.q, dev) for _ in range(3)], seq3, stream,
+                                          peak, {"token_budget": cfg3.budget, "k": cfg3.topk_blocks,
+                                                 "lengths": [int(x) for x in inp3.seqlens]})
+    del st3, reps3, inp3
+    torch.cuda.empty_cache()
+    res["threshold-loop-256"] = threshold_loop_row(S, dev, stream, peak, workers)
     torch.cuda.empty_cache()
     res["prefill-gt-8k"] = prefill_row(S, dev, stream)
     torch.cuda.synchronize()
@@ -475,7 +680,8 @@ def run_seer(args):
 
     cfg = config(WORKLOAD["cid"], **({"budget": args.budget} if args.budget else {}))
     cfg = config(WORKLOAD["cid"], seed=rank_seed(cfg.seed, rank), **({"budget": args.budget} if args.budget else {}))
-    inp = make_inputs(cfg)
+    workers = max(1, min(16, host_cores()))
+    inp = make_inputs(cfg, workers=workers)
     B, Hq, Hkv, d, dg, blk = cfg.B, cfg.Hq, cfg.Hkv, cfg.head_dim, cfg.gate_dim, cfg.block
     NB = inp.max_blocks
 
@@ -503,6 +709,15 @@ def run_seer(args):
 
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
+    if args.only == "step":
+        with torch.cuda.stream(stream):
+            for i in range(args.warmup + args.steps):
+                reps[i % R]["step"].run(reps[i % R]["q"], seqlens, stream=stream)
+        stream.synchronize()
+        if rank == 0:
+            print(json.dumps({"only": "step", "launches": args.warmup + args.steps, "replicas": R,
+                              "single_launch": reps[0]["step"].single_launch}), flush=True)
+        return 0
     if args.only == "decode":
         with torch.cuda.stream(stream):
             for rp in reps:
@@ -602,6 +817,14 @@ def run_seer(args):
 
     decode_us = part(run_decode)
     plan_us = part(run_plan)
+    # the whole step from a graph of consecutive steps (no host work between launches): the default
+    # two-launch form (plan, decode), and the whole step as one launch (seer_decode_step)
+    two_launch_us = ranks_max(time_step_graph([rp["step"] for rp in reps], [rp["q"] for rp in reps], seqlens,
+                                              stream) * 1e-3) * 1e3
+    one = [S.DecodeStep(shape, rp["step"].k, rp["step"].v, w_q, w_k, rp["step"].kcomp, rp["step"].valid_blocks,
+                        mode=S.SELECT_TOPK, token_budget=cfg.budget, num_split=-1, single_launch=True) for rp in reps]
+    one_launch_us = ranks_max(time_step_graph(one, [rp["q"] for rp in reps], seqlens, stream) * 1e-3) * 1e3
+    del one
     gate_us = part(run_gate)
     select_us = part(run_select)
     kcomp_noop_us = part(run_kcomp_noop)
@@ -658,7 +881,12 @@ def run_seer(args):
     idx_h, cnt_h = st0.block_idx.cpu().numpy(), st0.block_cnt.cpu().numpy()
     nbytes = algorithmic_bytes(cfg, inp.seqlens, cnt_h, idx_h, st0.capacity, NB)
     peak, peak_kind = _peaks()
-    achieved = nbytes["decode"] / (decode_us * 1e-6) / 1e9
+    single = reps[0]["step"].single_launch
+    # the dominant kernel: the one-launch step (all of the step's bytes), else the sparse decode
+    dom_us = one_launch_us if single else decode_us
+    dom_bytes = nbytes["step"] if single else nbytes["decode"]
+    achieved = dom_bytes / (dom_us * 1e-6) / 1e9
+    decode_gbs = nbytes["decode"] / (decode_us * 1e-6) / 1e9
     step_gbs = nbytes["step"] / (ms_step * 1e-3) / 1e9
 
     # ---------------- e2e through the public API: pinned H2D of q, D2H of out, every step.
@@ -734,7 +962,7 @@ def run_seer(args):
     # ---------------- the other roofline rows (single GPU)
     sweep = None
     if world == 1 and not args.no_sweep:
-        sweep = sweep_rows(S, dev, stream, peak, shape, reps, seqlens, cfg, inp)
+        sweep = sweep_rows(S, dev, stream, peak, shape, reps, seqlens, cfg, inp, workers)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -744,7 +972,7 @@ def run_seer(args):
                "sample": f"every one of the {B * Hkv} (b, kv-head) pairs of one step (gate, top-k, attention; K "
                          f"Compression Cache prebuilt), {cpu_steps} steps, pairs dealt to {W} host processes"}
 
-    launches_per_step = S.DecodeStep.KERNELS_PER_STEP
+    launches_per_step = reps[0]["step"].kernels_per_step
     line = {
         "metric": METRIC, "value": ms_step * 1e3, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": False, "scaling": "weak",
@@ -755,7 +983,8 @@ def run_seer(args):
                    "sparsity": 1.0 - float(cnt_h.mean()) / NB, "num_split": st0.num_split,
                    "l2": f"inputs rotate over {R} replicas ({R * nbytes['selected_kv'] / 1e6:.0f} MB selected K/V "
                          f"per rotation > 126 MB L2)", "parallelism": f"dp{world} (independent batches)"},
-        "parts_us": {"decode_plan": plan_us, "sparse_decode": decode_us,
+        "parts_us": {"two_launch_step": two_launch_us, "one_launch_step": one_launch_us,
+                     "decode_plan": plan_us, "sparse_decode": decode_us,
                      "unfused": {"kcomp_update_noop": kcomp_noop_us, "kcomp_update_fill": kcomp_fill_us,
                                  "kcomp_append_fold": append_fold_us, "kcomp_append_fill": append_fill_us,
                                  "gate_score": gate_us, "select_blocks": select_us}},
@@ -763,9 +992,14 @@ def run_seer(args):
         "bytes": {"decode_algorithmic": nbytes["decode"], "step_algorithmic": nbytes["step"]},
         "step_gbs": step_gbs,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": _profiled_traffic(), "traffic_unit": "bytes per launch (ncu dram read+write)",
-                     "kernel": "sparse_decode_kernel", "peak_kind": peak_kind,
+                     "traffic": _profiled_traffic() if single else _profiled_traffic(
+                         "sparse_decode_kernel.qwen3-8b-32k-decode.md", ["sparse_decode.cu"]),
+                     "traffic_unit": "bytes per launch (ncu dram read+write)",
+                     "kernel": "decode_step_kernel" if single else "sparse_decode_kernel",
+                     "algorithmic_bytes_per_launch": dom_bytes, "launch_us": dom_us, "peak_kind": peak_kind,
                      "nominal_peak": NOMINAL_HBM_GBS, "frac_of_nominal": achieved / NOMINAL_HBM_GBS},
+        "decode_only": {"kernel": "sparse_decode_kernel", "us": decode_us, "bytes": nbytes["decode"],
+                        "achieved": decode_gbs, "frac": decode_gbs / peak},
         "step_us_p10_p50_p90": step_pct,
         "sweep": sweep,
         "e2e": {"value": e2e_ms * 1e3, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

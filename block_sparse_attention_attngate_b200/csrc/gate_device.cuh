@@ -116,7 +116,7 @@ __device__ void gate_cluster(const GateParams& p, int b, int h, int rank, int L,
   constexpr int RPC = HALF / KC;           // rotation pairs per CTA
   constexpr int ROWS = 2 * RPC;            // projection rows per CTA
   using Tl = GateTiling<DG, KC>;
-  static_assert(NT == 256, "projection: 8 warps");
+  static_assert(NT >= 256 && NT % 32 == 0, "projection: warps 0..7 (any further warps only score)");
   constexpr int LPR = DG / 8;              // lanes per cache row (16-byte chunks)
   constexpr int RPW = 32 / LPR;            // cache rows per warp step
   constexpr int RPS = (NT / 32) * RPW;     // cache rows per CTA step
@@ -145,6 +145,8 @@ __device__ void gate_cluster(const GateParams& p, int b, int h, int rank, int L,
   {
     // projection on the tensor pipe: y[row] = W_q[row] . q for the CTA's ROWS rows, A from the
     // shared rows by ldmatrix; two accumulators halve the mma chain
+    // warps past the first 8 get kq >= kKQ: no k-steps, and their (zero) partials land in slots
+    // the sum below does not read
     const int mt = warp % Tl::kMT, kq = warp / Tl::kMT;
     const int KS = GD / 16, ST = gate_wq_stride<D>(g);
     const int ks0 = kq * KS / Tl::kKQ, ks1 = (kq + 1) * KS / Tl::kKQ;

@@ -45,7 +45,7 @@ template <int D, int BLK, int DG, int NT>
 __device__ void kcomp_group(const KcompParams& p, int b, int h, int g0, int ni, KcompSmem<D, DG, NT>& sm) {
   using SM = KcompSmem<D, DG, NT>;
   constexpr int CH = SM::CH, RG = SM::RG, P3 = 3 * D;
-  static_assert(BLK % RG == 0, "row groups must tile the block");
+  static_assert(NT % CH == 0 && RG <= BLK, "whole row groups, each with a token of the block");
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // ---------------- pooling, one block at a time
   for (int i = 0; i < ni; ++i) {

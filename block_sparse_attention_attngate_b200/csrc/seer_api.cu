@@ -504,11 +504,15 @@ seer_status seer_select_blocks(const seer_dims_t* dims, const float* logits, con
   return SEER_OK;
 }
 
-seer_status seer_decode_plan(const seer_dims_t* dims, const seer_kv_t* k_nope, const int32_t* seqlens,
-                             int32_t* valid_blocks, const void* w_k, void* kcomp, const void* q_nope,
-                             const void* w_q, float* logits_out, float* q_gate_out, int32_t mode,
-                             int32_t token_budget, float tau, int32_t* block_idx, int32_t* block_cnt,
-                             int32_t capacity, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Argument checks and kernel parameters of seer_decode_plan (shared with seer_decode_step).
+seer_status plan_params(const seer_dims_t* dims, const seer_kv_t* k_nope, const int32_t* seqlens,
+                        int32_t* valid_blocks, const void* w_k, void* kcomp, const void* q_nope, const void* w_q,
+                        float* logits_out, float* q_gate_out, int32_t mode, int32_t token_budget, float tau,
+                        int32_t* block_idx, int32_t* block_cnt, int32_t capacity, seer::PlanParams* pp) {
   seer_status st = check_dims(dims);
   if (st != SEER_OK) return st;
   if (!seqlens || !kcomp || !q_nope || !w_q || !block_idx || !block_cnt)
@@ -523,7 +527,7 @@ seer_status seer_decode_plan(const seer_dims_t* dims, const seer_kv_t* k_nope, c
   }
   int32_t kblocks = 0;
   if ((st = select_args(dims, mode, token_budget, tau, capacity, &kblocks)) != SEER_OK) return st;
-  seer::PlanParams p;
+  seer::PlanParams& p = *pp;
   p.update_cache = update;
   rope_thetas(dims, p.k.theta);
   if (update) p.k.k = plain(k_nope);
@@ -564,8 +568,79 @@ seer_status seer_decode_plan(const seer_dims_t* dims, const seer_kv_t* k_nope, c
   p.s.mode = mode;
   p.s.kblocks = kblocks;
   p.s.tau = (double)tau;
+  return SEER_OK;
+}
+
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+extern "C" {
+
+seer_status seer_decode_plan(const seer_dims_t* dims, const seer_kv_t* k_nope, const int32_t* seqlens,
+                             int32_t* valid_blocks, const void* w_k, void* kcomp, const void* q_nope,
+                             const void* w_q, float* logits_out, float* q_gate_out, int32_t mode,
+                             int32_t token_budget, float tau, int32_t* block_idx, int32_t* block_cnt,
+                             int32_t capacity, void* stream) {
+  seer::PlanParams p;
+  const seer_status st = plan_params(dims, k_nope, seqlens, valid_blocks, w_k, kcomp, q_nope, w_q, logits_out,
+                                     q_gate_out, mode, token_budget, tau, block_idx, block_cnt, capacity, &p);
+  if (st != SEER_OK) return st;
   cudaError_t e = seer::launch_plan(p, dims->head_dim, dims->block_size, dims->gate_dim, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode_plan launch");
+  return SEER_OK;
+}
+
+size_t seer_decode_step_workspace_bytes(const seer_dims_t* dims, int32_t capacity) {
+  if (check_dims(dims) != SEER_OK || capacity < 1) return 0;
+  return up256((size_t)dims->batch * dims->num_kv_heads * 4) + seer_sparse_decode_workspace_bytes(dims, capacity, -1);
+}
+
+int32_t seer_decode_step_supported(const seer_dims_t* dims, int32_t mode, int32_t capacity) {
+  if (check_dims(dims) != SEER_OK || capacity < 1) return 0;
+  if ((int64_t)dims->batch * dims->num_kv_heads > seer::kMaxDecodeBH) return 0;
+  if ((int64_t)dims->batch * dims->num_kv_heads * capacity >= (int64_t)1 << 30) return 0;
+  const int bh = dims->batch * dims->num_kv_heads;
+  return seer::step_grid(dims->head_dim, dims->block_size, dims->gate_dim, dims->num_q_heads / dims->num_kv_heads,
+                         dims->max_blocks, mode, dims->batch, bh) > 0;
+}
+
+seer_status seer_decode_step(const seer_dims_t* dims, const seer_kv_t* k_nope, const int32_t* seqlens,
+                             int32_t* valid_blocks, const void* w_k, void* kcomp, const void* q_nope,
+                             const void* w_q, float* logits_out, float* q_gate_out, int32_t mode,
+                             int32_t token_budget, float tau, int32_t* block_idx, int32_t* block_cnt,
+                             int32_t capacity, const void* q, const seer_kv_t* k, const seer_kv_t* v,
+                             void* workspace, size_t workspace_bytes, void* out, float* lse_out,
+                             int32_t* err_word, void* stream) {
+  seer::StepParams sp;
+  seer_status st = plan_params(dims, k_nope, seqlens, valid_blocks, w_k, kcomp, q_nope, w_q, logits_out, q_gate_out,
+                               mode, token_budget, tau, block_idx, block_cnt, capacity, &sp.pl);
+  if (st != SEER_OK) return st;
+  if (!workspace || !aligned16(workspace)) return fail(SEER_ERR_INVALID_ARG, "workspace is NULL or not 16-byte aligned");
+  const size_t flags = up256((size_t)dims->batch * dims->num_kv_heads * 4);
+  const size_t need = seer_decode_step_workspace_bytes(dims, capacity);
+  if (workspace_bytes < need)
+    return fail(SEER_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", workspace_bytes, need);
+  const int bh = dims->batch * dims->num_kv_heads;
+  const int grid = (int64_t)bh * capacity >= (int64_t)1 << 30
+                       ? 0
+                       : seer::step_grid(dims->head_dim, dims->block_size, dims->gate_dim,
+                                         dims->num_q_heads / dims->num_kv_heads, dims->max_blocks, mode, dims->batch, bh);
+  if (grid <= 0)
+    return fail(SEER_ERR_UNSUPPORTED, "no fused step for this shape (shared memory or cluster residency); call "
+                                      "seer_decode_plan and seer_sparse_decode instead");
+  seer::DecodeLaunch L;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  st = seer::prepare_sparse_decode(dims, q, k, v, block_idx, block_cnt, seqlens, capacity, -1, ws + flags,
+                                   workspace_bytes - flags, out, lse_out, err_word, &L);
+  if (st != SEER_OK) return st;
+  if (L.ctas < grid) return fail(SEER_ERR_UNSUPPORTED, "fused step grid %d above the decode's %d", grid, L.ctas);
+  sp.d = L.p;
+  sp.d.ready = reinterpret_cast<int32_t*>(ws);
+  sp.pl.k.err = err_word;
+  cudaError_t e = seer::launch_decode_step(L.tk, L.tv, sp, dims->head_dim, dims->block_size, dims->gate_dim, grid,
+                                           static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "decode_step launch");
   return SEER_OK;
 }
 
@@ -658,6 +733,7 @@ seer_status prepare_sparse_decode(const seer_dims_t* dims, const void* q, const 
   p.out = static_cast<uint16_t*>(out);
   p.lse_out = lse_out;
   p.err = err_word;
+  p.ready = nullptr;
   L->D = dims->head_dim;
   L->BLK = dims->block_size;
   L->ctas = ctas;

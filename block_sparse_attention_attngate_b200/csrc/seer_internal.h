@@ -171,10 +171,22 @@ struct DecodeParams {
   uint16_t* out;            // [B, Hq, D] bf16
   float* lse_out;           // [B, Hq] or null
   int32_t* err;
+  int32_t* ready;           // fused step: [B, Hkv] per-row list-ready flags (zero between calls); else null
 };
 cudaError_t launch_sparse_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                                  int D, int BLK, int grid_flat, cudaStream_t s);
 int decode_ctas_per_sm(int D, int BLK);
+
+// ---------------------------------------------------------------- fused decode step (plan + decode)
+struct StepParams {
+  DecodeParams d;   // capacity schedule (flat == 2), d.ready set
+  PlanParams pl;
+};
+// Grid of the fused step on the current device: 2 x the co-resident clusters of two, at most one
+// CTA per SM; 0 when the shape has no fused kernel or its shared memory does not fit.
+int step_grid(int D, int BLK, int DG, int g, int NB, int mode, int B, int BH);
+cudaError_t launch_decode_step(const CUtensorMap& tk, const CUtensorMap& tv, const StepParams& p, int D, int BLK,
+                               int DG, int grid, cudaStream_t s);
 
 // seer_sparse_decode in two stages: every argument check and the launch set-up (tensor maps,
 // parameters), which enqueues nothing, then the launch itself.

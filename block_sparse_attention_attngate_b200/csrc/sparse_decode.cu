@@ -45,6 +45,9 @@
 // arrive, merged by the consumers themselves.  All waits are bounded.
 #include "seer_device.cuh"
 #include "seer_internal.h"
+#include "step_plan.cuh"
+
+#include <algorithm>
 
 namespace seer {
 namespace {
@@ -256,12 +259,15 @@ __device__ void merge_partials(const DecodeParams& p, int bh, int nseg, int slot
   }
 }
 
-template <int D, int BLK, int NWG, int NG, int STAGES>
-__global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads, 1)
-    sparse_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                         const DecodeParams p) {
+// The decode, run by every thread of a CTA.  DG > 0 is the fused step (decode_step_kernel): the
+// CTA's cluster first plans its rows (step_plan.cuh) and each list position waits for its row's
+// ready flag; DG == 0 is the standalone decode over lists already in memory.
+template <int D, int BLK, int NWG, int NG, int STAGES, int DG>
+__device__ __forceinline__ void decode_body(const CUtensorMap* tmK, const CUtensorMap* tmV, const DecodeParams& p,
+                                            const PlanParams* plan) {
   using S = DecodeShape<D, BLK, NWG, NG, STAGES>;
   constexpr int CW = S::kCW;
+  constexpr bool FUSED = DG > 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
@@ -287,16 +293,36 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
   volatile int* issued = sh + S::kSh;         // [STAGES] tiles issued per stage
   volatile int* observed = issued + STAGES;   // [STAGES] full phases observed per stage
   int* slen = const_cast<int*>(observed + STAGES);   // [B] sequence lengths
-  int* pre = slen + p.B;                              // [BH + 1] list prefix
+  int* pre = slen + p.B;                              // [BH + 1] list prefix (+ 16 ints of scan scratch)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tid = threadIdx.x;
   const int BH = p.B * p.Hkv;
   const int g = p.g;
   auto seq_len = [&](int b) { return p.flat == 2 ? max(__ldg(p.seqlens + b), 0) : slen[b]; };
+  // fused step: the planning cluster's rows are those whose first list position falls in the
+  // cluster's two ranges (capacity schedule: row r starts at position r * capacity)
+  int r_lo = 0, r_hi = 0;
+  uint8_t* plan_raw = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(pre + BH + 1 + 16) + 15) & ~uintptr_t(15));
+  using PS = StepPlanSmem<D, (FUSED ? DG : 64), S::kThreads>;
+  PS& ps = *reinterpret_cast<PS*>(plan_raw);
+  if constexpr (FUSED) {
+    const int W = BH * p.cap, Gd = min((int)gridDim.x, max(W, 1));
+    const int c0 = (int)blockIdx.x & ~1;
+    auto lo = [&](int c) { return c >= Gd ? W : range_lo(c, W, Gd); };
+    r_lo = (lo(c0) + p.cap - 1) / p.cap;
+    r_hi = min(BH, (lo(c0 + 2) + p.cap - 1) / p.cap);
+  }
   if (tid == 0) {
-    tma_prefetch_desc(&tmK);
-    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(tmK);
+    tma_prefetch_desc(tmV);
+    if constexpr (FUSED) {
+      // the first row's W_q rows (weights: no wait needed) land while the previous kernel runs
+      if (r_lo < r_hi)
+        step_plan_prefetch<D, DG, S::kThreads>(*plan, r_lo, (int)blockIdx.x & 1, reinterpret_cast<uint16_t*>(ring),
+                                               ps);
+    }
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], NWG);
@@ -320,9 +346,21 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
                "l"(p.err), "l"(p.out), "r"(p.cap), "r"(p.flat), "r"(p.B), "r"(p.Hkv), "r"(p.k_perm[0]),
                "r"(p.v_perm[2]), "r"(p.per_split), "f"(p.scale_log2));
   const bool fast = p.flat == 2;
-  // (the capacity schedule's producer warp waits for the launch's inputs further down, after a dry
-  // pass over its issue code)
-  if (!(fast && warp == CW)) {
+  if constexpr (FUSED) {
+    // every thread of the cluster plans its rows, then the CTA decodes; lists of rows planned
+    // elsewhere are waited for per row (wait_ready), not per launch.  Both CTAs of the cluster
+    // have started before either writes into the other's shared memory (arrive now, wait after
+    // the launch dependency, so the barrier costs nothing on the critical path).
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+    pdl_wait();
+    pdl_trigger();
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+    cooperative_groups::cluster_group cluster = cooperative_groups::this_cluster();
+    step_plan_rows<D, BLK, DG, S::kThreads>(*plan, p.ready, r_lo, r_hi, reinterpret_cast<uint16_t*>(ring), Ow, ring,
+                                             ps, cluster);
+  } else if (!(fast && warp == CW)) {
+    // (the capacity schedule's producer warp waits for the launch's inputs further down, after a
+    // dry pass over its issue code)
     pdl_wait();
     pdl_trigger();
   }
@@ -471,7 +509,10 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
         merge_partials<D, 32, S::kEpi>(p, jb.bh, jb.nseg, jb.slot_first, jb.cf, lane, epi,
                                        [] { __syncwarp(); });
         __syncwarp();
-        if (lane == 0) p.counters[jb.bh] = 0;
+        if (lane == 0) {
+          p.counters[jb.bh] = 0;
+          if constexpr (FUSED) p.ready[jb.bh] = 0;   // every piece of the row is done with its list
+        }
       }
     }
     return;
@@ -483,6 +524,8 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
     const int fixed_bh = pbh;
     // resolve list position `it` of this CTA (one lane per position)
     bool dry = false;
+    int ready_bh = -1;      // fused step: the row whose ready flag this lane last acquired
+    bool ready_ok = false;
     auto resolve = [&](int it, int& n, int& bh, int& first, int& kb, int& kt, int& vb, int& vt) {
       n = -1;
       bh = fixed_bh;
@@ -503,10 +546,19 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
       }
       first = (it == 0 || pos == 0) ? kSegFirst : 0;
       const int b = bh / p.Hkv;
+      if constexpr (FUSED) {
+        // the row's list is written in this launch: acquire its flag, then read through L2
+        if (bh != ready_bh) {
+          ready_ok = wait_ready(p.ready + bh, sh);
+          if (!ready_ok) report(p.err, SEER_DEVERR_TIMEOUT);
+          ready_bh = bh;
+        }
+        if (!ready_ok) return;
+      }
       // the count (capacity schedule), the length and the block index, requested together
-      const int c = p.flat == 2 ? p.cnt[bh] : p.cap;
+      const int c = p.flat == 2 ? (FUSED ? __ldcg(p.cnt + bh) : p.cnt[bh]) : p.cap;
       const int Lb = seq_len(b);
-      const int blk = p.idx[(size_t)bh * p.cap + pos];
+      const int blk = FUSED ? __ldcg(p.idx + (size_t)bh * p.cap + pos) : p.idx[(size_t)bh * p.cap + pos];
       if (p.flat == 2) {   // list positions past the count are padding
         if (pos == 0 && c > p.cap && !dry) report(p.err, SEER_DEVERR_COUNT);
         if (pos >= c) return;
@@ -543,9 +595,9 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
     // read but the values are dropped, and no copy, barrier arrival or report is made).  Run for the
     // first time after the wait, this code delayed the first tile request by ~0.7 us more.
 #pragma unroll 1
-    for (int pass = fast ? 0 : 1; pass < 2; ++pass) {
+    for (int pass = (fast && !FUSED) ? 0 : 1; pass < 2; ++pass) {
       dry = pass == 0;
-      if (fast && !dry) {
+      if (fast && !dry && !FUSED) {
         pdl_wait();
         pdl_trigger();
       }
@@ -595,11 +647,11 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
                 tile_coords(p.k_perm, kt, h, kb, c1, c2, c3);
   #pragma unroll
                 for (int bx = 0; bx < S::kNBox; ++bx)
-                  tma_load_4d_hint(kdst + bx * S::kBox, &tmK, &full[s], bx * 64, c1, c2, c3, stream_pol);
+                  tma_load_4d_hint(kdst + bx * S::kBox, tmK, &full[s], bx * 64, c1, c2, c3, stream_pol);
                 tile_coords(p.v_perm, vt, h, vb, c1, c2, c3);
   #pragma unroll
                 for (int bx = 0; bx < S::kNBox; ++bx)
-                  tma_load_4d_hint(vdst + bx * S::kBox, &tmV, &full[s], bx * 64, c1, c2, c3, stream_pol);
+                  tma_load_4d_hint(vdst + bx * S::kBox, tmV, &full[s], bx * 64, c1, c2, c3, stream_pol);
               } else {
                 mbar_arrive(&full[s]);
               }
@@ -865,6 +917,9 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
         }
       }
     }
+    if constexpr (FUSED) {
+      if (nseg <= 1 && tid == 0) p.ready[bh] = 0;   // the row's only piece is done with its list
+    }
     if (nseg > 1 && !last_seg) {
       // the CTA's split first segment: the epilogue warp publishes / merges it
       if (tid == 0) job[0] = Job{bh, nseg, slot_first, cf};
@@ -891,7 +946,10 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
           alive = false;
           break;
         }
-        if (tid == 0) p.counters[bh] = 0;
+        if (tid == 0) {
+          p.counters[bh] = 0;
+          if constexpr (FUSED) p.ready[bh] = 0;   // every piece of the row is done with its list
+        }
       }
     }
     it0 = it1;
@@ -930,6 +988,24 @@ __global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads
       if (e < g && p.lse_out) p.lse_out[qh0 + e] = -INFINITY;
     }
   }
+}
+
+template <int D, int BLK, int NWG, int NG, int STAGES>
+__global__ void __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads, 1)
+    sparse_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                         const __grid_constant__ DecodeParams p) {
+  decode_body<D, BLK, NWG, NG, STAGES, 0>(&tmK, &tmV, p, nullptr);
+}
+
+// The fused decode step: plan (cache update, gate, selection) and decode in one launch, one CTA
+// per SM in clusters of two (the pair that plans a row shares its gate through distributed
+// shared memory).  Capacity schedule only.  Every CTA must be resident at once: the host sizes
+// the grid by the co-resident cluster count, and every wait is bounded.
+template <int D, int BLK, int DG, int NWG, int NG, int STAGES>
+__global__ void __cluster_dims__(kStepCluster, 1, 1) __launch_bounds__(DecodeShape<D, BLK, NWG, NG, STAGES>::kThreads, 1)
+    decode_step_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                       const __grid_constant__ StepParams sp) {
+  decode_body<D, BLK, NWG, NG, STAGES, DG>(&tmK, &tmV, sp.d, &sp.pl);
 }
 
 // ring depth and consumer groups per shape (stage = 2 * BLK * D * 2 bytes; one CTA per SM)
@@ -978,7 +1054,96 @@ int ctas_per_sm_t() {
   return n > 0 ? n : 1;
 }
 
+template <int D, int BLK, int DG>
+auto step_kernel() {
+  using C = Choice<D, BLK>;
+  return decode_step_kernel<D, BLK, DG, C::NWG, C::NG, C::ST>;
+}
+
+template <int D, int BLK, int DG>
+size_t step_smem_bytes(int B, int BH) {
+  return smem_bytes<D, BLK>(B, BH) + 16 + sizeof(StepPlanSmem<D, DG, ShapeOf<D, BLK>::kThreads>);
+}
+
+constexpr size_t kMaxDynSmem = 227 * 1024;
+
+// Whether the planning phase's shared regions fit the decode's: the W_q rows in the ring and the
+// q / merge areas before the barriers, the logit row in the merge area, the shared-memory
+// selection's keys in the ring.
+template <int D, int BLK, int DG>
+bool step_fits(int g, int NB, int mode, int B, int BH) {
+  using Sh = ShapeOf<D, BLK>;
+  if (step_smem_bytes<D, BLK, DG>(B, BH) > kMaxDynSmem) return false;
+  if (gate_wq_bytes<D, DG, kStepCluster>(g) > (size_t)Sh::kRing + 2 * Sh::kQBytes + (size_t)Sh::kMergeFloats * 4)
+    return false;
+  if ((size_t)NB * 4 > (size_t)Sh::kMergeFloats * 4) return false;
+  const bool regs = mode != 2 && NB <= 8 * Sh::kThreads;
+  if (!regs && select_smem_bytes(NB, mode) > (size_t)Sh::kRing) return false;
+  return true;
+}
+
+template <int D, int BLK, int DG>
+int step_grid_t(int g, int NB, int mode, int B, int BH) {
+  if (!step_fits<D, BLK, DG>(g, NB, mode, B, BH)) return 0;
+  auto kern = step_kernel<D, BLK, DG>();
+  static std::atomic<uint64_t> attr_done{0};
+  if (ensure_smem_limit(kern, (int)kMaxDynSmem, attr_done) != cudaSuccess) return 0;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kStepCluster * (sms / kStepCluster), 1, 1);
+  cfg.blockDim = dim3(ShapeOf<D, BLK>::kThreads);
+  cfg.dynamicSmemBytes = step_smem_bytes<D, BLK, DG>(B, BH);
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess) return 0;
+  clusters = std::min(clusters, sms / kStepCluster);
+  return clusters > 0 ? kStepCluster * clusters : 0;
+}
+
+template <int D, int BLK, int DG>
+cudaError_t launch_step_t(const CUtensorMap& tk, const CUtensorMap& tv, const StepParams& p, int grid,
+                          cudaStream_t st) {
+  auto kern = step_kernel<D, BLK, DG>();
+  static std::atomic<uint64_t> attr_done{0};
+  cudaError_t e = ensure_smem_limit(kern, (int)kMaxDynSmem, attr_done);
+  if (e != cudaSuccess) return e;
+  const size_t smem = step_smem_bytes<D, BLK, DG>(p.d.B, p.d.B * p.d.Hkv);
+  return launch_pdl(kern, dim3(grid), dim3(ShapeOf<D, BLK>::kThreads), smem, st, tk, tv, p);
+}
+
 }  // namespace
+
+int step_grid(int D, int BLK, int DG, int g, int NB, int mode, int B, int BH) {
+#define SEER_S(d, blk, dg) \
+  if (D == d && BLK == blk && DG == dg) return step_grid_t<d, blk, dg>(g, NB, mode, B, BH);
+  SEER_S(64, 64, 64)
+  SEER_S(64, 64, 128)
+  SEER_S(64, 128, 64)
+  SEER_S(64, 128, 128)
+  SEER_S(128, 64, 64)
+  SEER_S(128, 64, 128)
+  SEER_S(128, 128, 64)
+  SEER_S(128, 128, 128)
+#undef SEER_S
+  return 0;
+}
+
+cudaError_t launch_decode_step(const CUtensorMap& tk, const CUtensorMap& tv, const StepParams& p, int D, int BLK,
+                               int DG, int grid, cudaStream_t s) {
+#define SEER_S(d, blk, dg) \
+  if (D == d && BLK == blk && DG == dg) return launch_step_t<d, blk, dg>(tk, tv, p, grid, s);
+  SEER_S(64, 64, 64)
+  SEER_S(64, 64, 128)
+  SEER_S(64, 128, 64)
+  SEER_S(64, 128, 128)
+  SEER_S(128, 64, 64)
+  SEER_S(128, 64, 128)
+  SEER_S(128, 128, 64)
+  SEER_S(128, 128, 128)
+#undef SEER_S
+  return cudaErrorInvalidValue;
+}
 
 int decode_ctas_per_sm(int D, int BLK) {
   if (D == 64 && BLK == 64) return ctas_per_sm_t<64, 64>();

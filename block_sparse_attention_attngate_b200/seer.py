@@ -27,7 +27,9 @@ SELECT_TOPK, SELECT_THRESHOLD, SELECT_TOPP = 0, 1, 2
 DEVERR_BLOCK_INDEX, DEVERR_PAGE_INDEX, DEVERR_COUNT, DEVERR_TIMEOUT = 1, 2, 4, 8
 
 EXPORTED = (
-    "seer_kcomp_update", "seer_kcomp_state_bytes", "seer_kcomp_append", "seer_kcomp_state_init", "seer_gate_score", "seer_select_blocks", "seer_decode_plan", "seer_sparse_decode_auto_split",
+    "seer_kcomp_update", "seer_kcomp_state_bytes", "seer_kcomp_append", "seer_kcomp_state_init", "seer_gate_score",
+    "seer_select_blocks", "seer_decode_plan", "seer_decode_step_workspace_bytes", "seer_decode_step_supported",
+    "seer_decode_step", "seer_sparse_decode_auto_split",
     "seer_sparse_decode_workspace_bytes", "seer_sparse_decode", "seer_sparse_decode_noalloc",
     "seer_gate_truth_workspace_bytes", "seer_gate_truth", "seer_prefill_gt_workspace_bytes", "seer_prefill_gt",
     "seer_last_error", "seer_version",
@@ -67,6 +69,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "seer_gate_score": (I32, [DP, P, P, P, P, P, P, P]),
         "seer_select_blocks": (I32, [DP, P, P, I32, I32, F32, P, P, I32, P]),
         "seer_decode_plan": (I32, [DP, KP, P, P, P, P, P, P, P, P, I32, I32, F32, P, P, I32, P]),
+        "seer_decode_step_workspace_bytes": (SZ, [DP, I32]),
+        "seer_decode_step_supported": (I32, [DP, I32, I32]),
+        "seer_decode_step": (I32, [DP, KP, P, P, P, P, P, P, P, P, I32, I32, F32, P, P, I32, P, KP, KP, P, SZ, P, P, P,
+                                   P]),
         "seer_sparse_decode_auto_split": (I32, [DP, I32]),
         "seer_sparse_decode_workspace_bytes": (SZ, [DP, I32, I32]),
         "seer_sparse_decode": (I32, [DP, P, KP, KP, P, P, P, I32, I32, P, SZ, P, P, P, P]),
@@ -360,6 +366,66 @@ def decode_plan(shape: Shape, seqlens: torch.Tensor, kcomp: torch.Tensor, q_nope
                                  float(tau), _ptr(block_idx), _ptr(block_cnt), block_idx.shape[-1], _stream(stream)))
 
 
+def decode_step_workspace_bytes(shape: Shape, capacity: int) -> int:
+    dims = shape.c()
+    return int(_lib.seer_decode_step_workspace_bytes(ctypes.byref(dims), int(capacity)))
+
+
+def decode_step_supported(shape: Shape, mode: int, capacity: int) -> bool:
+    """Whether decode_step runs this shape and selection mode in one launch on the current device."""
+    dims = shape.c()
+    return bool(_lib.seer_decode_step_supported(ctypes.byref(dims), int(mode), int(capacity)))
+
+
+def alloc_step_workspace(shape: Shape, capacity: int, device=None) -> torch.Tensor:
+    """Zero-filled workspace for decode_step (its ready flags and arrival counters start at zero)."""
+    return torch.zeros(max(decode_step_workspace_bytes(shape, capacity), 16), dtype=torch.uint8,
+                       device=device or "cuda")
+
+
+def decode_step(shape: Shape, seqlens: torch.Tensor, kcomp: torch.Tensor, q_nope: torch.Tensor, w_q: torch.Tensor,
+                mode: int, block_idx: torch.Tensor, block_cnt: torch.Tensor, q: torch.Tensor, k: KVCache, v: KVCache,
+                out: torch.Tensor, workspace: torch.Tensor, token_budget: int = 0, tau: float = 0.0,
+                k_nope: Optional[KVCache] = None, valid_blocks: Optional[torch.Tensor] = None,
+                w_k: Optional[torch.Tensor] = None, logits: Optional[torch.Tensor] = None,
+                q_gate: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                err: Optional[torch.Tensor] = None, stream=None):
+    """decode_plan followed by sparse_decode (capacity schedule) in one launch (see seer_decode_step)."""
+    B, Hq, H, d, dg = shape.batch, shape.num_q_heads, shape.num_kv_heads, shape.head_dim, shape.gate_dim
+    _need_shape(seqlens, (B,), "seqlens")
+    _need_shape(kcomp, (B, H, shape.max_blocks, dg), "kcomp")
+    _need_shape(q_nope, (B, Hq, d), "q_nope")
+    _need_shape(w_q, (H, dg, shape.group * d), "w_q")
+    _decode_shapes(shape, q, k, v, block_idx, block_cnt, seqlens, out, lse, err)
+    if valid_blocks is not None:
+        _need_shape(valid_blocks, (B, H), "valid_blocks")
+        _need_shape(w_k, (H, dg, 3 * d), "w_k")
+        if k_nope is None:
+            raise ValueError("k_nope is required with valid_blocks")
+        k_nope.check(shape, "k_nope")
+    if logits is not None:
+        _need_shape(logits, (B, H, shape.max_blocks), "logits")
+    if q_gate is not None:
+        _need_shape(q_gate, (B, H, dg), "q_gate")
+    for t, dt, name in ((seqlens, torch.int32, "seqlens"), (kcomp, torch.bfloat16, "kcomp"),
+                        (q_nope, torch.bfloat16, "q_nope"), (w_q, torch.bfloat16, "w_q"),
+                        (block_idx, torch.int32, "block_idx"), (block_cnt, torch.int32, "block_cnt"),
+                        (q, torch.bfloat16, "q"), (out, torch.bfloat16, "out"), (workspace, torch.uint8, "workspace")):
+        _need(t, dt, name)
+    for t, dt, name in ((valid_blocks, torch.int32, "valid_blocks"), (w_k, torch.bfloat16, "w_k"),
+                        (logits, torch.float32, "logits"), (q_gate, torch.float32, "q_gate"),
+                        (lse, torch.float32, "lse"), (err, torch.int32, "err")):
+        if t is not None:
+            _need(t, dt, name)
+    dims = shape.c()
+    kv = ctypes.byref(k_nope.desc) if k_nope is not None else None
+    _check(_lib.seer_decode_step(ctypes.byref(dims), kv, _ptr(seqlens), _ptr(valid_blocks), _ptr(w_k), _ptr(kcomp),
+                                 _ptr(q_nope), _ptr(w_q), _ptr(logits), _ptr(q_gate), int(mode), int(token_budget),
+                                 float(tau), _ptr(block_idx), _ptr(block_cnt), block_idx.shape[-1], _ptr(q),
+                                 ctypes.byref(k.desc), ctypes.byref(v.desc), _ptr(workspace), workspace.numel(),
+                                 _ptr(out), _ptr(lse), _ptr(err), _stream(stream)))
+
+
 def sparse_decode_auto_split(shape: Shape, capacity: int) -> int:
     dims = shape.c()
     return int(_lib.seer_sparse_decode_auto_split(ctypes.byref(dims), int(capacity)))
@@ -519,7 +585,7 @@ class DecodeStep:
                  kcomp: torch.Tensor, valid_blocks: torch.Tensor, mode: int = SELECT_TOPK, token_budget: int = 0,
                  tau: float = 0.0, capacity: Optional[int] = None, num_split: Optional[int] = None,
                  k_nope: Optional[KVCache] = None, kcomp_state: Optional[torch.Tensor] = None,
-                 device=None):
+                 single_launch: Optional[bool] = None, device=None):
         dev = device or w_q.device
         self.shape, self.k, self.v, self.w_q, self.w_k = shape, k, v, w_q, w_k
         self.k_nope = k_nope or k
@@ -542,17 +608,42 @@ class DecodeStep:
             num_split = -1 if mode == SELECT_TOPK else 0
         self.num_split = num_split    # -1 capacity, 0 balanced, >= 1 the pages' grid
         self.workspace = alloc_workspace(shape, capacity, self.num_split, dev)
+        # single_launch=True runs the whole step as one launch (decode_step, capacity schedule); the
+        # default is the plan and the decode as two launches, which measured faster (the plan kernel's
+        # CTAs start while the previous decode drains; a launch that plans in its own CTAs cannot)
+        if single_launch is None:
+            single_launch = False
+        if single_launch and (self.num_split != -1 or not decode_step_supported(shape, mode, capacity)):
+            raise ValueError("single_launch needs num_split=-1 and a shape decode_step_supported accepts")
+        self.single_launch = bool(single_launch)
+        self.step_workspace = alloc_step_workspace(shape, capacity, dev) if self.single_launch else None
+        self.kernels_per_step = (1 if self.single_launch else 2) + (1 if kcomp_state is not None else 0)
         self.out = torch.empty(B, Hq, shape.head_dim, dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
 
     def run(self, q: torch.Tensor, seqlens: torch.Tensor, q_nope: Optional[torch.Tensor] = None, stream=None,
             fused: bool = True, k_new: Optional[torch.Tensor] = None):
-        """One decode step.  fused=True plans with seer_decode_plan (one launch); fused=False makes
-        the three separate calls (kcomp_update, gate_score, select_blocks) instead.  With running
+        """One decode step.  fused=True runs the whole step as one launch (seer_decode_step) when the
+        step was built for it (single_launch), else plans with seer_decode_plan (one launch) and then
+        decodes; fused=False makes the three separate planning calls (kcomp_update, gate_score,
+        select_blocks) and then decodes.  With running
         block statistics (kcomp_state), `k_new` holds the appended tokens' pre-RoPE keys."""
         s = self.shape
         qn = q if q_nope is None else q_nope
+        if self.single_launch and fused:
+            upd = self.kcomp_state is None
+            if not upd:
+                if k_new is None:
+                    raise ValueError("a step with running block statistics needs k_new, the appended pre-RoPE keys")
+                kcomp_append(s, k_new, seqlens, self.kcomp_state, self.valid_blocks, self.w_k, self.kcomp, self.err,
+                             stream)
+            decode_step(s, seqlens, self.kcomp, qn, self.w_q, self.mode, self.block_idx, self.block_cnt, q, self.k,
+                        self.v, self.out, self.step_workspace, self.token_budget, self.tau,
+                        k_nope=self.k_nope if upd else None, valid_blocks=self.valid_blocks if upd else None,
+                        w_k=self.w_k if upd else None, logits=self.logits, lse=self.lse, err=self.err,
+                        stream=stream)
+            return self.out
         if self.kcomp_state is not None:
             if k_new is None:
                 raise ValueError("a step with running block statistics needs k_new, the appended pre-RoPE keys")
@@ -573,4 +664,3 @@ class DecodeStep:
                       self.num_split, self.lse, self.err, stream)
         return self.out
 
-    KERNELS_PER_STEP = 2   # plan, decode

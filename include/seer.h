@@ -15,6 +15,8 @@
  *     seer_kcomp_update -> seer_gate_score -> seer_select_blocks -> seer_sparse_decode
  * or, with the first three fused into one launch,
  *     seer_decode_plan -> seer_sparse_decode
+ * or, the whole step in one launch,
+ *     seer_decode_step
  *
  * Conventions shared by every call
  *   - The caller owns all memory.  The library never allocates or frees.
@@ -289,6 +291,40 @@ seer_status seer_sparse_decode(const seer_dims_t* dims, const void* q, const see
                                int32_t capacity, int32_t num_split, void* workspace,
                                size_t workspace_bytes, void* out, float* lse_out,
                                int32_t* err_word, void* stream);
+
+/*
+ * seer_decode_step -- the whole decode step in one launch: seer_decode_plan followed by
+ * seer_sparse_decode with the capacity schedule (num_split == -1) [CP Knowl 1-2, Knowl 5,
+ * Knowl 6, as those calls].
+ *
+ * Arguments are those of seer_decode_plan (k_nope .. capacity) followed by those of
+ * seer_sparse_decode (q, k, v, workspace .. err_word); results are the same: the cache rows and
+ * fill counts, the optional logits / Q_gate, the block lists and counts, out and lse_out.
+ *   workspace  device, >= seer_decode_step_workspace_bytes(dims, capacity) bytes, 16-byte
+ *              aligned; its first B*Hkv int32 are per-row ready flags and the next section holds
+ *              the decode's arrival counters: both must be zero before the first call (allocate
+ *              zero-filled), and every completed call leaves them zero.  After a call that set
+ *              SEER_DEVERR_TIMEOUT, zero the workspace again before the next call.
+ * One CTA per SM in clusters of two: each cluster first plans the rows whose lists start in its
+ * two ranges (cache update, gate, selection, as seer_decode_plan), publishes each list with a
+ * per-row flag, then every CTA streams its range, waiting only for the rows it reads.  Requires
+ * every CTA of the grid to be resident at once (the grid is sized from the co-resident cluster
+ * count; each wait is bounded and reports SEER_DEVERR_TIMEOUT).
+ * Returns SEER_ERR_UNSUPPORTED when the shape has no fused kernel (see
+ * seer_decode_step_supported); use seer_decode_plan + seer_sparse_decode then.
+ * seer_decode_step_supported returns 1 when the current device runs this shape and selection
+ * mode fused (no device work), else 0.
+ * Calls on the same workspace must not overlap on the GPU.
+ */
+size_t seer_decode_step_workspace_bytes(const seer_dims_t* dims, int32_t capacity);
+int32_t seer_decode_step_supported(const seer_dims_t* dims, int32_t mode, int32_t capacity);
+seer_status seer_decode_step(const seer_dims_t* dims, const seer_kv_t* k_nope, const int32_t* seqlens,
+                             int32_t* valid_blocks, const void* w_k, void* kcomp, const void* q_nope,
+                             const void* w_q, float* logits_out, float* q_gate_out, int32_t mode,
+                             int32_t token_budget, float tau, int32_t* block_idx, int32_t* block_cnt,
+                             int32_t capacity, const void* q, const seer_kv_t* k, const seer_kv_t* v,
+                             void* workspace, size_t workspace_bytes, void* out, float* lse_out,
+                             int32_t* err_word, void* stream);
 
 /*
  * seer_sparse_decode_noalloc -- seer_sparse_decode for callers that cannot allocate.

@@ -34,9 +34,10 @@ def _rng(seed: int, *key: int) -> np.random.Generator:
 
 
 def bf16_bits_from_f32(x: np.ndarray) -> np.ndarray:
-    """Round float32 values to bf16 (nearest, ties to even); return uint16 bits."""
-    b = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
-    b = (b + 0x7FFF + ((b >> 16) & 1)) >> 16
+    """Round float32 values to bf16 (nearest, ties to even); return uint16 bits.  The sum is taken
+    modulo 2^32: only its bits 16..31 are kept, which a wider sum would give the same."""
+    b = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    b = (b + np.uint32(0x7FFF) + ((b >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)
     return b.astype(np.uint16)
 
 
@@ -199,12 +200,75 @@ def make_pair_inputs(cfg: DecodeConfig, b: int, h: int) -> PairInputs:
     return PairInputs(length=int(seqlens[b]), q=q[b, h * g:(h + 1) * g], k=k, v=v, w_q=w_q, w_k=w_k)
 
 
+def _kv_fill(cfg, path_k, path_v, shape, pairs, seqlens, final, q32, tail, results):
+    """Worker of make_inputs(workers > 1): draw a share of the (b, kv-head) slices straight into the
+    file-backed K and V arrays; puts the share's planted blocks on `results`."""
+    k = np.memmap(path_k, dtype=np.uint16, mode="r+", shape=shape)
+    v = np.memmap(path_v, dtype=np.uint16, mode="r+", shape=shape)
+    hot = {}
+    for (b, h) in pairs:
+        k[b, h], v[b, h], chosen = _kv_slice(cfg, b, h, int(seqlens[b]), int(final[b]), shape[2], q32, tail)
+        if chosen is not None:
+            hot[(b, h)] = chosen
+    k.flush()
+    v.flush()
+    del k, v
+    results.put(hot)
+
+
+def _kv_parallel(cfg, seqlens, final, lcap, q32, tail, workers):
+    """The K and V slices drawn by `workers` spawned processes (each slice has its own stream, so the
+    bytes are those of the serial loop).  A worker that dies raises here instead of being waited
+    for."""
+    import multiprocessing as mp
+    import os
+    import queue
+    import shutil
+    import tempfile
+    shape = (cfg.B, cfg.Hkv, lcap, cfg.head_dim)
+    pairs = [(b, h) for b in range(cfg.B) for h in range(cfg.Hkv)]
+    tmp = tempfile.mkdtemp(prefix="seer_inputs_")
+    ctx = mp.get_context("spawn")
+    procs = []
+    try:
+        pk, pv = os.path.join(tmp, "k.u16"), os.path.join(tmp, "v.u16")
+        for path in (pk, pv):
+            np.memmap(path, dtype=np.uint16, mode="w+", shape=shape).flush()
+        W = max(1, min(workers, len(pairs)))
+        results = ctx.Queue()
+        procs = [ctx.Process(target=_kv_fill, args=(cfg, pk, pv, shape, pairs[i::W], seqlens, final, q32, tail,
+                                                    results), daemon=True) for i in range(W)]
+        for p in procs:
+            p.start()
+        parts = []
+        while len(parts) < W:
+            try:
+                parts.append(results.get(timeout=5))
+            except queue.Empty:
+                if any(p.exitcode not in (None, 0) for p in procs):
+                    raise RuntimeError("a worker drawing the synthetic K / V slices failed")
+        for p in procs:
+            p.join()
+        k = np.array(np.memmap(pk, dtype=np.uint16, mode="r", shape=shape))
+        v = np.array(np.memmap(pv, dtype=np.uint16, mode="r", shape=shape))
+    finally:
+        for p in procs:
+            if p.is_alive():
+                p.kill()
+        shutil.rmtree(tmp, ignore_errors=True)
+    hot: Dict[Tuple[int, int], List[int]] = {}
+    for part in parts:
+        hot.update(part)
+    return k, v, dict(sorted(hot.items()))
+
+
 def make_inputs(cfg: DecodeConfig, *, tail: str = "random",
-                lengths: Optional[Sequence[int]] = None) -> DecodeInputs:
+                lengths: Optional[Sequence[int]] = None, workers: int = 1) -> DecodeInputs:
     """Draw one decode problem.
 
     tail="nan" fills cache rows past each sequence's final length with bf16
-    NaN, so any read of a masked token poisons the result.
+    NaN, so any read of a masked token poisons the result.  workers > 1 draws
+    the K / V slices in that many spawned processes (same bytes).
     """
     B, Hq, Hkv, d, dg, blk = cfg.B, cfg.Hq, cfg.Hkv, cfg.head_dim, cfg.gate_dim, cfg.block
     g = cfg.g
@@ -223,14 +287,17 @@ def make_inputs(cfg: DecodeConfig, *, tail: str = "random",
         w_k[h] = bf16_bits_from_f32(_rng(cfg.seed, _T_WK, h).standard_normal((dg, 3 * d), dtype=np.float32)
                                     / np.float32(math.sqrt(3 * d)))
 
-    k = np.empty((B, Hkv, lcap, d), dtype=np.uint16)
-    v = np.empty((B, Hkv, lcap, d), dtype=np.uint16)
-    hot: Dict[Tuple[int, int], List[int]] = {}
-    for b in range(B):
-        for h in range(Hkv):
-            k[b, h], v[b, h], chosen = _kv_slice(cfg, b, h, int(seqlens[b]), int(final[b]), lcap, q32, tail)
-            if chosen is not None:
-                hot[(b, h)] = chosen
+    if workers > 1 and B * Hkv > 1:
+        k, v, hot = _kv_parallel(cfg, seqlens, final, lcap, q32, tail, workers)
+    else:
+        k = np.empty((B, Hkv, lcap, d), dtype=np.uint16)
+        v = np.empty((B, Hkv, lcap, d), dtype=np.uint16)
+        hot = {}
+        for b in range(B):
+            for h in range(Hkv):
+                k[b, h], v[b, h], chosen = _kv_slice(cfg, b, h, int(seqlens[b]), int(final[b]), lcap, q32, tail)
+                if chosen is not None:
+                    hot[(b, h)] = chosen
     return DecodeInputs(cfg=cfg, seqlens=seqlens, final_lens=final.astype(np.int32), q=q, k=k, v=v,
                         w_q=w_q, w_k=w_k, hot=hot)
 

@@ -44,6 +44,12 @@ LSE_ABS = 2e-3
 THRESH_REL = 1e-6
 
 
+def draw_workers() -> int:
+    """Processes for drawing the large synthetic workloads (same bytes as one process)."""
+    import os
+    return max(1, min(16, os.cpu_count() or 1))
+
+
 def to_dev_bf16(bits: np.ndarray, device="cuda") -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(device).view(torch.bfloat16)
 

@@ -36,13 +36,19 @@ def test_profiled_traffic_follows_the_source(tmp_path):
     src = tmp_path / "block_sparse_attention_attngate_b200" / "csrc"
     src.mkdir(parents=True)
     (src / "k.cu").write_bytes(b"kernel source v1\n")
+    (src / "k.cuh").write_bytes(b"header v1\n")
     sha = hashlib.sha256(b"kernel source v1\n").hexdigest()
+    sha2 = hashlib.sha256(b"kernel source v1\nheader v1\n").hexdigest()
     (tmp_path / "profiles" / "k.md").write_text(f"# k\n\ntraffic_bytes_per_launch: 12345\nsource_sha256: {sha}\n")
+    (tmp_path / "profiles" / "k2.md").write_text(f"# k\n\ntraffic_bytes_per_launch: 777\nsource_sha256: {sha2}\n")
     bench.ROOT = str(tmp_path)
-    assert bench._profiled_traffic("k.md", "k.cu") == 12345
-    (src / "k.cu").write_bytes(b"kernel source v2\n")             # the kernel changed since the capture
-    assert bench._profiled_traffic("k.md", "k.cu") is None
-    assert bench._profiled_traffic("missing.md", "k.cu") is None
+    assert bench._profiled_traffic("k.md", ["k.cu"]) == 12345
+    assert bench._profiled_traffic("k2.md", ["k.cu", "k.cuh"]) == 777     # every source of the kernel, in order
+    (src / "k.cuh").write_bytes(b"header v2\n")                        # a header of the kernel changed
+    assert bench._profiled_traffic("k2.md", ["k.cu", "k.cuh"]) is None
+    (src / "k.cu").write_bytes(b"kernel source v2\n")                  # the kernel changed since the capture
+    assert bench._profiled_traffic("k.md", ["k.cu"]) is None
+    assert bench._profiled_traffic("missing.md", ["k.cu"]) is None
 
 
 def test_committed_profiles_carry_traffic_and_hash():

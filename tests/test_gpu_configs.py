@@ -20,7 +20,8 @@ import torch
 
 from oracle import seer_oracle as O
 from seer_harness import (LOGIT_RTOL, OracleBH, bf16_bits, check_attention, check_kcomp_rows, check_logits,
-                          check_logits_e2e, check_lse, check_selection, e2e_logit_bound, f64, gpu_list, to_dev_bf16)
+                          check_logits_e2e, check_lse, check_selection, draw_workers, e2e_logit_bound, f64, gpu_list,
+                          to_dev_bf16)
 from synthetic import (SWEEP_SPARSITIES, bf16_bits_from_f32, config, make_inputs, make_step_query,
                        scale_gate_weights)
 from synthetic.inputs import sweep_budget
@@ -46,9 +47,9 @@ class Problem:
         self.valid = torch.zeros(c.B, c.Hkv, dtype=torch.int32, device="cuda")
         self.obh = {(b, h): OracleBH(inp, b, h) for b in range(c.B) for h in range(c.Hkv)}
 
-    def step(self, mode, budget=0, tau=0.0):
+    def step(self, mode, budget=0, tau=0.0, **kw):
         return S.DecodeStep(self.sh, S.KVCache.contiguous(self.k), S.KVCache.contiguous(self.v), self.w_q, self.w_k,
-                            self.kc, self.valid, mode=mode, token_budget=budget, tau=tau)
+                            self.kc, self.valid, mode=mode, token_budget=budget, tau=tau, **kw)
 
 
 def _boundary_ok(z, gpu, ref, mode, bound, k_blocks=0, tau=0.0):
@@ -207,17 +208,20 @@ def _prefill(P, lengths):
     torch.cuda.synchronize()
 
 
-@pytest.mark.parametrize("cid", [1, 2, 3])
-def test_topk_workload(cid):
+@pytest.mark.parametrize("cid,single", [(1, False), (2, False), (3, False), (1, True), (2, True), (3, True)])
+def test_topk_workload(cid, single):
+    """single: the whole step as one launch (seer_decode_step); else the plan and the decode as two
+    launches (the default)."""
     cfg = config(cid)
-    inp = make_inputs(cfg, tail="nan")
+    inp = make_inputs(cfg, tail="nan", workers=draw_workers())
     P = Problem(inp)
     L = inp.seqlens
     _prefill(P, L)
     _check_kcomp(P, L)
     kb = cfg.topk_blocks
     _isolated_checks(P, inp.q, L, "topk", k_blocks=kb, label=f"cfg{cid}")
-    step = P.step(S.SELECT_TOPK, budget=cfg.budget)
+    step = P.step(S.SELECT_TOPK, budget=cfg.budget, single_launch=single)
+    assert step.single_launch == single
     mism, n, _ = _run_and_check(P, step, inp.q, L, "topk", k_blocks=kb, label=f"cfg{cid}")
     assert mism <= max(1, n // 20), f"cfg{cid}: {mism}/{n} lists differ (all at the cutoff)"
     if cfg.hot_blocks:
@@ -236,7 +240,7 @@ def test_paged_ragged_workload():
     outputs through DecodeStep against the oracle, as for the contiguous workloads."""
     from synthetic import paged_view
     cfg = config(3, B=4)
-    inp = make_inputs(cfg, tail="nan")
+    inp = make_inputs(cfg, tail="nan", workers=draw_workers())
     P = Problem(inp)
     L = inp.seqlens
     assert np.all(L % cfg.block != 0)
@@ -248,16 +252,89 @@ def test_paged_ragged_workload():
     S.kcomp_update(P.sh, kk, torch.from_numpy(L).cuda(), P.valid, P.w_k, P.kc)
     torch.cuda.synchronize()
     _check_kcomp(P, L)
-    step = S.DecodeStep(P.sh, kk, vv, P.w_q, P.w_k, P.kc, P.valid, mode=S.SELECT_TOPK, token_budget=cfg.budget)
-    mism, n, _ = _run_and_check(P, step, inp.q, L, "topk", k_blocks=cfg.topk_blocks, label="paged cfg3")
-    assert mism <= max(1, n // 20), f"paged cfg3: {mism}/{n} lists differ (all at the cutoff)"
-    cnt = step.block_cnt.cpu().numpy()
-    assert np.all(cnt == cfg.topk_blocks + 1), "every list holds k blocks plus the forced partial block"
+    for single in (False, True):
+        step = S.DecodeStep(P.sh, kk, vv, P.w_q, P.w_k, P.kc, P.valid, mode=S.SELECT_TOPK, token_budget=cfg.budget,
+                            num_split=-1, single_launch=single)
+        mism, n, _ = _run_and_check(P, step, inp.q, L, "topk", k_blocks=cfg.topk_blocks,
+                                    label=f"paged cfg3 single={single}")
+        assert mism <= max(1, n // 20), f"paged cfg3: {mism}/{n} lists differ (all at the cutoff)"
+        cnt = step.block_cnt.cpu().numpy()
+        assert np.all(cnt == cfg.topk_blocks + 1), "every list holds k blocks plus the forced partial block"
+
+
+def _step_loop(P, step, L0, steps, mode, k_blocks=0, tau=0.0, label=""):
+    """Decode `steps` appended tokens (step s sees L0 + s + 1): every step against the oracle, the
+    cache entries below the previous fill count frozen, the fill counts advancing as blocks fill."""
+    c = P.cfg
+    for s_ in range(steps):
+        L = L0 + s_ + 1
+        q_bits = make_step_query(c, s_)
+        before = P.kc.clone()
+        prev = torch.from_numpy(((L - 1) // c.block).astype(np.int32))
+        mism, n, _ = _run_and_check(P, step, q_bits, L, mode, k_blocks=k_blocks, tau=tau, label=f"{label} s{s_}")
+        assert mism <= max(1, n // 20)
+        for b in range(c.B):
+            pv = int(prev[b])
+            assert torch.equal(before[b, :, :pv].view(torch.int16), P.kc[b, :, :pv].view(torch.int16)), \
+                f"{label} s{s_}: frozen entries of b{b} changed"
+        assert P.valid.cpu().tolist() == [[int(x) // c.block] * c.Hkv for x in L], f"{label} s{s_}: fill counts"
+    _check_kcomp(P, L0 + steps)
+
+
+def test_single_launch_steps_across_block_fills():
+    """The one-launch step over appended tokens: blocks fill mid-run, so the launch's planning
+    phase writes new cache entries before its gate reads them; the ready flags must come back to
+    zero after every launch (each step depends on it)."""
+    blk = 64
+    L0 = np.array([40 * blk - 3, 33 * blk + 61, 17 * blk - 1], dtype=np.int32)
+    steps = 6
+    cfg = config(2, B=3, steps=steps + 1)   # the loop's last length is L0 + steps
+    inp = make_inputs(cfg, lengths=list(L0), tail="nan")
+    P = Problem(inp)
+    _prefill(P, L0)
+    step = P.step(S.SELECT_TOPK, budget=cfg.budget, num_split=-1, single_launch=True)
+    _step_loop(P, step, L0, steps, "topk", k_blocks=cfg.topk_blocks, label="fills")
+
+
+def test_single_launch_threshold_many_rows():
+    """Threshold selection on the capacity schedule as one launch, with more (b, h) rows than
+    planning clusters (clusters plan several rows each) and ragged short lengths."""
+    blk, d, g, Hkv, B = 64, 128, 4, 2, 48
+    rng = np.random.default_rng(77)
+    lengths = [int(x) for x in rng.integers(1, 24 * blk, B)]
+    cfg = config(1, B=B, Hq=g * Hkv, Hkv=Hkv, head_dim=d, gate_dim=128, block=blk, seed=8080, mode="threshold")
+    inp = make_inputs(cfg, lengths=lengths, tail="nan")
+    P = Problem(inp)
+    L = inp.seqlens
+    _prefill(P, L)
+    tau = 1.0 / 64.0   # exact in float32, the kernel's threshold type
+    step = P.step(S.SELECT_THRESHOLD, tau=tau, num_split=-1, single_launch=True)
+    for rep in range(2):
+        mism, n, _ = _run_and_check(P, step, inp.q, L, "threshold", tau=tau, label=f"threshold rep{rep}")
+        assert mism <= n // 50 + 1
+
+
+def test_single_launch_edge_lengths():
+    """Lengths 0, 1, b - 1, b, b + 1 and 2b + 2 in one launch: an empty row (zero output, lse -inf),
+    rows with only the forced partial block, a row with one full block and none partial."""
+    blk, d, g, Hkv = 64, 128, 4, 2
+    lengths = [0, 1, blk - 1, blk, blk + 1, 2 * blk + 2]
+    cfg = config(1, B=len(lengths), Hq=g * Hkv, Hkv=Hkv, head_dim=d, gate_dim=128, block=blk, seed=9191)
+    inp = make_inputs(cfg, lengths=lengths, tail="nan")
+    P = Problem(inp)
+    L = inp.seqlens
+    _prefill(P, L)
+    step = P.step(S.SELECT_TOPK, budget=2 * blk, num_split=-1, single_launch=True)
+    mism, n, _ = _run_and_check(P, step, inp.q, L, "topk", k_blocks=2, pairs=[(b, h) for b in range(1, 6)
+                                                                                for h in range(Hkv)], label="edges")
+    assert mism == 0
+    assert step.block_cnt[0].cpu().tolist() == [0] * Hkv
+    assert torch.all(step.out[0].float() == 0.0) and torch.all(torch.isneginf(step.lse[0]))
 
 
 def test_sparsity_sweep_and_dense_path():
     cfg = config(4)
-    inp = make_inputs(cfg)
+    inp = make_inputs(cfg, workers=draw_workers())
     P = Problem(inp)
     L = inp.seqlens
     _prefill(P, L)
@@ -317,7 +394,7 @@ def _calibrate_temperatures(inp, tau, fractions):
 
 def test_threshold_decode_loop_256_steps():
     cfg = config(5)
-    inp = make_inputs(cfg)
+    inp = make_inputs(cfg, workers=draw_workers())
     tau = cfg.tau
     fractions = np.linspace(0.05, 0.24, cfg.Hkv)
     temps = _calibrate_temperatures(inp, tau, fractions)

@@ -13,7 +13,7 @@ import pytest
 import torch
 
 from oracle import seer_oracle as O
-from seer_harness import OracleBH, bf16_bits, check_attention, check_lse, f64, to_dev_bf16
+from seer_harness import OracleBH, bf16_bits, check_attention, check_lse, draw_workers, f64, to_dev_bf16
 from synthetic import config, make_inputs
 
 pytestmark = pytest.mark.gpu
@@ -28,7 +28,7 @@ GT_REL_PREFILL = 4e-3    # as tests/test_gpu_prefill_gt.py
 @functools.lru_cache(maxsize=1)
 def _step_32k():
     cfg = config(2)
-    return cfg, make_inputs(cfg)
+    return cfg, make_inputs(cfg, workers=draw_workers())
 
 
 def test_ground_truth_32k_sampled():

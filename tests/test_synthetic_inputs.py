@@ -90,3 +90,29 @@ def test_pair_inputs_are_the_batch_slices():
                 assert np.array_equal(pi.k, inp.k[b, h]) and np.array_equal(pi.v, inp.v[b, h])
                 assert np.array_equal(pi.q, inp.q[b, h * cfg.g:(h + 1) * cfg.g])
                 assert np.array_equal(pi.w_q, inp.w_q[h]) and np.array_equal(pi.w_k, inp.w_k[h])
+
+
+def test_parallel_draw_is_the_serial_draw():
+    """Drawing the K / V slices in spawned processes gives the serial loop's bytes, planted blocks
+    and NaN tails."""
+    cfg = config(2, B=3, Hkv=2, Hq=8, length=700, steps=3)
+    a = make_inputs(cfg, tail="nan", lengths=[700, 650, 3])
+    b = make_inputs(cfg, tail="nan", lengths=[700, 650, 3], workers=3)
+    assert np.array_equal(a.k, b.k) and np.array_equal(a.v, b.v)
+    assert a.hot == b.hot and np.array_equal(a.seqlens, b.seqlens)
+
+
+def test_bf16_rounding_matches_torch():
+    """The generator's float32 -> bf16 rounding (nearest, ties to even) against torch's conversion on
+    every exponent with mantissas at, just below and just above the rounding midpoints, odd and even
+    kept parts, zeros, infinities and subnormals (NaN payloads excluded: torch canonicalises them)."""
+    import torch
+    from synthetic import bf16_bits_from_f32
+    mant = np.array([0, 1, 0x7FFF, 0x8000, 0x8001, 0x17FFF, 0x18000, 0x18001, 0x7FFFFF, 0x7F8000, 0x3FFFFF],
+                    dtype=np.uint32)
+    exps = np.arange(0, 255, dtype=np.uint32)
+    bits = ((exps[:, None] << np.uint32(23)) | mant[None, :]).ravel()
+    bits = np.concatenate([bits, bits | np.uint32(0x80000000), np.array([0x7F800000, 0xFF800000], np.uint32)])
+    x = bits.view(np.float32)
+    want = torch.from_numpy(x.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(bf16_bits_from_f32(x), want)

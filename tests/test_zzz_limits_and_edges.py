@@ -234,20 +234,20 @@ def test_repeat_runs_are_bitwise_identical():
     def bits(t):
         return t.contiguous().view(torch.int32 if t.element_size() == 4 else torch.int16).cpu()
 
-    for fused in (True, False):
+    for fused, ns in ((True, 2), (False, 2), (True, -1)):   # (True, -1): the whole step as one launch
         runs = []
         for _ in range(2):
             kc = torch.zeros((cfg.B, Hkv, nb, dg), dtype=torch.bfloat16, device="cuda")
             valid = torch.zeros(cfg.B, Hkv, dtype=torch.int32, device="cuda")
             st = S.DecodeStep(sh, kv_k, kv_v, dv["w_q"], dv["w_k"], kc, valid, mode=S.SELECT_TOPK,
-                              token_budget=4 * blk, num_split=2)
+                              token_budget=4 * blk, num_split=ns, single_launch=ns == -1)
             st.run(dv["q"], dv["seqlens"], fused=fused)
             torch.cuda.synchronize()
             assert int(st.err.item()) == 0
             runs.append(st)
         a, b = runs
         for name in ("kcomp", "valid_blocks", "block_idx", "block_cnt", "out", "lse"):
-            assert torch.equal(bits(getattr(a, name)), bits(getattr(b, name))), f"fused={fused}: {name}"
+            assert torch.equal(bits(getattr(a, name)), bits(getattr(b, name))), f"fused={fused} ns={ns}: {name}"
         for bb, L in enumerate(lengths):
             n = L // blk
             assert torch.equal(bits(a.logits[bb, :, :n]), bits(b.logits[bb, :, :n])), f"fused={fused}: logits"
