@@ -1,0 +1,535 @@
+// The prefill forward with block targets on the 5th-generation tensor cores
+// (tcgen05 / TMEM): causal attention over whole sequences, each query row's
+// maximum pre-softmax score per key block kept on the way, and from those the
+// block-level target of every position.
+//
+// "SeerAttention-R: Sparse Attention Adaptation for Long Reasoning"
+// (chapterpal.com summary), Knowl 3 (the target of query i: its softmax row,
+// 1-D max-pooled over each block's columns, max over the GQA group's heads,
+// normalised to sum to 1) and Knowl 4 (the extraction inside the attention
+// forward: per key tile each row's maximum pre-softmax score r is stored; once
+// the row's final maximum m and normaliser l are known, the block's score is
+// exp(r - m) / l).  Same results as prefill_gt.cu (the warp-level mma form,
+// kept for the shapes this kernel does not take: head_dim 64, groups that do
+// not divide 128 rows).
+//
+// One CTA per (128 query rows, kv head, sequence): the g heads of the group x
+// 128/g consecutive positions, row r = head (r / P) at position p0 + (r % P).
+// Key tiles of 128 keys (one or two blocks).
+//   warps 0, 6 producers: K tiles (three-stage ring, a stage freed once S has
+//              read it) and V tiles (two stages, freed once P.V has read
+//              them) by TMA (128-byte swizzle, boxes of 64 channels x b keys)
+//   warp 1     allocates TMEM; one lane issues the MMAs: S_n = Q K_n^T into
+//              TMEM S[n % 2] (M = 128 rows, N = 128 keys, K = d), then
+//              O += P_{n-1} V_{n-1} into TMEM O (N = d, K = 128 keys), each
+//              group closed by a commit to an mbarrier
+//   warps 2-5  one thread per row (its TMEM lane): S row by tcgen05.ld, causal
+//              mask, the row maximum of each block (stored for the targets),
+//              P = exp2(s - m_ref) as bf16 into a shared tile (once the last
+//              P.V has read it),
+//              V rows past the sequence zeroed (the cache may hold NaN there),
+//              at the end O / l, the LSE and the targets
+// The reference maximum m_ref moves only when a tile's maximum exceeds it by
+// more than 8 (log2 units), so P stays <= 2^8 and O in TMEM is rescaled (ld,
+// scale, st) only then; l and the LSE use the same reference, so the results
+// are those of the exact online softmax (l sums the probabilities before their
+// rounding to bf16 for the P.V product).  All waits are bounded.
+#include "seer_device.cuh"
+#include "seer_internal.h"
+
+namespace seer {
+namespace {
+
+constexpr float kLn2f = 0.6931471805599453f;
+constexpr int kD = 128;                 // head_dim of this kernel
+constexpr int kM = 128;                 // query rows per CTA
+constexpr int kKT = 128;                // keys per tile
+constexpr int kBoxB = kM * 128;         // bytes of a 128-row x 64-channel (or 64-key) 128B-swizzled box
+constexpr int kTileB = 2 * kBoxB;       // 32 KB: a K, V, Q or P tile (two boxes)
+constexpr int kKStages = 3;
+constexpr int kVStages = 2;
+constexpr int kThreads = 7 * 32;
+constexpr uint32_t kTmemCols = 512;     // S[0] 0..127, S[1] 128..255, O 256..383
+constexpr float kLazy = 8.f;            // m_ref moves when a tile maximum exceeds it by more than this
+constexpr size_t kSmem = 1024 + kTileB /* Q */ + (size_t)(kKStages + kVStages) * kTileB /* K, V */ + kTileB /* P */ +
+                         256 /* barriers */ + 2 * kM * 4 /* m, l */;
+
+// shared-memory matrix descriptors (sm_100 layout): start >> 4 in [0,14), leading byte offset
+// >> 4 in [16,30), stride byte offset >> 4 in [32,46), version 1 at bit 46, 128-byte swizzle (2)
+// in [61,64).  K-major operand in 128B-swizzled rows: stride offset = 8 rows (1024 B), leading
+// offset unused.  MN-major operand (V as B of P.V, keys along K): leading offset = the next 64
+// channels (one box), stride offset = the next 8 keys (1024 B).
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t saddr, uint32_t lbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+         ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// kind::f16 instruction descriptor: D f32 (bits 4-5 = 1), A and B bf16 (7-9 = 1, 10-12 = 1),
+// B major bit 16 (1 = MN-major), N / 8 in [17,23), M / 16 in [24,29)
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(da), "l"(db), "r"(idesc), "r"(acc));
+}
+// arrive on `bar` once every MMA this thread issued so far has completed
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+
+// 32 consecutive fp32 columns of this thread's TMEM lane
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
+      "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])),
+      "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
+      "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])),
+      "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31])));
+}
+// 2^x on the SFU (denormal results flushed to zero: a probability that small is zero in the sums)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void kv_coords(const int32_t perm[3], int t, int h, int bp, int& c1, int& c2, int& c3) {
+  int c[3];
+  c[perm[0]] = t;
+  c[perm[1]] = h;
+  c[perm[2]] = bp;
+  c1 = c[0];
+  c2 = c[1];
+  c3 = c[2];
+}
+
+template <int BLK>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                      const __grid_constant__ PrefillParams p) {
+  constexpr int NBT = kKT / BLK;   // blocks per key tile
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* qs = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* kring = qs + kTileB;                        // [kKStages] K tiles
+  uint8_t* vring = kring + (size_t)kKStages * kTileB;  // [kVStages] V tiles
+  uint8_t* ps = vring + (size_t)kVStages * kTileB;     // P tile
+  uint64_t* k_full = reinterpret_cast<uint64_t*>(ps + kTileB);
+  uint64_t* k_empty = k_full + kKStages;
+  uint64_t* v_full = k_empty + kKStages;
+  uint64_t* v_empty = v_full + kVStages;
+  uint64_t* s_full = v_empty + kVStages;   // [2]
+  uint64_t* s_free = s_full + 2;           // [2]
+  uint64_t* p_full = s_free + 2;
+  uint64_t* p_free = p_full + 1;     // one completion per P.V (P read; tiles 0..m in O)
+  uint64_t* o_fin = p_free + 1;      // the last P.V done (single use)
+  uint64_t* q_ready = o_fin + 1;
+  uint64_t* drain = q_ready + 1;
+  uint64_t* cbar = drain + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cbar + 1);
+  volatile int* sh = reinterpret_cast<volatile int*>(tmem_slot + 1);   // [0] abort
+  float* ms = reinterpret_cast<float*>(ps + kTileB + 256);             // [128] final m_ref per row
+  float* ls = ms + kM;                                                 // [128] final l per row
+
+  const int g = p.g, P = kM / g;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  const int b = blockIdx.z, hk = blockIdx.y;
+  const int p0 = ((int)gridDim.x - 1 - (int)blockIdx.x) * P;   // heaviest (latest) positions first
+
+  if (tid == 0) {
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+    }
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(&s_full[k], 1);
+      mbar_init(&s_free[k], 4);
+    }
+    mbar_init(p_full, 4);
+    mbar_init(p_free, 1);
+    mbar_init(o_fin, 1);
+    mbar_init(q_ready, 4);
+    mbar_init(drain, 1);
+    mbar_init(cbar, 4);
+    sh[0] = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  pdl_wait();
+  pdl_trigger();
+  const int Lr = max(p.seqlens[b], 0);
+  const int L = min(Lr, min(p.T, p.kcap));
+  if (Lr > L && blockIdx.x == 0 && hk == 0 && tid == 0) report(p.err, SEER_DEVERR_COUNT);
+  if (p0 >= L) return;   // the whole CTA: no position of these rows exists (no TMEM taken yet)
+  const int pend = min(p0 + P, L);
+  const int nt = (pend - 1) / kKT + 1;   // key tiles 0 .. nt-1 hold a key visible to some row
+
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS[2] = {tmem, tmem + 128}, tO = tmem + 256;
+
+  if (warp == 0 || warp == 6) {
+    // ---------------------------------------------------------------- producers (K: warp 0, V: warp 6)
+    const bool isK = warp == 0;
+    const int NS = isK ? kKStages : kVStages;
+    uint64_t* full = isK ? k_full : v_full;
+    uint64_t* empty = isK ? k_empty : v_empty;
+    uint8_t* ringb = isK ? kring : vring;
+    const CUtensorMap* tm = isK ? &tmK : &tmV;
+    const int32_t* perm = isK ? p.k_perm : p.v_perm;
+    if (lane == 0) {
+      int issued = 0;
+      for (int n = 0; n < nt; ++n) {
+        const int s = n % NS;
+        if (n >= NS && !mbar_wait(&empty[s], ((n / NS) - 1) & 1)) {
+          report(p.err, SEER_DEVERR_TIMEOUT);
+          sh[0] = 1;
+          break;
+        }
+        if (sh[0]) break;
+        issued = n + 1;
+        mbar_arrive_expect_tx(&full[s], (uint32_t)kTileB);
+        uint8_t* dst = ringb + (size_t)s * kTileB;
+#pragma unroll
+        for (int sub = 0; sub < NBT; ++sub) {
+          // a 64-channel box of BLK keys; the tile's two channel halves are kBoxB apart, its blocks
+          // BLK rows (BLK * 128 bytes) apart within a half
+          int c1, c2, c3;
+          kv_coords(perm, n * kKT + sub * BLK, hk, b, c1, c2, c3);
+#pragma unroll
+          for (int hx = 0; hx < 2; ++hx)
+            tma_load_4d(dst + hx * kBoxB + sub * BLK * 128, tm, &full[s], hx * 64, c1, c2, c3);
+        }
+      }
+      // copies still landing when a consumer gave up: wait for them (bounded) before shared memory
+      // is released; no later phase is ever armed on those stages
+      for (int n = max(0, issued - NS); n < issued; ++n) mbar_wait(&full[n % NS], (n / NS) & 1);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t id_s = idesc_bf16(kM, kKT, 0), id_o = idesc_bf16(kM, kD, 1);
+      const uint32_t qa = smem_u32(qs);
+      bool ok = mbar_wait(q_ready, 0);
+      auto issue_pv = [&](int m) {
+        const int sv = m % kVStages;
+        ok = ok && mbar_wait(p_full, m & 1) && mbar_wait(&v_full[sv], (m / kVStages) & 1);
+        if (!ok) return;
+        tc_fence_after();
+        const uint32_t pa = smem_u32(ps);
+        const uint32_t vb = smem_u32(vring + (size_t)sv * kTileB);
+#pragma unroll
+        for (int kk = 0; kk < kKT / 16; ++kk)
+          umma_f16(tO, desc_kmajor(pa + (kk >> 2) * kBoxB + (kk & 3) * 32), desc_mnmajor(vb + kk * 2048, kBoxB),
+                   id_o, (m > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&v_empty[sv]);
+        umma_commit(p_free);
+      };
+      for (int n = 0; n < nt && ok; ++n) {
+        const int sk = n % kKStages, k2 = n & 1;
+        ok = ok && mbar_wait(&k_full[sk], (n / kKStages) & 1);
+        ok = ok && (n < 2 || mbar_wait(&s_free[k2], ((n >> 1) - 1) & 1));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t kb = smem_u32(kring + (size_t)sk * kTileB);
+#pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks)
+          umma_f16(tS[k2], desc_kmajor(qa + (ks >> 2) * kBoxB + (ks & 3) * 32),
+                   desc_kmajor(kb + (ks >> 2) * kBoxB + (ks & 3) * 32), id_s, ks > 0 ? 1u : 0u);
+        umma_commit(&k_empty[sk]);
+        umma_commit(&s_full[k2]);
+        if (n > 0) issue_pv(n - 1);
+      }
+      if (ok) issue_pv(nt - 1);
+      if (ok) umma_commit(o_fin);
+      if (!ok) {
+        report(p.err, SEER_DEVERR_TIMEOUT);
+        sh[0] = 1;
+      }
+      // every MMA issued so far retires before TMEM is released (bounded)
+      umma_commit(drain);
+      mbar_wait(drain, 0);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax warps (one row each)
+    const int row = 32 * (warp & 3) + lane;   // TMEM lane of this thread (warp w reads lanes 32(w%4)..)
+    const int j = row / P, t = row - (row / P) * P;
+    const int h = hk * g + j, i = p0 + t;     // query head and position of the row
+    const bool live = i < L;
+    const int vis = min(i, L - 1);            // last key the row sees
+    const size_t qrow = ((size_t)b * p.Hq + h) * p.T;
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    // the Q row -> shared memory (K-major 128B swizzle: two 64-channel boxes), zero past L
+#pragma unroll
+    for (int c = 0; c < kD / 8; ++c) {
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (live) v = *reinterpret_cast<const uint4*>(p.q + (qrow + i) * kD + c * 8);
+      *reinterpret_cast<uint4*>(qs + (c >> 3) * kBoxB + sw128(row, c & 7)) = v;
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+    if (lane == 0) mbar_arrive(q_ready);
+    const float sl2 = p.scale_log2;
+    float* rws = p.rmax + ((size_t)b * p.Hq + h) * p.NB * p.T;
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int n = 0; n < nt && ok; ++n) {
+      const int k2 = n & 1, sv = n % kVStages;
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[k2], (n >> 1) & 1));
+      if (!ok) break;
+      tc_fence_after();
+      float x[kKT];
+#pragma unroll
+      for (int c0 = 0; c0 < kKT; c0 += 32) tmem_ld32(tS[k2] + lane_base + c0, x + c0);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[k2]);   // S[k2] may be overwritten (tile n + 2)
+      // causal mask (key kt visible to row i iff kt <= min(i, L - 1)) where the tile needs one, and
+      // the row maximum of each block of the tile (raw scores: the scale is positive)
+      const int k0 = n * kKT;
+      const bool masked = k0 + kKT - 1 > vis;
+      if (masked) {
+#pragma unroll
+        for (int c = 0; c < kKT; ++c) x[c] = (k0 + c <= vis) ? x[c] : -INFINITY;
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int sub = 0; sub < NBT; ++sub) {
+        float r = -INFINITY;
+#pragma unroll
+        for (int c = sub * BLK; c < (sub + 1) * BLK; ++c) r = fmaxf(r, x[c]);
+        r *= sl2;   // log2 domain
+        const int blk = n * NBT + sub;
+        if (live && blk * BLK <= i) rws[(size_t)blk * p.T + i] = r;
+        mx = fmaxf(mx, r);
+      }
+      // reference maximum: the first tile's, moved only when a tile exceeds it by more than kLazy;
+      // then O (in TMEM, holding tiles 0..n-1) and l are rescaled
+      float alpha = 1.f;
+      bool move = false;
+      if (n == 0) {
+        m_ref = mx;
+      } else if (mx > m_ref + kLazy) {
+        alpha = ex2(m_ref - mx);
+        m_ref = mx;
+        move = true;
+      }
+      l *= alpha;
+      // the P.V of tile n - 1 (the n-th completion of p_free; S_n's commit, observed above, came after
+      // the P.V of tile n - 2, so the barrier is at most one completion behind and a parity wait is
+      // exact) has read the P tile and added tile n - 1 to O
+      if (n > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(p_free, (n - 1) & 1));
+        if (!ok) break;
+      }
+      if (__any_sync(0xffffffffu, move)) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int c0 = 0; c0 < kD; c0 += 32) {
+          float o[32];
+          tmem_ld32(tO + lane_base + c0, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] *= alpha;
+          tmem_st32(tO + lane_base + c0, o);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+      }
+      // P = exp2(s * scale - m_ref) (<= 2^kLazy; masked keys give 0) as bf16; l sums the same values
+      const float mu = m_ref == -INFINITY ? 0.f : m_ref;
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < kKT / 8; ++c) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float a = ex2(fmaf(x[8 * c + 2 * e], sl2, -mu)), bb = ex2(fmaf(x[8 * c + 2 * e + 1], sl2, -mu));
+          sum += a + bb;
+          w[e] = pack_bf16(a, bb);
+        }
+        *reinterpret_cast<uint4*>(ps + (c >> 3) * kBoxB + sw128(row, c & 7)) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      l += sum;
+      if (k0 + kKT > L) {
+        // V rows past L may hold anything (even NaN): zero them so that P = 0 there gives 0.  Wait for
+        // the tile's copy here too (its phase is at most one behind, as for the MMA issuer); whole
+        // 128-byte rows, so the swizzle does not matter.
+        ok = __all_sync(0xffffffffu, mbar_wait(&v_full[sv], (n / kVStages) & 1));
+        if (!ok) break;
+        uint8_t* vt = vring + (size_t)sv * kTileB;
+        const int r0 = max(0, L - k0), nchunk = (kKT - r0) * 8;   // 16-byte chunks per channel half
+        for (int e = tid - 64; e < 2 * nchunk; e += 128) {
+          const int hx = e / nchunk, rr = r0 + (e - hx * nchunk) / 8, cc = e & 7;
+          *reinterpret_cast<uint4*>(vt + hx * kBoxB + rr * 128 + cc * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    if (ok) {
+      // the last P.V (its own barrier: p_free may be two completions behind here), then O / l, the
+      // LSE, the row statistics
+      ok = __all_sync(0xffffffffu, mbar_wait(o_fin, 0));
+    }
+    if (ok) {
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll 1
+      for (int c0 = 0; c0 < kD; c0 += 32) {
+        float o[32];
+        tmem_ld32(tO + lane_base + c0, o);
+        tmem_wait_ld();
+        if (live) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 w;
+            w.x = pack_bf16(o[e] * inv, o[e + 1] * inv);
+            w.y = pack_bf16(o[e + 2] * inv, o[e + 3] * inv);
+            w.z = pack_bf16(o[e + 4] * inv, o[e + 5] * inv);
+            w.w = pack_bf16(o[e + 6] * inv, o[e + 7] * inv);
+            *reinterpret_cast<uint4*>(p.o + (qrow + i) * kD + c0 + e) = w;
+          }
+        }
+      }
+      if (live && p.lse) p.lse[qrow + i] = l > 0.f ? (m_ref + log2f(l)) * kLn2f : -INFINITY;
+      ms[row] = m_ref;
+      ls[row] = l;
+    } else {
+      if (lane == 0) report(p.err, SEER_DEVERR_TIMEOUT);
+      sh[0] = 1;
+    }
+    // ---- the targets: the four softmax warps meet (bounded; the block maxima the other warps
+    // wrote are read back through L2), then 8 threads per position, blocks strided by 8
+    __threadfence();
+    uint32_t cph = 0;
+    const bool met = warps_sync(cbar, cph) && ok;
+    if (!met && lane == 0) report(p.err, SEER_DEVERR_TIMEOUT);
+    const int st = tid - 64;   // 0..127
+    const int sub = st & 7;
+    float* gt_b = p.gt + ((size_t)b * p.Hkv + hk) * p.T * p.NB;
+    const float* r_b = p.rmax + ((size_t)b * p.Hq + (size_t)hk * g) * p.NB * p.T;
+    for (int base = 0; base < P && met; base += 16) {
+      const int pi = base + st / 8;
+      const int ip = p0 + pi;
+      const bool lv = pi < P && ip < L;
+      const int nb_i = lv ? ip / BLK + 1 : 0;   // blocks with a key visible to position ip
+      // a block's score, four blocks at a time with every load issued before any use (two passes:
+      // the sum, then the normalised stores)
+      auto scores4 = [&](int n0, float (&v)[4]) {
+        float r[4][kMaxGroup];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int jj = 0; jj < kMaxGroup; ++jj)
+            r[u][jj] = (jj < g && n0 + 8 * u < nb_i) ? __ldcg(r_b + ((size_t)jj * p.NB + n0 + 8 * u) * p.T + ip)
+                                                      : -INFINITY;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          v[u] = 0.f;
+#pragma unroll
+          for (int jj = 0; jj < kMaxGroup; ++jj)
+            if (jj < g && n0 + 8 * u < nb_i) v[u] = fmaxf(v[u], exp2f(r[u][jj] - ms[jj * P + pi]) / ls[jj * P + pi]);
+        }
+      };
+      float sum = 0.f;
+      for (int n0 = sub; n0 < nb_i; n0 += 32) {
+        float v[4];
+        scores4(n0, v);
+        sum += (v[0] + v[1]) + (v[2] + v[3]);
+      }
+      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+      sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+      const float inv = sum > 0.f ? 1.f / sum : 0.f;
+      if (lv) {
+        for (int n0 = sub; n0 < nb_i; n0 += 32) {
+          float v[4];
+          scores4(n0, v);
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (n0 + 8 * u < nb_i) gt_b[(size_t)ip * p.NB + n0 + 8 * u] = v[u] * inv;
+        }
+        for (int nn = (nb_i & ~7) + sub; nn < p.NB; nn += 8)
+          if (nn >= nb_i) gt_b[(size_t)ip * p.NB + nn] = 0.f;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+  }
+}
+
+template <int BLK>
+cudaError_t launch_tc_t(const CUtensorMap& tk, const CUtensorMap& tv, const PrefillParams& p, int max_len,
+                        cudaStream_t st) {
+  auto kern = prefill_tc_kernel<BLK>;
+  static std::atomic<uint64_t> attr_done{0};
+  cudaError_t e = ensure_smem_limit(kern, (int)kSmem, attr_done);
+  if (e != cudaSuccess) return e;
+  const int P = kM / p.g;
+  const dim3 grid((max_len + P - 1) / P, p.Hkv, p.B);
+  return launch_pdl(kern, grid, dim3(kThreads), kSmem, st, tk, tv, p);
+}
+
+}  // namespace
+
+bool prefill_tc_supported(int D, int BLK, int g) {
+  return D == kD && (BLK == 64 || BLK == 128) && (g == 1 || g == 2 || g == 4 || g == 8);
+}
+
+cudaError_t launch_prefill_tc(const CUtensorMap& tk, const CUtensorMap& tv, const PrefillParams& p, int D, int BLK,
+                              int max_len, cudaStream_t s) {
+  if (!prefill_tc_supported(D, BLK, p.g)) return cudaErrorInvalidValue;
+  return BLK == 64 ? launch_tc_t<64>(tk, tv, p, max_len, s) : launch_tc_t<128>(tk, tv, p, max_len, s);
+}
+
+}  // namespace seer

@@ -391,8 +391,12 @@ seer_status seer_prefill_gt(const seer_dims_t* dims, const void* q, int32_t max_
   const float scale = dims->softmax_scale > 0.f ? dims->softmax_scale : 1.0f / sqrtf((float)dims->head_dim);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.err = err_word;
-  cudaError_t e = seer::launch_prefill_gt(tk, tv, p, dims->head_dim, dims->block_size, max_len,
-                                          static_cast<cudaStream_t>(stream));
+  // the tcgen05 / TMEM kernel where it takes the shape, the warp-level mma kernel otherwise
+  cudaError_t e = seer::prefill_tc_supported(dims->head_dim, dims->block_size, p.g)
+                      ? seer::launch_prefill_tc(tk, tv, p, dims->head_dim, dims->block_size, max_len,
+                                                static_cast<cudaStream_t>(stream))
+                      : seer::launch_prefill_gt(tk, tv, p, dims->head_dim, dims->block_size, max_len,
+                                                static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "prefill_gt launch");
   return SEER_OK;
 }

@@ -78,3 +78,45 @@ def _check_case(d, blk, g, Hkv, nan_tail, lengths=None):
                                          (128, 64, 5, 1)])
 def test_prefill_gt_vs_oracle(d, blk, g, Hkv):
     _check_case(d, blk, g, Hkv, nan_tail=False)
+
+
+def test_prefill_rescales_when_later_keys_dominate():
+    """Keys planted in the second and third 128-key tiles score far above everything before them for
+    every query row: each row's running maximum jumps by more than 2^8 (log2 units) once past key 150
+    and again past key 290 -- so a kernel that moves its reference maximum lazily must rescale its
+    accumulated output -- while the scores stay moderate (<= 17 in natural units: q = noise
+    orthogonal to a direction u plus 2u; planted keys 5 sqrt(d) u and 8.5 sqrt(d) u, so their
+    scores are 10 and 17 against N(0, 1) elsewhere).  Output, LSE and targets against the exact
+    softmax of the oracle."""
+    d, blk, g, Hkv, T = 128, 64, 4, 1, 400
+    rng = np.random.default_rng(4711)
+    u = rng.standard_normal(d)
+    u /= np.linalg.norm(u)
+    noise = rng.standard_normal((1, g * Hkv, T, d))
+    noise -= (noise @ u)[..., None] * u
+    qf = noise + 2.0 * u
+    kf = rng.standard_normal((1, Hkv, T, d))
+    kf[0, :, 150] = 5.0 * u * math.sqrt(d)         # tile 1 (keys 128..255)
+    kf[0, :, 290] = 8.5 * u * math.sqrt(d)         # tile 2 (keys 256..383)
+    q, k = _bf16_bits(qf), _bf16_bits(kf)
+    v = _bf16_bits(rng.standard_normal((1, Hkv, T, d)))
+    sh = S.Shape(1, g * Hkv, Hkv, d, 64, blk, -(-T // blk))
+    seq = torch.tensor([T], dtype=torch.int32, device="cuda")
+    out = torch.empty((1, g * Hkv, T, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((1, g * Hkv, T), dtype=torch.float32, device="cuda")
+    gt = torch.empty((1, Hkv, T, sh.max_blocks), dtype=torch.float32, device="cuda")
+    ws = torch.empty(S.prefill_gt_workspace_bytes(sh, T), dtype=torch.uint8, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    S.prefill_gt(sh, to_dev_bf16(q), S.KVCache.contiguous(to_dev_bf16(k)), S.KVCache.contiguous(to_dev_bf16(v)),
+                 seq, out, gt, ws, lse=lse, err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    ro, rl, rg = O.prefill_ground_truth(f64(q[0]), f64(k[0, 0]), f64(v[0, 0]), blk, 1.0 / math.sqrt(d))
+    # the planted keys do raise the maxima: positions past key 290 put most of their mass on it
+    assert float(np.median(rg[300:, 290 // blk])) > 0.5
+    o_h, lse_h, gt_h = f64(bf16_bits(out)), lse.cpu().numpy().astype(np.float64), gt.cpu().numpy()
+    for j in range(g):
+        check_attention(o_h[0, j], ro[j], f"head {j}")
+        check_lse(lse_h[0, j], rl[j], f"head {j}")
+    bad = np.abs(gt_h[0, 0, :, :rg.shape[1]] - rg) > GT_REL * rg + 1e-7
+    assert not bad.any(), f"{int(bad.sum())} target entries off"
