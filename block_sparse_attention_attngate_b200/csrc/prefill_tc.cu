@@ -16,15 +16,17 @@
 // One CTA per (128 query rows, kv head, sequence): the g heads of the group x
 // 128/g consecutive positions, row r = head (r / P) at position p0 + (r % P).
 // Key tiles of 128 keys (one or two blocks).
-//   warps 0, 6 producers: K tiles (three-stage ring, a stage freed once S has
+//   warps 0, 10 producers: K tiles (two-stage ring, a stage freed once S has
 //              read it) and V tiles (two stages, freed once P.V has read
 //              them) by TMA (128-byte swizzle, boxes of 64 channels x b keys)
 //   warp 1     allocates TMEM; one lane issues the MMAs: S_n = Q K_n^T into
 //              TMEM S[n % 2] (M = 128 rows, N = 128 keys, K = d), then
 //              O += P_{n-1} V_{n-1} into TMEM O (N = d, K = 128 keys), each
 //              group closed by a commit to an mbarrier
-//   warps 2-5  one thread per row (its TMEM lane): S row by tcgen05.ld, causal
-//              mask, the row maximum of each block (stored for the targets),
+//   warps 2-9  two threads per row (the row's TMEM lane; one thread per half of
+//              the 128 keys, the pair exchanging the tile's maxima through
+//              shared memory): S by tcgen05.ld, causal mask, the row maximum of
+//              each block (stored for the targets),
 //              P = exp2(s - m_ref) as bf16 into a shared tile (once the last
 //              P.V has read it),
 //              V rows past the sequence zeroed (the cache may hold NaN there),
@@ -46,13 +48,15 @@ constexpr int kM = 128;                 // query rows per CTA
 constexpr int kKT = 128;                // keys per tile
 constexpr int kBoxB = kM * 128;         // bytes of a 128-row x 64-channel (or 64-key) 128B-swizzled box
 constexpr int kTileB = 2 * kBoxB;       // 32 KB: a K, V, Q or P tile (two boxes)
-constexpr int kKStages = 3;
+constexpr int kKStages = 2;
 constexpr int kVStages = 2;
-constexpr int kThreads = 7 * 32;
+constexpr int kThreads = 11 * 32;
 constexpr uint32_t kTmemCols = 512;     // S[0] 0..127, S[1] 128..255, O 256..383
 constexpr float kLazy = 8.f;            // m_ref moves when a tile maximum exceeds it by more than this
 constexpr size_t kSmem = 1024 + kTileB /* Q */ + (size_t)(kKStages + kVStages) * kTileB /* K, V */ + kTileB /* P */ +
-                         256 /* barriers */ + 2 * kM * 4 /* m, l */;
+                         256 /* barriers */ + 2 * 2 * kM * 4 /* the pairs' tile maxima, two tiles */;
+
+static_assert(kSmem <= 227 * 1024, "dynamic shared memory above the per-CTA limit");
 
 // shared-memory matrix descriptors (sm_100 layout): start >> 4 in [0,14), leading byte offset
 // >> 4 in [16,30), stride byte offset >> 4 in [32,46), version 1 at bit 46, 128-byte swizzle (2)
@@ -156,10 +160,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* q_ready = o_fin + 1;
   uint64_t* drain = q_ready + 1;
   uint64_t* cbar = drain + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cbar + 1);
+  uint64_t* pbar = cbar + 1;         // [4] the two warps of each TMEM lane quarter
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pbar + 4);
   volatile int* sh = reinterpret_cast<volatile int*>(tmem_slot + 1);   // [0] abort
-  float* ms = reinterpret_cast<float*>(ps + kTileB + 256);             // [128] final m_ref per row
+  float* xch = reinterpret_cast<float*>(ps + kTileB + 256);            // [tile & 1][half][row] tile maxima
+  // after the last P.V the P tile is free: the row statistics live there
+  float* ms = reinterpret_cast<float*>(ps);                            // [128] final m_ref per row
   float* ls = ms + kM;                                                 // [128] final l per row
+  float* lh = ls + kM;                                                 // [2][128] each half's l
 
   const int g = p.g, P = kM / g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
@@ -179,14 +187,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(&s_full[k], 1);
-      mbar_init(&s_free[k], 4);
+      mbar_init(&s_free[k], 8);
     }
-    mbar_init(p_full, 4);
+    for (int k = 0; k < 4; ++k) mbar_init(&pbar[k], 2);
+    mbar_init(p_full, 8);
     mbar_init(p_free, 1);
     mbar_init(o_fin, 1);
-    mbar_init(q_ready, 4);
+    mbar_init(q_ready, 8);
     mbar_init(drain, 1);
-    mbar_init(cbar, 4);
+    mbar_init(cbar, 8);
     sh[0] = 0;
     fence_barrier_init();
   }
@@ -211,8 +220,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t tS[2] = {tmem, tmem + 128}, tO = tmem + 256;
 
-  if (warp == 0 || warp == 6) {
-    // ---------------------------------------------------------------- producers (K: warp 0, V: warp 6)
+  if (warp == 0 || warp == 10) {
+    // ---------------------------------------------------------------- producers (K: warp 0, V: warp 10)
     const bool isK = warp == 0;
     const int NS = isK ? kKStages : kVStages;
     uint64_t* full = isK ? k_full : v_full;
@@ -294,20 +303,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(drain, 0);
     }
   } else {
-    // ---------------------------------------------------------------- softmax warps (one row each)
-    const int row = 32 * (warp & 3) + lane;   // TMEM lane of this thread (warp w reads lanes 32(w%4)..)
+    // ---------------------------------------------------------------- softmax warps (two per row)
+    constexpr int HK = kKT / 2;               // keys per thread (a half of the tile)
+    const int quarter = warp & 3;             // warp w reads TMEM lanes 32(w % 4) .. 32(w % 4) + 31
+    const int half = (warp - 2) >> 2;         // warps 2-5: keys 0..63 of each tile, warps 6-9: 64..127
+    const int row = 32 * quarter + lane;
     const int j = row / P, t = row - (row / P) * P;
     const int h = hk * g + j, i = p0 + t;     // query head and position of the row
     const bool live = i < L;
     const int vis = min(i, L - 1);            // last key the row sees
     const size_t qrow = ((size_t)b * p.Hq + h) * p.T;
-    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-    // the Q row -> shared memory (K-major 128B swizzle: two 64-channel boxes), zero past L
+    const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
+    const int st = tid - 64;                  // 0..255 over the softmax warps
+    uint32_t pph = 0;                         // the pair barrier's phase
+    // this thread's half of the Q row (64 channels, one 128B-swizzled box) -> shared memory, zero past L
 #pragma unroll
-    for (int c = 0; c < kD / 8; ++c) {
+    for (int c = 0; c < 8; ++c) {
       uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (live) v = *reinterpret_cast<const uint4*>(p.q + (qrow + i) * kD + c * 8);
-      *reinterpret_cast<uint4*>(qs + (c >> 3) * kBoxB + sw128(row, c & 7)) = v;
+      if (live) v = *reinterpret_cast<const uint4*>(p.q + (qrow + i) * kD + half * 64 + c * 8);
+      *reinterpret_cast<uint4*>(qs + half * kBoxB + sw128(row, c)) = v;
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncwarp();
@@ -321,31 +335,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&s_full[k2], (n >> 1) & 1));
       if (!ok) break;
       tc_fence_after();
-      float x[kKT];
+      float x[HK];
 #pragma unroll
-      for (int c0 = 0; c0 < kKT; c0 += 32) tmem_ld32(tS[k2] + lane_base + c0, x + c0);
+      for (int c0 = 0; c0 < HK; c0 += 32) tmem_ld32(tS[k2] + lane_base + half * HK + c0, x + c0);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[k2]);   // S[k2] may be overwritten (tile n + 2)
-      // causal mask (key kt visible to row i iff kt <= min(i, L - 1)) where the tile needs one, and
-      // the row maximum of each block of the tile (raw scores: the scale is positive)
-      const int k0 = n * kKT;
-      const bool masked = k0 + kKT - 1 > vis;
-      if (masked) {
+      // causal mask (key kt visible to row i iff kt <= min(i, L - 1)) where the tile needs one; the
+      // maximum of this half (raw scores: the scale is positive)
+      const int k0 = n * kKT + half * HK;     // first key of this half
+      if (k0 + HK - 1 > vis) {
 #pragma unroll
-        for (int c = 0; c < kKT; ++c) x[c] = (k0 + c <= vis) ? x[c] : -INFINITY;
+        for (int c = 0; c < HK; ++c) x[c] = (k0 + c <= vis) ? x[c] : -INFINITY;
       }
-      float mx = -INFINITY;
+      float hm = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < HK; ++c) hm = fmaxf(hm, x[c]);
+      hm *= sl2;   // log2 domain
+      // the pair's tile maximum (double-buffered by tile parity: the partner has read tile n - 2's
+      // value before it arrived at tile n - 1's barrier)
+      xch[(k2 * 2 + half) * kM + row] = hm;
+      if (!warps_sync(&pbar[quarter], pph)) {
+        ok = false;
+        break;
+      }
+      const float hm2 = xch[(k2 * 2 + (half ^ 1)) * kM + row];
+      const float mx = fmaxf(hm, hm2);
+      // the row maximum of each block: a 64-key block is this half; a 128-key block is the tile
 #pragma unroll
       for (int sub = 0; sub < NBT; ++sub) {
-        float r = -INFINITY;
-#pragma unroll
-        for (int c = sub * BLK; c < (sub + 1) * BLK; ++c) r = fmaxf(r, x[c]);
-        r *= sl2;   // log2 domain
+        if (NBT == 2 ? sub != half : half != 0) continue;
         const int blk = n * NBT + sub;
-        if (live && blk * BLK <= i) rws[(size_t)blk * p.T + i] = r;
-        mx = fmaxf(mx, r);
+        if (live && blk * BLK <= i) rws[(size_t)blk * p.T + i] = NBT == 2 ? hm : mx;
       }
       // reference maximum: the first tile's, moved only when a tile exceeds it by more than kLazy;
       // then O (in TMEM, holding tiles 0..n-1) and l are rescaled
@@ -369,22 +391,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (__any_sync(0xffffffffu, move)) {
         tc_fence_after();
 #pragma unroll 1
-        for (int c0 = 0; c0 < kD; c0 += 32) {
+        for (int c0 = 0; c0 < kD / 2; c0 += 32) {
           float o[32];
-          tmem_ld32(tO + lane_base + c0, o);
+          tmem_ld32(tO + lane_base + half * (kD / 2) + c0, o);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] *= alpha;
-          tmem_st32(tO + lane_base + c0, o);
+          tmem_st32(tO + lane_base + half * (kD / 2) + c0, o);
         }
         tmem_wait_st();
         tc_fence_before();
       }
-      // P = exp2(s * scale - m_ref) (<= 2^kLazy; masked keys give 0) as bf16; l sums the same values
+      // P = exp2(s * scale - m_ref) (<= 2^kLazy; masked keys give 0) as bf16 into this half's box of
+      // the P tile; l sums the same values
       const float mu = m_ref == -INFINITY ? 0.f : m_ref;
       float sum = 0.f;
+      uint8_t* pbox = ps + half * kBoxB;
 #pragma unroll
-      for (int c = 0; c < kKT / 8; ++c) {
+      for (int c = 0; c < HK / 8; ++c) {
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -392,18 +416,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           sum += a + bb;
           w[e] = pack_bf16(a, bb);
         }
-        *reinterpret_cast<uint4*>(ps + (c >> 3) * kBoxB + sw128(row, c & 7)) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(pbox + sw128(row, c)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
       l += sum;
-      if (k0 + kKT > L) {
+      if (n * kKT + kKT > L) {
         // V rows past L may hold anything (even NaN): zero them so that P = 0 there gives 0.  Wait for
         // the tile's copy here too (its phase is at most one behind, as for the MMA issuer); whole
         // 128-byte rows, so the swizzle does not matter.
         ok = __all_sync(0xffffffffu, mbar_wait(&v_full[sv], (n / kVStages) & 1));
         if (!ok) break;
         uint8_t* vt = vring + (size_t)sv * kTileB;
-        const int r0 = max(0, L - k0), nchunk = (kKT - r0) * 8;   // 16-byte chunks per channel half
-        for (int e = tid - 64; e < 2 * nchunk; e += 128) {
+        const int r0 = max(0, L - n * kKT), nchunk = (kKT - r0) * 8;   // 16-byte chunks per channel half
+        for (int e = st; e < 2 * nchunk; e += 256) {
           const int hx = e / nchunk, rr = r0 + (e - hx * nchunk) / 8, cc = e & 7;
           *reinterpret_cast<uint4*>(vt + hx * kBoxB + rr * 128 + cc * 16) = make_uint4(0u, 0u, 0u, 0u);
         }
@@ -413,17 +437,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(p_full);
     }
     if (ok) {
-      // the last P.V (its own barrier: p_free may be two completions behind here), then O / l, the
-      // LSE, the row statistics
+      // the last P.V (its own barrier: p_free may be two completions behind here); from here on the
+      // P tile holds the row statistics
       ok = __all_sync(0xffffffffu, mbar_wait(o_fin, 0));
     }
     if (ok) {
+      lh[half * kM + row] = l;
+      ok = warps_sync(&pbar[quarter], pph);
+    }
+    if (ok) {
+      const float lt = lh[row] + lh[kM + row];   // the row's l (both halves; one reference maximum)
       tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
 #pragma unroll 1
-      for (int c0 = 0; c0 < kD; c0 += 32) {
+      for (int c0 = 0; c0 < kD / 2; c0 += 32) {
         float o[32];
-        tmem_ld32(tO + lane_base + c0, o);
+        tmem_ld32(tO + lane_base + half * (kD / 2) + c0, o);
         tmem_wait_ld();
         if (live) {
 #pragma unroll
@@ -433,28 +462,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             w.y = pack_bf16(o[e + 2] * inv, o[e + 3] * inv);
             w.z = pack_bf16(o[e + 4] * inv, o[e + 5] * inv);
             w.w = pack_bf16(o[e + 6] * inv, o[e + 7] * inv);
-            *reinterpret_cast<uint4*>(p.o + (qrow + i) * kD + c0 + e) = w;
+            *reinterpret_cast<uint4*>(p.o + (qrow + i) * kD + half * (kD / 2) + c0 + e) = w;
           }
         }
       }
-      if (live && p.lse) p.lse[qrow + i] = l > 0.f ? (m_ref + log2f(l)) * kLn2f : -INFINITY;
-      ms[row] = m_ref;
-      ls[row] = l;
+      if (half == 0) {
+        if (live && p.lse) p.lse[qrow + i] = lt > 0.f ? (m_ref + log2f(lt)) * kLn2f : -INFINITY;
+        ms[row] = m_ref;
+        ls[row] = lt;
+      }
     } else {
       if (lane == 0) report(p.err, SEER_DEVERR_TIMEOUT);
       sh[0] = 1;
     }
-    // ---- the targets: the four softmax warps meet (bounded; the block maxima the other warps
+    // ---- the targets: the eight softmax warps meet (bounded; the block maxima the other warps
     // wrote are read back through L2), then 8 threads per position, blocks strided by 8
     __threadfence();
     uint32_t cph = 0;
     const bool met = warps_sync(cbar, cph) && ok;
     if (!met && lane == 0) report(p.err, SEER_DEVERR_TIMEOUT);
-    const int st = tid - 64;   // 0..127
     const int sub = st & 7;
     float* gt_b = p.gt + ((size_t)b * p.Hkv + hk) * p.T * p.NB;
     const float* r_b = p.rmax + ((size_t)b * p.Hq + (size_t)hk * g) * p.NB * p.T;
-    for (int base = 0; base < P && met; base += 16) {
+    for (int base = 0; base < P && met; base += 32) {
       const int pi = base + st / 8;
       const int ip = p0 + pi;
       const bool lv = pi < P && ip < L;
