@@ -30,7 +30,10 @@
 //              P = exp2(s - m_ref) as bf16 into a shared tile (once the last
 //              P.V has read it),
 //              V rows past the sequence zeroed (the cache may hold NaN there),
-//              at the end O / l, the LSE and the targets
+//              at the end O / l, the LSE and the row's log2 normaliser m + log2 l
+// A second kernel (prefill_targets_kernel, launched behind it) forms the targets from the stored
+// block maxima and normalisers: bandwidth-bound work that would otherwise hold each CTA's tensor
+// cores idle at its end.
 // The reference maximum m_ref moves only when a tile's maximum exceeds it by
 // more than 8 (log2 units), so P stays <= 2^8 and O in TMEM is rescaled (ld,
 // scale, st) only then; l and the LSE use the same reference, so the results
@@ -159,15 +162,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* o_fin = p_free + 1;      // the last P.V done (single use)
   uint64_t* q_ready = o_fin + 1;
   uint64_t* drain = q_ready + 1;
-  uint64_t* cbar = drain + 1;
-  uint64_t* pbar = cbar + 1;         // [4] the two warps of each TMEM lane quarter
+  uint64_t* pbar = drain + 1;        // [4] the two warps of each TMEM lane quarter
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pbar + 4);
   volatile int* sh = reinterpret_cast<volatile int*>(tmem_slot + 1);   // [0] abort
   float* xch = reinterpret_cast<float*>(ps + kTileB + 256);            // [tile & 1][half][row] tile maxima
-  // after the last P.V the P tile is free: the row statistics live there
-  float* ms = reinterpret_cast<float*>(ps);                            // [128] final m_ref per row
-  float* ls = ms + kM;                                                 // [128] final l per row
-  float* lh = ls + kM;                                                 // [2][128] each half's l
+  // after the last P.V the P tile is free: each half's l meets there
+  float* lh = reinterpret_cast<float*>(ps);                            // [2][128]
 
   const int g = p.g, P = kM / g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
@@ -195,7 +195,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(o_fin, 1);
     mbar_init(q_ready, 8);
     mbar_init(drain, 1);
-    mbar_init(cbar, 8);
     sh[0] = 0;
     fence_barrier_init();
   }
@@ -438,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok) {
       // the last P.V (its own barrier: p_free may be two completions behind here); from here on the
-      // P tile holds the row statistics
+      // P tile is free for the two halves' l
       ok = __all_sync(0xffffffffu, mbar_wait(o_fin, 0));
     }
     if (ok) {
@@ -466,68 +465,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (half == 0) {
-        if (live && p.lse) p.lse[qrow + i] = lt > 0.f ? (m_ref + log2f(lt)) * kLn2f : -INFINITY;
-        ms[row] = m_ref;
-        ls[row] = lt;
+      if (half == 0 && live) {
+        const float c = lt > 0.f ? m_ref + log2f(lt) : -INFINITY;   // log2 of the row's normaliser
+        if (p.lse) p.lse[qrow + i] = c * kLn2f;
+        p.rnorm[qrow + i] = c;
       }
     } else {
       if (lane == 0) report(p.err, SEER_DEVERR_TIMEOUT);
       sh[0] = 1;
-    }
-    // ---- the targets: the eight softmax warps meet (bounded; the block maxima the other warps
-    // wrote are read back through L2), then 8 threads per position, blocks strided by 8
-    __threadfence();
-    uint32_t cph = 0;
-    const bool met = warps_sync(cbar, cph) && ok;
-    if (!met && lane == 0) report(p.err, SEER_DEVERR_TIMEOUT);
-    const int sub = st & 7;
-    float* gt_b = p.gt + ((size_t)b * p.Hkv + hk) * p.T * p.NB;
-    const float* r_b = p.rmax + ((size_t)b * p.Hq + (size_t)hk * g) * p.NB * p.T;
-    for (int base = 0; base < P && met; base += 32) {
-      const int pi = base + st / 8;
-      const int ip = p0 + pi;
-      const bool lv = pi < P && ip < L;
-      const int nb_i = lv ? ip / BLK + 1 : 0;   // blocks with a key visible to position ip
-      // a block's score, four blocks at a time with every load issued before any use (two passes:
-      // the sum, then the normalised stores)
-      auto scores4 = [&](int n0, float (&v)[4]) {
-        float r[4][kMaxGroup];
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-#pragma unroll
-          for (int jj = 0; jj < kMaxGroup; ++jj)
-            r[u][jj] = (jj < g && n0 + 8 * u < nb_i) ? __ldcg(r_b + ((size_t)jj * p.NB + n0 + 8 * u) * p.T + ip)
-                                                      : -INFINITY;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          v[u] = 0.f;
-#pragma unroll
-          for (int jj = 0; jj < kMaxGroup; ++jj)
-            if (jj < g && n0 + 8 * u < nb_i) v[u] = fmaxf(v[u], exp2f(r[u][jj] - ms[jj * P + pi]) / ls[jj * P + pi]);
-        }
-      };
-      float sum = 0.f;
-      for (int n0 = sub; n0 < nb_i; n0 += 32) {
-        float v[4];
-        scores4(n0, v);
-        sum += (v[0] + v[1]) + (v[2] + v[3]);
-      }
-      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-      sum += __shfl_xor_sync(0xffffffffu, sum, 4);
-      const float inv = sum > 0.f ? 1.f / sum : 0.f;
-      if (lv) {
-        for (int n0 = sub; n0 < nb_i; n0 += 32) {
-          float v[4];
-          scores4(n0, v);
-#pragma unroll
-          for (int u = 0; u < 4; ++u)
-            if (n0 + 8 * u < nb_i) gt_b[(size_t)ip * p.NB + n0 + 8 * u] = v[u] * inv;
-        }
-        for (int nn = (nb_i & ~7) + sub; nn < p.NB; nn += 8)
-          if (nn >= nb_i) gt_b[(size_t)ip * p.NB + nn] = 0.f;
-      }
     }
   }
   tc_fence_before();
@@ -535,6 +480,112 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+  }
+}
+
+// ---------------------------------------------------------------- the targets
+// One CTA per (32 positions, kv head, sequence), 8 warps; lane t is position i0 + t while the
+// scores are formed (the row maxima are position-contiguous per (head, block): 128-byte loads),
+// and the block index while the rows are written (block-contiguous per position: 128-byte
+// stores).  Score of block n for position i: max over the group's heads j of exp2(r_j - c_j)
+// (c = m + log2 l, the row's final log2 normaliser), for the blocks holding a key at or before i,
+// normalised to sum to 1; 0 for the other blocks.  Blocks are taken kTgChunk at a time through
+// shared memory; with more blocks than one chunk the sum is a first pass of its own and each
+// chunk's scores are formed again (from L2: the CTA's maxima are a few hundred KB at most).
+constexpr int kTgPos = 32;
+constexpr int kTgWarps = 8;
+constexpr int kTgChunk = 256;
+
+template <int BLK>
+__global__ void __launch_bounds__(kTgWarps * 32)
+    prefill_targets_kernel(const __grid_constant__ PrefillParams p) {
+  __shared__ float vals[kTgChunk][kTgPos + 1];
+  __shared__ float psum[kTgWarps][kTgPos];
+  __shared__ float inv_s[kTgPos];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.z, hk = blockIdx.y, i0 = blockIdx.x * kTgPos;
+  const int g = p.g;
+  pdl_wait();   // the forward's row maxima and normalisers are complete
+  pdl_trigger();
+  const int L = min(max(p.seqlens[b], 0), min(p.T, p.kcap));
+  if (i0 >= L) return;
+  const int i = i0 + lane;
+  const bool live = i < L;
+  const int nb_i = live ? i / BLK + 1 : 0;                 // blocks with a key visible to position i
+  const int nb_max = (min(i0 + kTgPos, L) - 1) / BLK + 1;  // the largest nb_i of the CTA
+  const float* r_b = p.rmax + ((size_t)b * p.Hq + (size_t)hk * g) * p.NB * p.T;
+  float c[kMaxGroup];
+#pragma unroll
+  for (int j = 0; j < kMaxGroup; ++j)
+    c[j] = (j < g && live) ? __ldg(p.rnorm + ((size_t)b * p.Hq + (size_t)hk * g + j) * p.T + i) : 0.f;
+  // scores of blocks n0 + 8u (u = 0..3), every load issued before any use
+  auto score4 = [&](int n0, float (&v)[4]) {
+    float r[4][kMaxGroup];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int j = 0; j < kMaxGroup; ++j)
+        r[u][j] = (j < g && n0 + kTgWarps * u < nb_i) ? __ldcg(r_b + ((size_t)j * p.NB + n0 + kTgWarps * u) * p.T + i)
+                                                       : -INFINITY;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      v[u] = 0.f;
+#pragma unroll
+      for (int j = 0; j < kMaxGroup; ++j)
+        if (j < g && n0 + kTgWarps * u < nb_i) v[u] = fmaxf(v[u], exp2f(r[u][j] - c[j]));
+    }
+  };
+  // chunk [n_lo, n_hi): scores into vals (and into the sum when `add`)
+  auto fill = [&](int n_lo, int n_hi, bool add, float& part) {
+    for (int n0 = n_lo + warp; n0 < n_hi; n0 += 4 * kTgWarps) {
+      float v[4];
+      score4(n0, v);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int n = n0 + kTgWarps * u;
+        if (n < n_hi) {
+          vals[n - n_lo][lane] = v[u];
+          if (add) part += v[u];
+        }
+      }
+    }
+  };
+  const bool one = nb_max <= kTgChunk;
+  float part = 0.f;
+  if (one) {
+    fill(0, nb_max, true, part);
+  } else {
+    for (int n0 = warp; n0 < nb_max; n0 += 4 * kTgWarps) {
+      float v[4];
+      score4(n0, v);
+      part += (v[0] + v[1]) + (v[2] + v[3]);   // blocks past nb_i score 0
+    }
+  }
+  psum[warp][lane] = part;
+  __syncthreads();
+  if (warp == 0) {
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < kTgWarps; ++w) s += psum[w][lane];
+    inv_s[lane] = s > 0.f ? 1.f / s : 0.f;
+  }
+  __syncthreads();
+  float* gt_b = p.gt + ((size_t)b * p.Hkv + hk) * p.T * p.NB;
+  const int npos = min(kTgPos, L - i0);
+  for (int n_lo = 0; n_lo < p.NB; n_lo += kTgChunk) {
+    const int n_hi = min(p.NB, n_lo + kTgChunk);
+    if (!one && n_lo < nb_max) {
+      float unused = 0.f;
+      fill(n_lo, min(n_hi, nb_max), false, unused);
+      __syncthreads();
+    }
+    for (int t = warp; t < npos; t += kTgWarps) {
+      const int nb_t = (i0 + t) / BLK + 1;
+      const float inv = inv_s[t];
+      float* row = gt_b + (size_t)(i0 + t) * p.NB;
+      for (int n = n_lo + lane; n < n_hi; n += 32) __stcs(row + n, n < nb_t ? vals[n - n_lo][t] * inv : 0.f);
+    }
+    if (!one) __syncthreads();   // vals is refilled for the next chunk
   }
 }
 
@@ -547,7 +598,10 @@ cudaError_t launch_tc_t(const CUtensorMap& tk, const CUtensorMap& tv, const Pref
   if (e != cudaSuccess) return e;
   const int P = kM / p.g;
   const dim3 grid((max_len + P - 1) / P, p.Hkv, p.B);
-  return launch_pdl(kern, grid, dim3(kThreads), kSmem, st, tk, tv, p);
+  e = launch_pdl(kern, grid, dim3(kThreads), kSmem, st, tk, tv, p);
+  if (e != cudaSuccess) return e;
+  const dim3 tgrid((max_len + kTgPos - 1) / kTgPos, p.Hkv, p.B);
+  return launch_pdl(prefill_targets_kernel<BLK>, tgrid, dim3(kTgWarps * 32), 0, st, p);
 }
 
 }  // namespace

@@ -346,7 +346,7 @@ seer_status seer_kcomp_update(const seer_dims_t* dims, const seer_kv_t* k_nope, 
 
 size_t seer_prefill_gt_workspace_bytes(const seer_dims_t* dims, int32_t max_len) {
   if (check_dims(dims) != SEER_OK || max_len < 1) return 0;
-  return (size_t)dims->batch * dims->num_q_heads * dims->max_blocks * (size_t)max_len * sizeof(float);
+  return (size_t)dims->batch * dims->num_q_heads * (dims->max_blocks + (size_t)1) * (size_t)max_len * sizeof(float);
 }
 
 seer_status seer_prefill_gt(const seer_dims_t* dims, const void* q, int32_t max_len, const seer_kv_t* k,
@@ -379,6 +379,7 @@ seer_status seer_prefill_gt(const seer_dims_t* dims, const void* q, int32_t max_
   p.lse = lse_out;
   p.gt = gt;
   p.rmax = static_cast<float*>(workspace);
+  p.rnorm = p.rmax + (size_t)dims->batch * dims->num_q_heads * dims->max_blocks * (size_t)max_len;
   p.seqlens = seqlens;
   p.B = dims->batch;
   p.Hq = dims->num_q_heads;

@@ -102,6 +102,7 @@ struct PrefillParams {
   float* lse;              // [B, Hq, T] or null
   float* gt;               // [B, Hkv, T, NB]
   float* rmax;             // workspace [B, Hq, NB, T]: each row's tile maxima (log2 domain)
+  float* rnorm;            // workspace [B, Hq, T]: each row's final m + log2(l) (tcgen05 path)
   const int32_t* seqlens;  // [B]
   int32_t k_perm[3], v_perm[3];
   int32_t B, Hq, Hkv, g, NB, T;

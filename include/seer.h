@@ -404,10 +404,14 @@ seer_status seer_gate_truth(const seer_dims_t* dims, const void* q, const seer_k
  *   lse_out    device fp32 [B, Hq, max_len] or NULL
  *   gt         device fp32 [B, Hkv, max_len, max_blocks]
  *   workspace  device, >= seer_prefill_gt_workspace_bytes(dims, max_len) bytes (each query row's
- *              per-block score maxima, fp32 [B, Hq, max_blocks, max_len]), 16-byte aligned
+ *              per-block score maxima, fp32 [B, Hq, max_blocks, max_len], then each row's log2
+ *              normaliser, fp32 [B, Hq, max_len]), 16-byte aligned
  *   err_word   device int32 or NULL (SEER_DEVERR_* bits ORed in)
- * One CTA per (16 * floor(8 / g) positions, KV head, sequence); the group's query heads share
- * every K/V tile.  Paged caches: SEER_ERR_UNSUPPORTED.
+ * head_dim 128 with g in {1, 2, 4, 8}: the tcgen05 / TMEM forward (one CTA per 128 / g positions of
+ * the group's g heads, KV head, sequence), then a bandwidth-bound kernel forming the targets (two
+ * launches).  Other shapes: the warp-level mma forward, one CTA per (16 * floor(8 / g) positions,
+ * KV head, sequence), targets formed in its epilogue.  The group's query heads share every K/V
+ * tile.  Paged caches: SEER_ERR_UNSUPPORTED.
  */
 size_t seer_prefill_gt_workspace_bytes(const seer_dims_t* dims, int32_t max_len);
 seer_status seer_prefill_gt(const seer_dims_t* dims, const void* q, int32_t max_len,

@@ -185,7 +185,7 @@ def test_prefill_gt_validation(lib, S):
     d = _dims(S)
     k = _kv(S)
     n = lib.seer_prefill_gt_workspace_bytes(ctypes.byref(d), 4096)
-    assert n == 8 * 32 * d.max_blocks * 4096 * 4
+    assert n == 8 * 32 * (d.max_blocks + 1) * 4096 * 4   # block maxima, then one normaliser per row
     assert lib.seer_prefill_gt_workspace_bytes(ctypes.byref(d), 0) == 0
     assert lib.seer_prefill_gt(ctypes.byref(d), None, 64, ctypes.byref(k), ctypes.byref(k), P, P, None, P, P,
                                1 << 30, None, None) == 1

@@ -88,3 +88,43 @@ def test_prefill_8k_sampled():
             bad = np.abs(row[:len(ref)] - ref) > GT_REL_PREFILL * ref + 1e-7
             assert not bad.any(), f"h{h} i{i}: {int(bad.sum())} target entries off"
             assert np.all(row[len(ref):] == 0.0)
+
+
+@pytest.mark.parametrize("blk,g,L,T", [(64, 4, 20001, 20032), (128, 8, 33001, 33024)])
+def test_prefill_long_sampled(blk, g, L, T):
+    """Sequences with more than 256 blocks (the targets are then formed in several block chunks, the
+    sum first), a ragged length and rows past it that must stay untouched; sampled rows against the
+    oracle, one position at a time, at block and chunk boundaries."""
+    B, Hkv, d = 1, 1, 128
+    Hq, NB = g * Hkv, -(-T // blk)
+    rng = np.random.default_rng(77 + blk)
+
+    def bits(shape):
+        x = torch.from_numpy(rng.standard_normal(shape, dtype=np.float32)).to(torch.bfloat16)
+        return x.view(torch.int16).numpy().view(np.uint16)
+
+    q, k, v = bits((B, Hq, T, d)), bits((B, Hkv, T, d)), bits((B, Hkv, T, d))
+    sh = S.Shape(B, Hq, Hkv, d, d, blk, NB)
+    out = torch.empty(B, Hq, T, d, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(B, Hq, T, dtype=torch.float32, device="cuda")
+    gt = torch.full((B, Hkv, T, NB), 7.0, dtype=torch.float32, device="cuda")
+    ws = torch.empty(S.prefill_gt_workspace_bytes(sh, T), dtype=torch.uint8, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    S.prefill_gt(sh, to_dev_bf16(q), S.KVCache.contiguous(to_dev_bf16(k)), S.KVCache.contiguous(to_dev_bf16(v)),
+                 torch.full((B,), L, dtype=torch.int32, device="cuda"), out, gt, ws, lse=lse, err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert torch.all(gt[0, 0, L:] == 7.0), "rows past the length were written"
+    scale = 1.0 / math.sqrt(d)
+    kk, vv = f64(k[0, 0]), f64(v[0, 0])
+    for i in (0, 256 * blk - 1, 256 * blk, 256 * blk + 31, L - 33, L - 1):
+        qi = f64(q[0, :, i])
+        ro, rl = O.attend(qi, kk, vv, np.arange(i + 1), scale)
+        check_attention(f64(bf16_bits(out[0, :, i])), ro, f"i{i}")
+        check_lse(lse[0, :, i].cpu().numpy().astype(np.float64), rl, f"i{i}")
+        ref = O.decode_ground_truth(qi, kk, i + 1, blk, scale)
+        row = gt[0, 0, i].cpu().numpy().astype(np.float64)
+        bad = np.abs(row[:len(ref)] - ref) > GT_REL_PREFILL * ref + 1e-7
+        assert not bad.any(), f"i{i}: {int(bad.sum())} target entries off"
+        assert np.all(row[len(ref):] == 0.0)
+        assert abs(row.sum() - 1.0) <= 1e-4
