@@ -447,7 +447,7 @@ def threshold_loop_row(S, dev, stream, peak, workers, steps=256):
     """The 256-step decode loop with threshold selection (Qwen3-8B-shaped heads, B = 32, start
     context 16384): one token per step, the K Compression Cache filling every 64 steps, per-head
     gate temperatures set at step 0 so that the median sequence of head h selects f_h of the blocks
-    (f_h spaced 5 %..24 %), tau = 1/512.  The whole loop is one CUDA graph (the fill counts reset at
+    (f_h spaced 7 %..20 %), tau = 1/512.  The whole loop is one CUDA graph (the fill counts reset at
     its start), so a step's time is the loop's over its steps; the realised spread of selected
     fractions is recorded per step."""
     import torch
@@ -466,7 +466,7 @@ def threshold_loop_row(S, dev, stream, peak, workers, steps=256):
     S.gate_score(shape, _up(make_step_query(cfg, 0), dev), _up(inp.w_q, dev), kc, L1, lg)
     nfull = (int(inp.seqlens[0]) + 1) // blk
     z = lg[:, :, :nfull].double().cpu().numpy()
-    fr = np.linspace(0.05, 0.24, Hkv)
+    fr = np.linspace(0.07, 0.20, Hkv)
 
     def count(c, zz):
         e = np.exp(c * (zz - zz.max()))

@@ -16,29 +16,33 @@
 // One CTA per (128 query rows, kv head, sequence): the g heads of the group x
 // 128/g consecutive positions, row r = head (r / P) at position p0 + (r % P).
 // Key tiles of 128 keys (one or two blocks).
-//   warps 0, 10 producers: K tiles (two-stage ring, a stage freed once S has
+//   warps 0, 10 producers: K tiles (three-stage ring, a stage freed once S has
 //              read it) and V tiles (two stages, freed once P.V has read
 //              them) by TMA (128-byte swizzle, boxes of 64 channels x b keys)
 //   warp 1     allocates TMEM; one lane issues the MMAs: S_n = Q K_n^T into
-//              TMEM S[n % 2] (M = 128 rows, N = 128 keys, K = d), then
-//              O += P_{n-1} V_{n-1} into TMEM O (N = d, K = 128 keys), each
-//              group closed by a commit to an mbarrier
+//              TMEM S[n % 2] (M = 128 rows, N = 128 keys, K = d; both
+//              operands in shared memory), then O += P_{n-1} V_{n-1} into TMEM O
+//              (N = d, K = 128 keys; P read from TMEM P[(n-1) % 2], V from
+//              shared memory), each group closed by a commit to an mbarrier
 //   warps 2-9  two threads per row (the row's TMEM lane; one thread per half of
 //              the 128 keys, the pair exchanging the tile's maxima through
 //              shared memory): S by tcgen05.ld, causal mask, the row maximum of
 //              each block (stored for the targets),
-//              P = exp2(s - m_ref) as bf16 into a shared tile (once the last
-//              P.V has read it),
+//              P = exp2(s - m_ref) as bf16 pairs into TMEM P[n % 2] by
+//              tcgen05.st (once the P.V of tile n - 2 has read that buffer, so
+//              tile n's exponentials overlap the P.V of tile n - 1),
 //              V rows past the sequence zeroed (the cache may hold NaN there),
 //              at the end O / l, the LSE and the row's log2 normaliser m + log2 l
+// TMEM columns: S[0] 0-127, S[1] 128-255, O 256-383, P[0] 384-447, P[1] 448-511.
 // A second kernel (prefill_targets_kernel, launched behind it) forms the targets from the stored
 // block maxima and normalisers: bandwidth-bound work that would otherwise hold each CTA's tensor
 // cores idle at its end.
 // The reference maximum m_ref moves only when a tile's maximum exceeds it by
 // more than 8 (log2 units), so P stays <= 2^8 and O in TMEM is rescaled (ld,
-// scale, st) only then; l and the LSE use the same reference, so the results
-// are those of the exact online softmax (l sums the probabilities before their
-// rounding to bf16 for the P.V product).  All waits are bounded.
+// scale, st; after the P.V of the previous tile has landed) only then; l and
+// the LSE use the same reference, so the results are those of the exact online
+// softmax (l sums the probabilities before their rounding to bf16 for the P.V
+// product).  All waits are bounded.
 #include "seer_device.cuh"
 #include "seer_internal.h"
 
@@ -50,14 +54,15 @@ constexpr int kD = 128;                 // head_dim of this kernel
 constexpr int kM = 128;                 // query rows per CTA
 constexpr int kKT = 128;                // keys per tile
 constexpr int kBoxB = kM * 128;         // bytes of a 128-row x 64-channel (or 64-key) 128B-swizzled box
-constexpr int kTileB = 2 * kBoxB;       // 32 KB: a K, V, Q or P tile (two boxes)
-constexpr int kKStages = 2;
+constexpr int kTileB = 2 * kBoxB;       // 32 KB: a K, V or Q tile (two boxes)
+constexpr int kKStages = 3;
 constexpr int kVStages = 2;
 constexpr int kThreads = 11 * 32;
-constexpr uint32_t kTmemCols = 512;     // S[0] 0..127, S[1] 128..255, O 256..383
+constexpr uint32_t kTmemCols = 512;     // S[0] 0..127, S[1] 128..255, O 256..383, P[0] 384..447, P[1] 448..511
 constexpr float kLazy = 8.f;            // m_ref moves when a tile maximum exceeds it by more than this
-constexpr size_t kSmem = 1024 + kTileB /* Q */ + (size_t)(kKStages + kVStages) * kTileB /* K, V */ + kTileB /* P */ +
-                         256 /* barriers */ + 2 * 2 * kM * 4 /* the pairs' tile maxima, two tiles */;
+constexpr size_t kSmem = 1024 + kTileB /* Q */ + (size_t)(kKStages + kVStages) * kTileB /* K, V */ +
+                         256 /* barriers */ + 2 * 2 * kM * 4 /* the pairs' tile maxima, two tiles */ +
+                         2 * kM * 4 /* each half's l */;
 
 static_assert(kSmem <= 227 * 1024, "dynamic shared memory above the per-CTA limit");
 
@@ -87,6 +92,15 @@ __device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t da, uint64_t 
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
       "l"(da), "l"(db), "r"(idesc), "r"(acc));
 }
+// the same with A (M rows x 16 K elements, two bf16 per 32-bit column, the lower K index in the low
+// half) read from tensor memory at `tmem_a`
+__device__ __forceinline__ void umma_f16_ta(uint32_t tmem_d, uint32_t tmem_a, uint64_t db, uint32_t idesc,
+                                            uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(db), "r"(idesc), "r"(acc));
+}
 // arrive on `bar` once every MMA this thread issued so far has completed
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -108,6 +122,15 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
       : "r"(taddr));
 #pragma unroll
   for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+}
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
+      "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+      "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31]));
 }
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
   asm volatile(
@@ -150,24 +173,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* qs = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* kring = qs + kTileB;                        // [kKStages] K tiles
   uint8_t* vring = kring + (size_t)kKStages * kTileB;  // [kVStages] V tiles
-  uint8_t* ps = vring + (size_t)kVStages * kTileB;     // P tile
-  uint64_t* k_full = reinterpret_cast<uint64_t*>(ps + kTileB);
+  uint64_t* k_full = reinterpret_cast<uint64_t*>(vring + (size_t)kVStages * kTileB);
   uint64_t* k_empty = k_full + kKStages;
   uint64_t* v_full = k_empty + kKStages;
   uint64_t* v_empty = v_full + kVStages;
   uint64_t* s_full = v_empty + kVStages;   // [2]
   uint64_t* s_free = s_full + 2;           // [2]
-  uint64_t* p_full = s_free + 2;
-  uint64_t* p_free = p_full + 1;     // one completion per P.V (P read; tiles 0..m in O)
-  uint64_t* o_fin = p_free + 1;      // the last P.V done (single use)
+  uint64_t* p_full = s_free + 2;     // [2] P[k] written (tile n, k = n % 2)
+  uint64_t* p_free = p_full + 2;     // [2] one completion per P.V of P[k] (P[k] read; tiles 0..m in O)
+  uint64_t* o_fin = p_free + 2;      // the last P.V done (single use)
   uint64_t* q_ready = o_fin + 1;
   uint64_t* drain = q_ready + 1;
   uint64_t* pbar = drain + 1;        // [4] the two warps of each TMEM lane quarter
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pbar + 4);
   volatile int* sh = reinterpret_cast<volatile int*>(tmem_slot + 1);   // [0] abort
-  float* xch = reinterpret_cast<float*>(ps + kTileB + 256);            // [tile & 1][half][row] tile maxima
-  // after the last P.V the P tile is free: each half's l meets there
-  float* lh = reinterpret_cast<float*>(ps);                            // [2][128]
+  float* xch = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(k_full) + 256);   // [tile & 1][half][row]
+  float* lh = xch + 2 * 2 * kM;                                                      // [half][row] l
 
   const int g = p.g, P = kM / g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
@@ -190,8 +211,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s_free[k], 8);
     }
     for (int k = 0; k < 4; ++k) mbar_init(&pbar[k], 2);
-    mbar_init(p_full, 8);
-    mbar_init(p_free, 1);
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(&p_full[k], 8);
+      mbar_init(&p_free[k], 1);
+    }
     mbar_init(o_fin, 1);
     mbar_init(q_ready, 8);
     mbar_init(drain, 1);
@@ -217,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS[2] = {tmem, tmem + 128}, tO = tmem + 256;
+  const uint32_t tS[2] = {tmem, tmem + 128}, tO = tmem + 256, tP[2] = {tmem + 384, tmem + 448};
 
   if (warp == 0 || warp == 10) {
     // ---------------------------------------------------------------- producers (K: warp 0, V: warp 10)
@@ -263,18 +286,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t qa = smem_u32(qs);
       bool ok = mbar_wait(q_ready, 0);
       auto issue_pv = [&](int m) {
-        const int sv = m % kVStages;
-        ok = ok && mbar_wait(p_full, m & 1) && mbar_wait(&v_full[sv], (m / kVStages) & 1);
+        const int sv = m % kVStages, pb = m & 1;
+        ok = ok && mbar_wait(&p_full[pb], (m >> 1) & 1) && mbar_wait(&v_full[sv], (m / kVStages) & 1);
         if (!ok) return;
         tc_fence_after();
-        const uint32_t pa = smem_u32(ps);
         const uint32_t vb = smem_u32(vring + (size_t)sv * kTileB);
 #pragma unroll
         for (int kk = 0; kk < kKT / 16; ++kk)
-          umma_f16(tO, desc_kmajor(pa + (kk >> 2) * kBoxB + (kk & 3) * 32), desc_mnmajor(vb + kk * 2048, kBoxB),
-                   id_o, (m > 0 || kk > 0) ? 1u : 0u);
+          umma_f16_ta(tO, tP[pb] + kk * 8, desc_mnmajor(vb + kk * 2048, kBoxB), id_o, (m > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&v_empty[sv]);
-        umma_commit(p_free);
+        umma_commit(&p_free[pb]);
       };
       for (int n = 0; n < nt && ok; ++n) {
         const int sk = n % kKStages, k2 = n & 1;
@@ -380,14 +401,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         move = true;
       }
       l *= alpha;
-      // the P.V of tile n - 1 (the n-th completion of p_free; S_n's commit, observed above, came after
-      // the P.V of tile n - 2, so the barrier is at most one completion behind and a parity wait is
-      // exact) has read the P tile and added tile n - 1 to O
-      if (n > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(p_free, (n - 1) & 1));
+      // P[n % 2] is free once the P.V of tile n - 2 has read it (that buffer's (n / 2)-th completion;
+      // the next one needs P of tile n, not yet written, so a parity wait is exact).  A rescale of O
+      // waits for the P.V of tile n - 1 as well (O then holds tiles 0..n-1 and nothing adds to it).
+      const int pb = n & 1;
+      if (n > 1) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&p_free[pb], ((n >> 1) - 1) & 1));
         if (!ok) break;
       }
       if (__any_sync(0xffffffffu, move)) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&p_free[pb ^ 1], ((n - 1) >> 1) & 1));
+        if (!ok) break;
         tc_fence_after();
 #pragma unroll 1
         for (int c0 = 0; c0 < kD / 2; c0 += 32) {
@@ -401,21 +425,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
       }
-      // P = exp2(s * scale - m_ref) (<= 2^kLazy; masked keys give 0) as bf16 into this half's box of
-      // the P tile; l sums the same values
+      // P = exp2(s * scale - m_ref) (<= 2^kLazy; masked keys give 0) as bf16 pairs into this half's
+      // 32 columns of P[n % 2] in TMEM; l sums the same values
       const float mu = m_ref == -INFINITY ? 0.f : m_ref;
       float sum = 0.f;
-      uint8_t* pbox = ps + half * kBoxB;
+      {
+        uint32_t w[HK / 2];
 #pragma unroll
-      for (int c = 0; c < HK / 8; ++c) {
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float a = ex2(fmaf(x[8 * c + 2 * e], sl2, -mu)), bb = ex2(fmaf(x[8 * c + 2 * e + 1], sl2, -mu));
+        for (int e = 0; e < HK / 2; ++e) {
+          const float a = ex2(fmaf(x[2 * e], sl2, -mu)), bb = ex2(fmaf(x[2 * e + 1], sl2, -mu));
           sum += a + bb;
           w[e] = pack_bf16(a, bb);
         }
-        *reinterpret_cast<uint4*>(pbox + sw128(row, c)) = make_uint4(w[0], w[1], w[2], w[3]);
+        tmem_st32u(tP[pb] + lane_base + half * (HK / 2), w);
       }
       l += sum;
       if (n * kKT + kKT > L) {
@@ -430,14 +452,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int hx = e / nchunk, rr = r0 + (e - hx * nchunk) / 8, cc = e & 7;
           *reinterpret_cast<uint4*>(vt + hx * kBoxB + rr * 128 + cc * 16) = make_uint4(0u, 0u, 0u, 0u);
         }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tmem_wait_st();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[pb]);
     }
     if (ok) {
-      // the last P.V (its own barrier: p_free may be two completions behind here); from here on the
-      // P tile is free for the two halves' l
+      // the last P.V (its own barrier: p_free may be two completions behind here)
       ok = __all_sync(0xffffffffu, mbar_wait(o_fin, 0));
     }
     if (ok) {

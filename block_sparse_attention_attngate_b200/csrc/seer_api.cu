@@ -8,6 +8,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <string>
 
@@ -310,6 +311,29 @@ extern "C" {
 const char* seer_last_error(void) { return g_err.c_str(); }
 
 const char* seer_version(void) { return "libseer 0.1 (sm_100a)"; }
+
+// process-wide bound and debug switch of the sparse decode's waits, read at each launch
+namespace {
+std::atomic<long long> g_wait_limit{seer::kWaitLimitCycles};
+std::atomic<int32_t> g_debug{0};
+}  // namespace
+
+seer_status seer_set_wait_limit(int64_t cycles) {
+  if (cycles == 0) cycles = seer::kWaitLimitCycles;
+  if (cycles < SEER_WAIT_LIMIT_MIN || cycles > SEER_WAIT_LIMIT_MAX)
+    return fail(SEER_ERR_INVALID_ARG, "wait limit %lld cycles outside [%lld, %lld] (0 = the default)",
+                (long long)cycles, (long long)SEER_WAIT_LIMIT_MIN, (long long)SEER_WAIT_LIMIT_MAX);
+  g_wait_limit.store(cycles);
+  return SEER_OK;
+}
+
+int64_t seer_get_wait_limit(void) { return g_wait_limit.load(); }
+
+seer_status seer_set_debug_flags(int32_t flags) {
+  if (flags & ~SEER_DEBUG_STARVE_COPIES) return fail(SEER_ERR_INVALID_ARG, "unknown debug flags 0x%x", flags);
+  g_debug.store(flags);
+  return SEER_OK;
+}
 
 seer_status seer_kcomp_update(const seer_dims_t* dims, const seer_kv_t* k_nope, const int32_t* seqlens,
                               int32_t* valid_blocks, const void* w_k, void* kcomp, void* stream) {
@@ -642,6 +666,7 @@ seer_status seer_decode_step(const seer_dims_t* dims, const seer_kv_t* k_nope, c
   if (L.ctas < grid) return fail(SEER_ERR_UNSUPPORTED, "fused step grid %d above the decode's %d", grid, L.ctas);
   sp.d = L.p;
   sp.d.ready = reinterpret_cast<int32_t*>(ws);
+  sp.d.starve = 0;   // the debug switch covers the two-launch decode only
   sp.pl.k.err = err_word;
   cudaError_t e = seer::launch_decode_step(L.tk, L.tv, sp, dims->head_dim, dims->block_size, dims->gate_dim, grid,
                                            static_cast<cudaStream_t>(stream));
@@ -739,6 +764,8 @@ seer_status prepare_sparse_decode(const seer_dims_t* dims, const void* q, const 
   p.lse_out = lse_out;
   p.err = err_word;
   p.ready = nullptr;
+  p.wait_limit = g_wait_limit.load();
+  p.starve = (g_debug.load() & SEER_DEBUG_STARVE_COPIES) ? 1 : 0;
   L->D = dims->head_dim;
   L->BLK = dims->block_size;
   L->ctas = ctas;

@@ -45,6 +45,8 @@ cudaError_t ensure_smem_limit(Kernel kern, int bytes, std::atomic<uint64_t>& don
 }
 
 
+// ~1 s at 2 GHz: a wait that runs this long means a copy never landed (the default bound).
+constexpr long long kWaitLimitCycles = 2000000000LL;
 constexpr int kMaxGroup = 8;        // query heads per KV head
 constexpr int kMaxBlocksRow = 8192; // max_blocks limit (selection keeps a row in shared memory)
 constexpr int kMaxDecodeB = 4096;   // decode keeps the sequence lengths in shared memory
@@ -177,6 +179,8 @@ struct DecodeParams {
   float* lse_out;           // [B, Hq] or null
   int32_t* err;
   int32_t* ready;           // fused step: [B, Hkv] per-row list-ready flags (zero between calls); else null
+  long long wait_limit;     // bound of every copy / hand-off wait, in SM cycles
+  int32_t starve;           // debug: the producer issues no copy (every first wait runs out); 0 in use
 };
 cudaError_t launch_sparse_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                                  int D, int BLK, int grid_flat, cudaStream_t s);

@@ -496,7 +496,7 @@ __device__ __forceinline__ void decode_body(const CUtensorMap* tmK, const CUtens
     // is published (and merged, if it arrives last) here.
     const bool expect = nit > 0 && p.flat && sh[16] != sh[6] && sh[11] > 1;
     if (expect) {
-      if (!__all_sync(0xffffffffu, mbar_wait(jbar, 0))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(jbar, 0, p.wait_limit))) {
         if (lane == 0) report(p.err, SEER_DEVERR_TIMEOUT);
         return;
       }
@@ -620,11 +620,11 @@ __device__ __forceinline__ void decode_body(const CUtensorMap* tmK, const CUtens
             if (first) {
               // the segment's q rows -> segment buffer nq & 1, once the segment two back has read it
               const int k = nq & 1, u = nq >> 1;
-              if (u >= 1 && !mbar_wait(&qempty[k], (u - 1) & 1)) {
+              if (u >= 1 && !mbar_wait(&qempty[k], (u - 1) & 1, p.wait_limit)) {
                 report(p.err, SEER_DEVERR_TIMEOUT);
                 sh[0] = 1;
               }
-              if (!sh[0]) {
+              if (!sh[0] && !p.starve) {
                 const int b = bh / p.Hkv, h = bh - b * p.Hkv;
                 mbar_arrive_expect_tx(&qfull[k], qbytes);
                 bulk_load(qseg + k * S::kQBytes, p.q + ((size_t)b * p.Hq + (size_t)h * g) * D, qbytes, &qfull[k]);
@@ -632,11 +632,11 @@ __device__ __forceinline__ void decode_body(const CUtensorMap* tmK, const CUtens
               ++nq;
             }
             const int s = it % STAGES;
-            if (!sh[0] && it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) - 1) & 1)) {
+            if (!sh[0] && it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) - 1) & 1, p.wait_limit)) {
               report(p.err, SEER_DEVERR_TIMEOUT);
               sh[0] = 1;
             }
-            if (!sh[0]) {
+            if (!sh[0] && !p.starve) {
               info[s].n = n;
               if (n >= 0) {
                 mbar_arrive_expect_tx(&full[s], 2u * S::kTile);
@@ -697,7 +697,7 @@ __device__ __forceinline__ void decode_body(const CUtensorMap* tmK, const CUtens
       it1 = nit;
     }
     // the group's q rows (rows >= g stay zero), then release the segment buffer
-    if (!__all_sync(0xffffffffu, mbar_wait(&qfull[seg & 1], (seg >> 1) & 1))) {
+    if (!__all_sync(0xffffffffu, mbar_wait(&qfull[seg & 1], (seg >> 1) & 1, p.wait_limit))) {
       alive = false;
       break;
     }
@@ -720,7 +720,7 @@ __device__ __forceinline__ void decode_body(const CUtensorMap* tmK, const CUtens
     for (int it = it0 + ((cg - it0 % NG) + NG) % NG; it < it1; it += NG) {
       const int s = it % STAGES;
       // every lane observes the phase (acquire); the warp leaves together if any lane gave up
-      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (it / STAGES) & 1))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (it / STAGES) & 1, p.wait_limit))) {
         alive = false;
         break;
       }
@@ -969,7 +969,7 @@ __device__ __forceinline__ void decode_body(const CUtensorMap* tmK, const CUtens
       while (!sh[9] && clock64() - t0 < kWaitLimitCycles) {
       }
       for (int s = 0; s < STAGES; ++s)
-        if (issued[s] > observed[s]) mbar_wait(&full[s], observed[s] & 1);
+        if (issued[s] > observed[s]) mbar_wait(&full[s], observed[s] & 1, p.wait_limit);
     }
     return;
   }

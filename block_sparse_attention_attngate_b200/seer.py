@@ -25,6 +25,8 @@ STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CAPACITY", 4: "
 KV_CONTIGUOUS, KV_PAGED = 0, 1
 SELECT_TOPK, SELECT_THRESHOLD, SELECT_TOPP = 0, 1, 2
 DEVERR_BLOCK_INDEX, DEVERR_PAGE_INDEX, DEVERR_COUNT, DEVERR_TIMEOUT = 1, 2, 4, 8
+WAIT_LIMIT_MIN, WAIT_LIMIT_MAX = 1000, 100_000_000_000
+DEBUG_STARVE_COPIES = 1
 
 EXPORTED = (
     "seer_kcomp_update", "seer_kcomp_state_bytes", "seer_kcomp_append", "seer_kcomp_state_init", "seer_gate_score",
@@ -32,7 +34,7 @@ EXPORTED = (
     "seer_decode_step", "seer_sparse_decode_auto_split",
     "seer_sparse_decode_workspace_bytes", "seer_sparse_decode", "seer_sparse_decode_noalloc",
     "seer_gate_truth_workspace_bytes", "seer_gate_truth", "seer_prefill_gt_workspace_bytes", "seer_prefill_gt",
-    "seer_last_error", "seer_version",
+    "seer_set_wait_limit", "seer_get_wait_limit", "seer_set_debug_flags", "seer_last_error", "seer_version",
 )
 
 
@@ -81,6 +83,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "seer_gate_truth": (I32, [DP, P, KP, P, P, P, P, SZ, P, P]),
         "seer_prefill_gt_workspace_bytes": (SZ, [DP, I32]),
         "seer_prefill_gt": (I32, [DP, P, I32, KP, KP, P, P, P, P, P, SZ, P, P]),
+        "seer_set_wait_limit": (I32, [I64]),
+        "seer_get_wait_limit": (I64, []),
+        "seer_set_debug_flags": (I32, [I32]),
         "seer_last_error": (ctypes.c_char_p, []),
         "seer_version": (ctypes.c_char_p, []),
     }
@@ -101,6 +106,22 @@ def version() -> str:
 def _check(status: int):
     if status != SEER_OK:
         raise SeerError(status, _lib.seer_last_error().decode())
+
+
+def set_wait_limit(cycles: int) -> None:
+    """Bound (SM clock cycles) of the sparse decode's copy and hand-off waits, process-wide;
+    0 restores the default (about one second)."""
+    _check(_lib.seer_set_wait_limit(int(cycles)))
+
+
+def get_wait_limit() -> int:
+    return int(_lib.seer_get_wait_limit())
+
+
+def set_debug_flags(flags: int) -> None:
+    """Process-wide debug switches of the sparse decode (DEBUG_STARVE_COPIES: no copy is issued,
+    so every CTA's first wait runs out and the launch reports DEVERR_TIMEOUT); 0 turns them off."""
+    _check(_lib.seer_set_debug_flags(int(flags)))
 
 
 def _ptr(t: Optional[torch.Tensor]):

@@ -419,6 +419,32 @@ seer_status seer_prefill_gt(const seer_dims_t* dims, const void* q, int32_t max_
                             void* out, float* lse_out, float* gt, void* workspace,
                             size_t workspace_bytes, int32_t* err_word, void* stream);
 
+/*
+ * Bounded waits of the sparse decode (seer_sparse_decode, seer_sparse_decode_noalloc and the
+ * decode launch of the two-launch step).  No passage defines these: they are part of the
+ * library's own error behaviour (a wait that runs out reports SEER_DEVERR_TIMEOUT and the kernel
+ * returns, so the context stays usable).
+ *
+ * seer_set_wait_limit: the bound of every copy and hand-off wait of those kernels, in SM clock
+ *   cycles, process-wide, taken at each launch.  0 restores the default (2e9 cycles, about one
+ *   second).  Values outside [SEER_WAIT_LIMIT_MIN, SEER_WAIT_LIMIT_MAX]: SEER_ERR_INVALID_ARG
+ *   and the bound is left as it was.  A small bound can make a healthy launch report a timeout.
+ * seer_get_wait_limit: the bound in force.
+ * seer_set_debug_flags: process-wide debug switches taken at each launch; 0 turns them off.
+ *   SEER_DEBUG_STARVE_COPIES: the decode's producer issues no copy and arms no barrier, so the
+ *   first wait of every CTA runs out; the launch writes no output, reports SEER_DEVERR_TIMEOUT and
+ *   leaves the workspace's split counters zero.  For tests of the timeout path only.  Unknown
+ *   bits: SEER_ERR_INVALID_ARG.  (The one-launch step, seer_decode_step, ignores the switch.)
+ * After a launch that reported SEER_DEVERR_TIMEOUT for any other reason, zero the workspace
+ * (seer_sparse_decode's split counters) before the next call.
+ */
+#define SEER_WAIT_LIMIT_MIN 1000LL
+#define SEER_WAIT_LIMIT_MAX 100000000000LL
+#define SEER_DEBUG_STARVE_COPIES 1
+seer_status seer_set_wait_limit(int64_t cycles);
+int64_t seer_get_wait_limit(void);
+seer_status seer_set_debug_flags(int32_t flags);
+
 /* Thread-local text describing the last non-OK status returned on this thread. */
 const char* seer_last_error(void);
 

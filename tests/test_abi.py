@@ -16,7 +16,7 @@ HEADER = os.path.join(ROOT, "include", "seer.h")
 
 def _header_functions():
     src = open(HEADER).read()
-    return re.findall(r"^(?:seer_status|size_t|int32_t|const char\*)\s+(seer_\w+)\s*\(", src, re.M)
+    return re.findall(r"^(?:seer_status|size_t|int32_t|int64_t|const char\*)\s+(seer_\w+)\s*\(", src, re.M)
 
 
 def _header_defines():
@@ -77,6 +77,8 @@ def test_header_constants_match_binding(S):
     assert d["SEER_SELECT_TOPP"] == S.SELECT_TOPP
     assert d["SEER_DEVERR_BLOCK_INDEX"] == S.DEVERR_BLOCK_INDEX and d["SEER_DEVERR_TIMEOUT"] == S.DEVERR_TIMEOUT
     assert d["SEER_DEVERR_PAGE_INDEX"] == S.DEVERR_PAGE_INDEX and d["SEER_DEVERR_COUNT"] == S.DEVERR_COUNT
+    assert d["SEER_WAIT_LIMIT_MIN"] == S.WAIT_LIMIT_MIN and d["SEER_WAIT_LIMIT_MAX"] == S.WAIT_LIMIT_MAX
+    assert d["SEER_DEBUG_STARVE_COPIES"] == S.DEBUG_STARVE_COPIES
 
 
 def _dims(S, **kw):
@@ -237,3 +239,20 @@ def test_missing_library_fails_loudly(tmp_path):
     from block_sparse_attention_attngate_b200 import seer
     with pytest.raises(ImportError):
         seer.load_library(str(tmp_path / "libseer.so"))
+
+
+def test_wait_limit_and_debug_flags(lib, S):
+    """The decode's wait bound and debug switch: range checks, 0 = the default, and a rejected
+    value leaves the setting as it was (no launch involved)."""
+    assert lib.seer_get_wait_limit() == 2_000_000_000
+    try:
+        assert lib.seer_set_wait_limit(5000) == 0 and lib.seer_get_wait_limit() == 5000
+        assert lib.seer_set_wait_limit(999) == 1 and lib.seer_get_wait_limit() == 5000
+        assert lib.seer_set_wait_limit(100_000_000_001) == 1 and lib.seer_get_wait_limit() == 5000
+        assert lib.seer_set_wait_limit(-5) == 1
+        assert lib.seer_set_wait_limit(0) == 0 and lib.seer_get_wait_limit() == 2_000_000_000
+        assert lib.seer_set_debug_flags(2) == 1 and lib.seer_set_debug_flags(-1) == 1
+        assert lib.seer_set_debug_flags(1) == 0
+    finally:
+        lib.seer_set_debug_flags(0)
+        lib.seer_set_wait_limit(0)

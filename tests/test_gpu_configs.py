@@ -396,7 +396,7 @@ def test_threshold_decode_loop_256_steps():
     cfg = config(5)
     inp = make_inputs(cfg, workers=draw_workers())
     tau = cfg.tau
-    fractions = np.linspace(0.05, 0.24, cfg.Hkv)
+    fractions = np.linspace(0.07, 0.20, cfg.Hkv)
     temps = _calibrate_temperatures(inp, tau, fractions)
     wq = scale_gate_weights(inp.w_q, temps)
     P = Problem(inp, w_q_bits=wq)
@@ -430,5 +430,5 @@ def test_threshold_decode_loop_256_steps():
     within = float(((fr >= 0.02) & (fr <= 0.30)).mean())
     print(f"threshold loop: selected fraction min {fr.min():.3f} median {np.median(fr):.3f} max {fr.max():.3f}; "
           f"{within:.1%} of (step, b, h) within [2%, 30%]; list mismatches at the cutoff {mism_total}/{compared}")
-    assert within >= 0.9
+    assert within >= 0.95
     assert mism_total <= compared // 100 + 1
