@@ -13,24 +13,30 @@
 // kept for the shapes this kernel does not take: head_dim 64, groups that do
 // not divide 128 rows).
 //
-// One CTA per (128 query rows, kv head, sequence): the g heads of the group x
-// 128/g consecutive positions, row r = head (r / P) at position p0 + (r % P).
-// Key tiles of 128 keys (one or two blocks).
-//   warps 0, 10 producers: K tiles (three-stage ring, a stage freed once S has
-//              read it) and V tiles (two stages, freed once P.V has read
-//              them) by TMA (128-byte swizzle, boxes of 64 channels x b keys)
-//   warp 1     allocates TMEM; one lane issues the MMAs: S_n = Q K_n^T into
-//              TMEM S[n % 2] (M = 128 rows, N = 128 keys, K = d; both
-//              operands in shared memory), then O += P_{n-1} V_{n-1} into TMEM O
-//              (N = d, K = 128 keys; P read from TMEM P[(n-1) % 2], V from
+// Work item: 128 query rows of one kv head of one sequence (the g heads of the
+// group x 128/g consecutive positions, row r = head (r / P) at position
+// p0 + (r % P)).  One persistent CTA per SM takes items in rounds, heaviest
+// (latest positions) first, alternating direction each round; the pipelines
+// below run on across items (the next item's Q is staged while the current
+// item's last P.V runs, and its first P.V waits until the previous O has been
+// read out of TMEM).  Key tiles of 128 keys (one or two blocks).
+//   warp 0 and the last warp: producers, K tiles (three-stage ring, a stage
+//              freed once S has read it) and V tiles (two stages, freed once
+//              P.V has read them) by TMA (128-byte swizzle, boxes of 64
+//              channels x b keys)
+//   warp 1     allocates TMEM; one lane issues the MMAs: S_u = Q K_u^T into
+//              TMEM S[u % 2] (M = 128 rows, N = 128 keys, K = d; both operands
+//              in shared memory) two tiles ahead -- S_{u+2} as soon as the
+//              softmax has read S_u, before P_u exists -- and O += P_u V_u into
+//              TMEM O (N = d, K = 128 keys; P read from TMEM P[u % 2], V from
 //              shared memory), each group closed by a commit to an mbarrier
-//   warps 2-9  two threads per row (the row's TMEM lane; one thread per half of
-//              the 128 keys, the pair exchanging the tile's maxima through
-//              shared memory): S by tcgen05.ld, causal mask, the row maximum of
-//              each block (stored for the targets),
-//              P = exp2(s - m_ref) as bf16 pairs into TMEM P[n % 2] by
-//              tcgen05.st (once the P.V of tile n - 2 has read that buffer, so
-//              tile n's exponentials overlap the P.V of tile n - 1),
+//   warps 2 .. 1 + 4 kNP: kNP threads per row (the row's TMEM lane; one
+//              thread per 128 / kNP keys of the tile, the kNP exchanging their
+//              maxima through shared memory): S by tcgen05.ld, causal mask, the
+//              row maximum of each block (stored for the targets),
+//              P = exp2(s - m_ref) as bf16 pairs into TMEM P[u % 2] by
+//              tcgen05.st (once the P.V of tile u - 2 has read that buffer, so
+//              tile u's exponentials overlap the P.V of tile u - 1),
 //              V rows past the sequence zeroed (the cache may hold NaN there),
 //              at the end O / l, the LSE and the row's log2 normaliser m + log2 l
 // TMEM columns: S[0] 0-127, S[1] 128-255, O 256-383, P[0] 384-447, P[1] 448-511.
@@ -43,6 +49,8 @@
 // the LSE use the same reference, so the results are those of the exact online
 // softmax (l sums the probabilities before their rounding to bf16 for the P.V
 // product).  All waits are bounded.
+#include <algorithm>
+
 #include "seer_device.cuh"
 #include "seer_internal.h"
 
@@ -57,12 +65,15 @@ constexpr int kBoxB = kM * 128;         // bytes of a 128-row x 64-channel (or 6
 constexpr int kTileB = 2 * kBoxB;       // 32 KB: a K, V or Q tile (two boxes)
 constexpr int kKStages = 3;
 constexpr int kVStages = 2;
-constexpr int kThreads = 11 * 32;
+constexpr int kNP = 2;                  // softmax threads per row (each a 128 / kNP-key part of the tile)
+constexpr int kSW = 4 * kNP;            // softmax warps (kNP per TMEM lane quarter)
+constexpr int kVWarp = 2 + kSW;         // the V producer (after the softmax warps)
+constexpr int kThreads = (kSW + 3) * 32;
 constexpr uint32_t kTmemCols = 512;     // S[0] 0..127, S[1] 128..255, O 256..383, P[0] 384..447, P[1] 448..511
 constexpr float kLazy = 8.f;            // m_ref moves when a tile maximum exceeds it by more than this
 constexpr size_t kSmem = 1024 + kTileB /* Q */ + (size_t)(kKStages + kVStages) * kTileB /* K, V */ +
-                         256 /* barriers */ + 2 * 2 * kM * 4 /* the pairs' tile maxima, two tiles */ +
-                         2 * kM * 4 /* each half's l */;
+                         256 /* barriers */ + 2 * kNP * kM * 4 /* the parts' tile maxima, two tiles */ +
+                         kNP * kM * 4 /* each part's l */;
 
 static_assert(kSmem <= 227 * 1024, "dynamic shared memory above the per-CTA limit");
 
@@ -132,6 +143,13 @@ __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* v) {
       "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
       "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31]));
 }
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]));
+}
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
@@ -154,14 +172,39 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// TMA coordinates 1..3 of (token t, head h, sequence bp): perm[k] is the dimension (0..2 for
+// coordinates 1..3) that holds token / head / sequence (selects, not a runtime-indexed array)
 __device__ __forceinline__ void kv_coords(const int32_t perm[3], int t, int h, int bp, int& c1, int& c2, int& c3) {
-  int c[3];
-  c[perm[0]] = t;
-  c[perm[1]] = h;
-  c[perm[2]] = bp;
-  c1 = c[0];
-  c2 = c[1];
-  c3 = c[2];
+  auto at = [&](int d) { return perm[0] == d ? t : (perm[1] == d ? h : bp); };
+  c1 = at(0);
+  c2 = at(1);
+  c3 = at(2);
+}
+
+// The work items (128 query rows of one KV head of one sequence: the group's g heads x 128 / g
+// positions), heaviest (latest positions) first.
+struct TcItem {
+  int b, hk, p0, L, nt;
+};
+
+// Item `it` of the order (position tiles from the last, then KV head, then sequence); nt = 0 when
+// none of its positions exists.
+__device__ __forceinline__ TcItem tc_item(const PrefillParams& p, int P, int npt, int it) {
+  TcItem w;
+  const int per = p.Hkv * p.B, pr = it / per, rem = it - pr * per;
+  w.hk = rem % p.Hkv;
+  w.b = rem / p.Hkv;
+  w.p0 = (npt - 1 - pr) * P;
+  w.L = min(max(p.seqlens[w.b], 0), min(p.T, p.kcap));
+  w.nt = w.p0 < w.L ? (min(w.p0 + P, w.L) - 1) / kKT + 1 : 0;
+  return w;
+}
+
+// Round r of CTA c: item r * G + c on even rounds, r * G + (G - 1 - c) on odd ones, so that each
+// CTA's items alternate between the heavy and the light end of a round.
+__device__ __forceinline__ int tc_item_index(int r) {
+  const int G = (int)gridDim.x, c = (int)blockIdx.x;
+  return r * G + ((r & 1) ? G - 1 - c : c);
 }
 
 template <int BLK>
@@ -179,21 +222,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* v_empty = v_full + kVStages;
   uint64_t* s_full = v_empty + kVStages;   // [2]
   uint64_t* s_free = s_full + 2;           // [2]
-  uint64_t* p_full = s_free + 2;     // [2] P[k] written (tile n, k = n % 2)
-  uint64_t* p_free = p_full + 2;     // [2] one completion per P.V of P[k] (P[k] read; tiles 0..m in O)
-  uint64_t* o_fin = p_free + 2;      // the last P.V done (single use)
-  uint64_t* q_ready = o_fin + 1;
+  uint64_t* p_full = s_free + 2;     // [2] P[k] written (tile u, k = u % 2)
+  uint64_t* p_free = p_full + 2;     // [2] one completion per P.V of P[k]
+  uint64_t* o_fin = p_free + 2;      // an item's last P.V done (one completion per item)
+  uint64_t* o_drain = o_fin + 1;     // an item's O read out of TMEM (one completion per item)
+  uint64_t* q_ready = o_drain + 1;   // an item's Q tile in shared memory (one completion per item)
   uint64_t* drain = q_ready + 1;
-  uint64_t* pbar = drain + 1;        // [4] the two warps of each TMEM lane quarter
+  uint64_t* pbar = drain + 1;        // [4] the kNP warps of each TMEM lane quarter
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pbar + 4);
   volatile int* sh = reinterpret_cast<volatile int*>(tmem_slot + 1);   // [0] abort
-  float* xch = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(k_full) + 256);   // [tile & 1][half][row]
-  float* lh = xch + 2 * 2 * kM;                                                      // [half][row] l
+  float* xch = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(k_full) + 256);   // [tile & 1][part][row]
+  float* lh = xch + 2 * kNP * kM;                                                    // [part][row] l
 
   const int g = p.g, P = kM / g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
-  const int b = blockIdx.z, hk = blockIdx.y;
-  const int p0 = ((int)gridDim.x - 1 - (int)blockIdx.x) * P;   // heaviest (latest) positions first
+  const int npt = (p.T + P - 1) / P;               // position tiles per (KV head, sequence)
+  const int n_items = npt * p.Hkv * p.B;
+  const int rounds = (n_items + (int)gridDim.x - 1) / (int)gridDim.x;
 
   if (tid == 0) {
     tma_prefetch_desc(&tmK);
@@ -208,29 +253,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(&s_full[k], 1);
-      mbar_init(&s_free[k], 8);
+      mbar_init(&s_free[k], kSW);
     }
-    for (int k = 0; k < 4; ++k) mbar_init(&pbar[k], 2);
+    for (int k = 0; k < 4; ++k) mbar_init(&pbar[k], kNP);
     for (int k = 0; k < 2; ++k) {
-      mbar_init(&p_full[k], 8);
+      mbar_init(&p_full[k], kSW);
       mbar_init(&p_free[k], 1);
     }
     mbar_init(o_fin, 1);
-    mbar_init(q_ready, 8);
+    mbar_init(o_drain, kSW);
+    mbar_init(q_ready, kSW);
     mbar_init(drain, 1);
     sh[0] = 0;
     fence_barrier_init();
   }
-  __syncthreads();
-  pdl_wait();
-  pdl_trigger();
-  const int Lr = max(p.seqlens[b], 0);
-  const int L = min(Lr, min(p.T, p.kcap));
-  if (Lr > L && blockIdx.x == 0 && hk == 0 && tid == 0) report(p.err, SEER_DEVERR_COUNT);
-  if (p0 >= L) return;   // the whole CTA: no position of these rows exists (no TMEM taken yet)
-  const int pend = min(p0 + P, L);
-  const int nt = (pend - 1) / kKT + 1;   // key tiles 0 .. nt-1 hold a key visible to some row
-
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                  "r"(kTmemCols));
@@ -240,10 +276,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS[2] = {tmem, tmem + 128}, tO = tmem + 256, tP[2] = {tmem + 384, tmem + 448};
+  // TMEM columns: S[k] at 128 k, O at 256, P[k] at 384 + 64 k (computed, not indexed: a runtime index into
+  // a local array would put it in local memory)
+  const uint32_t tO = tmem + 256;
+  auto tS = [tmem](uint32_t k) { return tmem + 128u * k; };
+  auto tP = [tmem](uint32_t k) { return tmem + 384u + 64u * k; };
+  pdl_wait();
+  pdl_trigger();
+  if (blockIdx.x == 0 && tid == 0)
+    for (int bb = 0; bb < p.B; ++bb)
+      if (p.seqlens[bb] > min(p.T, p.kcap)) report(p.err, SEER_DEVERR_COUNT);
 
-  if (warp == 0 || warp == 10) {
-    // ---------------------------------------------------------------- producers (K: warp 0, V: warp 10)
+  if (warp == 0 || warp == kVWarp) {
+    // ---------------------------------------------------------------- producers (K: warp 0, V: the last)
     const bool isK = warp == 0;
     const int NS = isK ? kKStages : kVStages;
     uint64_t* full = isK ? k_full : v_full;
@@ -252,68 +297,93 @@ __global__ void __launch_bounds__(kThreads, 1)
     const CUtensorMap* tm = isK ? &tmK : &tmV;
     const int32_t* perm = isK ? p.k_perm : p.v_perm;
     if (lane == 0) {
-      int issued = 0;
-      for (int n = 0; n < nt; ++n) {
-        const int s = n % NS;
-        if (n >= NS && !mbar_wait(&empty[s], ((n / NS) - 1) & 1)) {
-          report(p.err, SEER_DEVERR_TIMEOUT);
-          sh[0] = 1;
-          break;
-        }
-        if (sh[0]) break;
-        issued = n + 1;
-        mbar_arrive_expect_tx(&full[s], (uint32_t)kTileB);
-        uint8_t* dst = ringb + (size_t)s * kTileB;
+      uint32_t u = 0;   // tiles issued (over every item of this CTA)
+      for (int r = 0; r < rounds && !sh[0]; ++r) {
+        const int it = tc_item_index(r);
+        if (it >= n_items) continue;
+        const TcItem w = tc_item(p, P, npt, it);
+        for (int n = 0; n < w.nt; ++n, ++u) {
+          const uint32_t s = u % NS;
+          if (u >= (uint32_t)NS && !mbar_wait(&empty[s], ((u / NS) - 1) & 1)) {
+            report(p.err, SEER_DEVERR_TIMEOUT);
+            sh[0] = 1;
+          }
+          if (sh[0]) break;
+          mbar_arrive_expect_tx(&full[s], (uint32_t)kTileB);
+          uint8_t* dst = ringb + (size_t)s * kTileB;
 #pragma unroll
-        for (int sub = 0; sub < NBT; ++sub) {
-          // a 64-channel box of BLK keys; the tile's two channel halves are kBoxB apart, its blocks
-          // BLK rows (BLK * 128 bytes) apart within a half
-          int c1, c2, c3;
-          kv_coords(perm, n * kKT + sub * BLK, hk, b, c1, c2, c3);
+          for (int sub = 0; sub < NBT; ++sub) {
+            // a 64-channel box of BLK keys; the tile's two channel halves are kBoxB apart, its blocks
+            // BLK rows (BLK * 128 bytes) apart within a half
+            int c1, c2, c3;
+            kv_coords(perm, n * kKT + sub * BLK, w.hk, w.b, c1, c2, c3);
 #pragma unroll
-          for (int hx = 0; hx < 2; ++hx)
-            tma_load_4d(dst + hx * kBoxB + sub * BLK * 128, tm, &full[s], hx * 64, c1, c2, c3);
+            for (int hx = 0; hx < 2; ++hx)
+              tma_load_4d(dst + hx * kBoxB + sub * BLK * 128, tm, &full[s], hx * 64, c1, c2, c3);
+          }
         }
       }
       // copies still landing when a consumer gave up: wait for them (bounded) before shared memory
       // is released; no later phase is ever armed on those stages
-      for (int n = max(0, issued - NS); n < issued; ++n) mbar_wait(&full[n % NS], (n / NS) & 1);
+      for (uint32_t m = u > (uint32_t)NS ? u - NS : 0; m < u; ++m) mbar_wait(&full[m % NS], (m / NS) & 1);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_bf16(kM, kKT, 0), id_o = idesc_bf16(kM, kD, 1);
       const uint32_t qa = smem_u32(qs);
-      bool ok = mbar_wait(q_ready, 0);
-      auto issue_pv = [&](int m) {
-        const int sv = m % kVStages, pb = m & 1;
+      bool ok = true;
+      uint32_t u0 = 0;   // tiles of the earlier items
+      int items = 0;     // items started before this one
+      // O += P_m V_m (m counts tiles over every item); the item's first P.V overwrites O, once the
+      // previous item's O has been read out
+      auto issue_pv = [&](uint32_t m, bool first) {
+        const uint32_t sv = m % kVStages, pb = m & 1;
         ok = ok && mbar_wait(&p_full[pb], (m >> 1) & 1) && mbar_wait(&v_full[sv], (m / kVStages) & 1);
+        if (first && items > 0) ok = ok && mbar_wait(o_drain, (items - 1) & 1);
         if (!ok) return;
         tc_fence_after();
         const uint32_t vb = smem_u32(vring + (size_t)sv * kTileB);
 #pragma unroll
         for (int kk = 0; kk < kKT / 16; ++kk)
-          umma_f16_ta(tO, tP[pb] + kk * 8, desc_mnmajor(vb + kk * 2048, kBoxB), id_o, (m > 0 || kk > 0) ? 1u : 0u);
+          umma_f16_ta(tO, tP(pb) + kk * 8, desc_mnmajor(vb + kk * 2048, kBoxB), id_o, (!first || kk > 0) ? 1u : 0u);
         umma_commit(&v_empty[sv]);
         umma_commit(&p_free[pb]);
       };
-      for (int n = 0; n < nt && ok; ++n) {
-        const int sk = n % kKStages, k2 = n & 1;
-        ok = ok && mbar_wait(&k_full[sk], (n / kKStages) & 1);
-        ok = ok && (n < 2 || mbar_wait(&s_free[k2], ((n >> 1) - 1) & 1));
-        if (!ok) break;
+      // S_u = Q K_u^T into S[u % 2], once K_u has landed and the softmax has read S_{u-2}
+      auto issue_s = [&](uint32_t u) {
+        const uint32_t sk = u % kKStages, k2 = u & 1;
+        ok = ok && mbar_wait(&k_full[sk], (u / kKStages) & 1);
+        ok = ok && (u < 2 || mbar_wait(&s_free[k2], ((u >> 1) - 1) & 1));
+        if (!ok) return;
         tc_fence_after();
         const uint32_t kb = smem_u32(kring + (size_t)sk * kTileB);
 #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks)
-          umma_f16(tS[k2], desc_kmajor(qa + (ks >> 2) * kBoxB + (ks & 3) * 32),
+          umma_f16(tS(k2), desc_kmajor(qa + (ks >> 2) * kBoxB + (ks & 3) * 32),
                    desc_kmajor(kb + (ks >> 2) * kBoxB + (ks & 3) * 32), id_s, ks > 0 ? 1u : 0u);
         umma_commit(&k_empty[sk]);
         umma_commit(&s_full[k2]);
-        if (n > 0) issue_pv(n - 1);
+      };
+      // Issue order within an item: S_0, S_1, then for each tile n: S_{n+2} (as soon as the softmax
+      // has read S_n, before P_n exists) and P_n V_n.  S thus runs two tiles ahead and never queues
+      // behind a P.V that waits for the softmax.
+      for (int r = 0; r < rounds && ok; ++r) {
+        const int it = tc_item_index(r);
+        if (it >= n_items) continue;
+        const TcItem w = tc_item(p, P, npt, it);
+        if (w.nt == 0) continue;
+        ok = mbar_wait(q_ready, items & 1);
+        issue_s(u0);
+        if (w.nt > 1) issue_s(u0 + 1);
+        for (int n = 0; n < w.nt && ok; ++n) {
+          if (n + 2 < w.nt) issue_s(u0 + n + 2);
+          issue_pv(u0 + n, n == 0);
+        }
+        if (ok) umma_commit(o_fin);
+        u0 += w.nt;
+        ++items;
       }
-      if (ok) issue_pv(nt - 1);
-      if (ok) umma_commit(o_fin);
       if (!ok) {
         report(p.err, SEER_DEVERR_TIMEOUT);
         sh[0] = 1;
@@ -323,177 +393,226 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(drain, 0);
     }
   } else {
-    // ---------------------------------------------------------------- softmax warps (two per row)
-    constexpr int HK = kKT / 2;               // keys per thread (a half of the tile)
+    // ---------------------------------------------------------------- softmax warps (kNP per row)
+    constexpr int HK = kKT / kNP;             // keys per thread (a part of the tile)
+    constexpr int CP = kD / kNP;              // O channels per thread
     const int quarter = warp & 3;             // warp w reads TMEM lanes 32(w % 4) .. 32(w % 4) + 31
-    const int half = (warp - 2) >> 2;         // warps 2-5: keys 0..63 of each tile, warps 6-9: 64..127
+    const int part = (warp - 2) >> 2;         // warps 2-5: keys 0..HK-1 of each tile, warps 6-9 the next HK, ...
     const int row = 32 * quarter + lane;
-    const int j = row / P, t = row - (row / P) * P;
-    const int h = hk * g + j, i = p0 + t;     // query head and position of the row
-    const bool live = i < L;
-    const int vis = min(i, L - 1);            // last key the row sees
-    const size_t qrow = ((size_t)b * p.Hq + h) * p.T;
+    const int j = row / P, t = row - (row / P) * P;   // the row's head in the group and position offset
     const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
-    const int st = tid - 64;                  // 0..255 over the softmax warps
-    uint32_t pph = 0;                         // the pair barrier's phase
-    // this thread's half of the Q row (64 channels, one 128B-swizzled box) -> shared memory, zero past L
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (live) v = *reinterpret_cast<const uint4*>(p.q + (qrow + i) * kD + half * 64 + c * 8);
-      *reinterpret_cast<uint4*>(qs + half * kBoxB + sw128(row, c)) = v;
-    }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    __syncwarp();
-    if (lane == 0) mbar_arrive(q_ready);
+    const int st = tid - 64;                  // 0 .. 32 kSW - 1 over the softmax warps
     const float sl2 = p.scale_log2;
-    float* rws = p.rmax + ((size_t)b * p.Hq + h) * p.NB * p.T;
-    float m_ref = -INFINITY, l = 0.f;
-    bool ok = true;
-    for (int n = 0; n < nt && ok; ++n) {
-      const int k2 = n & 1, sv = n % kVStages;
-      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[k2], (n >> 1) & 1));
-      if (!ok) break;
-      tc_fence_after();
-      float x[HK];
+    uint32_t pph = 0;                         // the quarter barrier's phase
+    // this thread's CP channels of an item's Q row (in the 128B-swizzled box of its 64 channels) ->
+    // shared memory, zero past L; then the item's Q is announced
+    auto load_q = [&](const TcItem& w) {
+      const int i = w.p0 + t;
+      const size_t qrow = ((size_t)w.b * p.Hq + (size_t)w.hk * g + j) * p.T;
 #pragma unroll
-      for (int c0 = 0; c0 < HK; c0 += 32) tmem_ld32(tS[k2] + lane_base + half * HK + c0, x + c0);
-      tmem_wait_ld();
-      tc_fence_before();
+      for (int c = 0; c < CP / 8; ++c) {
+        const int ch = part * CP + c * 8;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (i < w.L) v = *reinterpret_cast<const uint4*>(p.q + (qrow + i) * kD + ch);
+        *reinterpret_cast<uint4*>(qs + (ch >> 6) * kBoxB + sw128(row, (ch & 63) >> 3)) = v;
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[k2]);   // S[k2] may be overwritten (tile n + 2)
-      // causal mask (key kt visible to row i iff kt <= min(i, L - 1)) where the tile needs one; the
-      // maximum of this half (raw scores: the scale is positive)
-      const int k0 = n * kKT + half * HK;     // first key of this half
-      if (k0 + HK - 1 > vis) {
-#pragma unroll
-        for (int c = 0; c < HK; ++c) x[c] = (k0 + c <= vis) ? x[c] : -INFINITY;
+      if (lane == 0) mbar_arrive(q_ready);
+    };
+    // the next round (from r on) with an item that has work
+    auto next_round = [&](int r) {
+      for (; r < rounds; ++r) {
+        const int it = tc_item_index(r);
+        if (it < n_items && tc_item(p, P, npt, it).nt > 0) return r;
       }
-      float hm = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < HK; ++c) hm = fmaxf(hm, x[c]);
-      hm *= sl2;   // log2 domain
-      // the pair's tile maximum (double-buffered by tile parity: the partner has read tile n - 2's
-      // value before it arrived at tile n - 1's barrier)
-      xch[(k2 * 2 + half) * kM + row] = hm;
-      if (!warps_sync(&pbar[quarter], pph)) {
-        ok = false;
-        break;
-      }
-      const float hm2 = xch[(k2 * 2 + (half ^ 1)) * kM + row];
-      const float mx = fmaxf(hm, hm2);
-      // the row maximum of each block: a 64-key block is this half; a 128-key block is the tile
-#pragma unroll
-      for (int sub = 0; sub < NBT; ++sub) {
-        if (NBT == 2 ? sub != half : half != 0) continue;
-        const int blk = n * NBT + sub;
-        if (live && blk * BLK <= i) rws[(size_t)blk * p.T + i] = NBT == 2 ? hm : mx;
-      }
-      // reference maximum: the first tile's, moved only when a tile exceeds it by more than kLazy;
-      // then O (in TMEM, holding tiles 0..n-1) and l are rescaled
-      float alpha = 1.f;
-      bool move = false;
-      if (n == 0) {
-        m_ref = mx;
-      } else if (mx > m_ref + kLazy) {
-        alpha = ex2(m_ref - mx);
-        m_ref = mx;
-        move = true;
-      }
-      l *= alpha;
-      // P[n % 2] is free once the P.V of tile n - 2 has read it (that buffer's (n / 2)-th completion;
-      // the next one needs P of tile n, not yet written, so a parity wait is exact).  A rescale of O
-      // waits for the P.V of tile n - 1 as well (O then holds tiles 0..n-1 and nothing adds to it).
-      const int pb = n & 1;
-      if (n > 1) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&p_free[pb], ((n >> 1) - 1) & 1));
-        if (!ok) break;
-      }
-      if (__any_sync(0xffffffffu, move)) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&p_free[pb ^ 1], ((n - 1) >> 1) & 1));
+      return rounds;
+    };
+    bool ok = true;
+    uint32_t u0 = 0;   // tiles of the earlier items
+    int items = 0;
+    int r = next_round(0);
+    if (r < rounds) load_q(tc_item(p, P, npt, tc_item_index(r)));
+    while (r < rounds && ok) {
+      const TcItem w = tc_item(p, P, npt, tc_item_index(r));
+      const int L = w.L, h = w.hk * g + j, i = w.p0 + t;   // query head and position of the row
+      const bool live = i < L;
+      const int vis = min(i, L - 1);            // last key the row sees
+      const size_t qrow = ((size_t)w.b * p.Hq + h) * p.T;
+      float* rws = p.rmax + ((size_t)w.b * p.Hq + h) * p.NB * p.T;
+      float m_ref = -INFINITY, l = 0.f;
+      for (int n = 0; n < w.nt && ok; ++n) {
+        const uint32_t u = u0 + n, k2 = u & 1, sv = u % kVStages;
+        ok = __all_sync(0xffffffffu, mbar_wait(&s_full[k2], (u >> 1) & 1));
         if (!ok) break;
         tc_fence_after();
-#pragma unroll 1
-        for (int c0 = 0; c0 < kD / 2; c0 += 32) {
-          float o[32];
-          tmem_ld32(tO + lane_base + half * (kD / 2) + c0, o);
-          tmem_wait_ld();
+        float x[HK];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] *= alpha;
-          tmem_st32(tO + lane_base + half * (kD / 2) + c0, o);
+        for (int c0 = 0; c0 < HK; c0 += 32) tmem_ld32(tS(k2) + lane_base + part * HK + c0, x + c0);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_free[k2]);   // S[k2] may be overwritten (tile u + 2)
+        // causal mask (key kt visible to row i iff kt <= min(i, L - 1)) where the tile needs one; the
+        // maximum of this part (raw scores: the scale is positive)
+        const int k0 = n * kKT + part * HK;     // first key of this part
+        if (k0 + HK - 1 > vis) {
+#pragma unroll
+          for (int c = 0; c < HK; ++c) x[c] = (k0 + c <= vis) ? x[c] : -INFINITY;
+        }
+        // (eight independent running maxima: a single chain would be HK dependent max operations)
+        float m8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m8[e] = x[e];
+#pragma unroll
+        for (int c = 8; c < HK; c += 8)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) m8[e] = fmaxf(m8[e], x[c + e]);
+        float hm = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        hm *= sl2;   // log2 domain
+        // the parts' maxima (double-buffered by tile parity: every part has read tile u - 2's values
+        // before it arrived at tile u - 1's barrier)
+        xch[(k2 * kNP + part) * kM + row] = hm;
+        if (!warps_sync(&pbar[quarter], pph)) {
+          ok = false;
+          break;
+        }
+        float pm[kNP];
+#pragma unroll
+        for (int q = 0; q < kNP; ++q) pm[q] = xch[(k2 * kNP + q) * kM + row];
+        float mx = pm[0];
+#pragma unroll
+        for (int q = 1; q < kNP; ++q) mx = fmaxf(mx, pm[q]);
+        // the row maximum of each block (PPB parts), written by the block's first part
+        constexpr int PPB = BLK / HK;
+#pragma unroll
+        for (int sub = 0; sub < NBT; ++sub) {
+          if (part != sub * PPB) continue;
+          float bm = pm[sub * PPB];
+#pragma unroll
+          for (int q = 1; q < PPB; ++q) bm = fmaxf(bm, pm[sub * PPB + q]);
+          const int blk = n * NBT + sub;
+          if (live && blk * BLK <= i) rws[(size_t)blk * p.T + i] = bm;
+        }
+        // reference maximum: the item's first tile's, moved only when a tile exceeds it by more than
+        // kLazy; then O (in TMEM, holding the item's tiles before this one) and l are rescaled
+        float alpha = 1.f;
+        bool move = false;
+        if (n == 0) {
+          m_ref = mx;
+        } else if (mx > m_ref + kLazy) {
+          alpha = ex2(m_ref - mx);
+          m_ref = mx;
+          move = true;
+        }
+        l *= alpha;
+        // P[u % 2] is free once the P.V of tile u - 2 has read it (that buffer's (u / 2)-th completion;
+        // the next one needs P of tile u, not yet written, so a parity wait is exact).  A rescale of O
+        // waits for the P.V of tile u - 1 as well (O then holds the item's earlier tiles and nothing
+        // adds to it).
+        const uint32_t pb = u & 1;
+        if (u > 1) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&p_free[pb], ((u >> 1) - 1) & 1));
+          if (!ok) break;
+        }
+        if (__any_sync(0xffffffffu, move)) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&p_free[pb ^ 1], ((u - 1) >> 1) & 1));
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll 1
+          for (int c0 = 0; c0 < CP; c0 += 32) {
+            float o[32];
+            tmem_ld32(tO + lane_base + part * CP + c0, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= alpha;
+            tmem_st32(tO + lane_base + part * CP + c0, o);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+        }
+        // P = exp2(s * scale - m_ref) (<= 2^kLazy; masked keys give 0) as bf16 pairs into this part's
+        // HK / 2 columns of P[u % 2] in TMEM; l sums the same values
+        const float mu = m_ref == -INFINITY ? 0.f : m_ref;
+        {
+          uint32_t pw[HK / 2];
+          float s8[8];   // independent partial sums (one chain would be HK dependent adds)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) s8[e] = 0.f;
+#pragma unroll
+          for (int e = 0; e < HK / 2; ++e) {
+            const float a = ex2(fmaf(x[2 * e], sl2, -mu)), bb = ex2(fmaf(x[2 * e + 1], sl2, -mu));
+            s8[e & 7] += a + bb;
+            pw[e] = pack_bf16(a, bb);
+          }
+          if constexpr (HK == 64) tmem_st32u(tP(pb) + lane_base + part * (HK / 2), pw);
+          else tmem_st16u(tP(pb) + lane_base + part * (HK / 2), pw);
+          l += ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
+        }
+        if (n * kKT + kKT > L) {
+          // V rows past L may hold anything (even NaN): zero them so that P = 0 there gives 0.  Wait for
+          // the tile's copy here too (its phase is at most one behind, as for the MMA issuer); whole
+          // 128-byte rows, so the swizzle does not matter.
+          ok = __all_sync(0xffffffffu, mbar_wait(&v_full[sv], (u / kVStages) & 1));
+          if (!ok) break;
+          uint8_t* vt = vring + (size_t)sv * kTileB;
+          const int r0 = max(0, L - n * kKT), nchunk = (kKT - r0) * 8;   // 16-byte chunks per channel half
+          for (int e = st; e < 2 * nchunk; e += kSW * 32) {
+            const int hx = e / nchunk, rr = r0 + (e - hx * nchunk) / 8, cc = e & 7;
+            *reinterpret_cast<uint4*>(vt + hx * kBoxB + rr * 128 + cc * 16) = make_uint4(0u, 0u, 0u, 0u);
+          }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         }
         tmem_wait_st();
         tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[pb]);
       }
-      // P = exp2(s * scale - m_ref) (<= 2^kLazy; masked keys give 0) as bf16 pairs into this half's
-      // 32 columns of P[n % 2] in TMEM; l sums the same values
-      const float mu = m_ref == -INFINITY ? 0.f : m_ref;
-      float sum = 0.f;
-      {
-        uint32_t w[HK / 2];
+      if (!ok) break;
+      // the next item's Q: every S of this item has completed (this thread saw the last one's
+      // commit, which covers every earlier MMA), so the Q tile is free
+      const int rn = next_round(r + 1);
+      if (rn < rounds) load_q(tc_item(p, P, npt, tc_item_index(rn)));
+      // this item's last P.V (one o_fin completion per item; the next needs this item's O read out)
+      ok = __all_sync(0xffffffffu, mbar_wait(o_fin, items & 1));
+      if (ok) {
+        lh[part * kM + row] = l;
+        ok = warps_sync(&pbar[quarter], pph);
+      }
+      if (!ok) break;
+      float lt = 0.f;   // the row's l (all parts; one reference maximum)
 #pragma unroll
-        for (int e = 0; e < HK / 2; ++e) {
-          const float a = ex2(fmaf(x[2 * e], sl2, -mu)), bb = ex2(fmaf(x[2 * e + 1], sl2, -mu));
-          sum += a + bb;
-          w[e] = pack_bf16(a, bb);
-        }
-        tmem_st32u(tP[pb] + lane_base + half * (HK / 2), w);
-      }
-      l += sum;
-      if (n * kKT + kKT > L) {
-        // V rows past L may hold anything (even NaN): zero them so that P = 0 there gives 0.  Wait for
-        // the tile's copy here too (its phase is at most one behind, as for the MMA issuer); whole
-        // 128-byte rows, so the swizzle does not matter.
-        ok = __all_sync(0xffffffffu, mbar_wait(&v_full[sv], (n / kVStages) & 1));
-        if (!ok) break;
-        uint8_t* vt = vring + (size_t)sv * kTileB;
-        const int r0 = max(0, L - n * kKT), nchunk = (kKT - r0) * 8;   // 16-byte chunks per channel half
-        for (int e = st; e < 2 * nchunk; e += 256) {
-          const int hx = e / nchunk, rr = r0 + (e - hx * nchunk) / 8, cc = e & 7;
-          *reinterpret_cast<uint4*>(vt + hx * kBoxB + rr * 128 + cc * 16) = make_uint4(0u, 0u, 0u, 0u);
-        }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      }
-      tmem_wait_st();
+      for (int q = 0; q < kNP; ++q) lt += lh[q * kM + row];
+      tc_fence_after();
+      float o[CP];
+#pragma unroll
+      for (int c0 = 0; c0 < CP; c0 += 32) tmem_ld32(tO + lane_base + part * CP + c0, o + c0);
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[pb]);
-    }
-    if (ok) {
-      // the last P.V (its own barrier: p_free may be two completions behind here)
-      ok = __all_sync(0xffffffffu, mbar_wait(o_fin, 0));
-    }
-    if (ok) {
-      lh[half * kM + row] = l;
-      ok = warps_sync(&pbar[quarter], pph);
-    }
-    if (ok) {
-      const float lt = lh[row] + lh[kM + row];   // the row's l (both halves; one reference maximum)
-      tc_fence_after();
+      if (lane == 0) mbar_arrive(o_drain);   // O may be overwritten by the next item
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
-#pragma unroll 1
-      for (int c0 = 0; c0 < kD / 2; c0 += 32) {
-        float o[32];
-        tmem_ld32(tO + lane_base + half * (kD / 2) + c0, o);
-        tmem_wait_ld();
-        if (live) {
+      if (live) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            uint4 w;
-            w.x = pack_bf16(o[e] * inv, o[e + 1] * inv);
-            w.y = pack_bf16(o[e + 2] * inv, o[e + 3] * inv);
-            w.z = pack_bf16(o[e + 4] * inv, o[e + 5] * inv);
-            w.w = pack_bf16(o[e + 6] * inv, o[e + 7] * inv);
-            *reinterpret_cast<uint4*>(p.o + (qrow + i) * kD + half * (kD / 2) + c0 + e) = w;
-          }
+        for (int e = 0; e < CP; e += 8) {
+          uint4 v;
+          v.x = pack_bf16(o[e] * inv, o[e + 1] * inv);
+          v.y = pack_bf16(o[e + 2] * inv, o[e + 3] * inv);
+          v.z = pack_bf16(o[e + 4] * inv, o[e + 5] * inv);
+          v.w = pack_bf16(o[e + 6] * inv, o[e + 7] * inv);
+          *reinterpret_cast<uint4*>(p.o + (qrow + i) * kD + part * CP + e) = v;
+        }
+        if (part == 0) {
+          const float c = lt > 0.f ? m_ref + log2f(lt) : -INFINITY;   // log2 of the row's normaliser
+          if (p.lse) p.lse[qrow + i] = c * kLn2f;
+          p.rnorm[qrow + i] = c;
         }
       }
-      if (half == 0 && live) {
-        const float c = lt > 0.f ? m_ref + log2f(lt) : -INFINITY;   // log2 of the row's normaliser
-        if (p.lse) p.lse[qrow + i] = c * kLn2f;
-        p.rnorm[qrow + i] = c;
-      }
-    } else {
+      u0 += w.nt;
+      ++items;
+      r = rn;
+    }
+    if (!ok) {
       if (lane == 0) report(p.err, SEER_DEVERR_TIMEOUT);
       sh[0] = 1;
     }
@@ -614,13 +733,14 @@ __global__ void __launch_bounds__(kTgWarps * 32)
 
 template <int BLK>
 cudaError_t launch_tc_t(const CUtensorMap& tk, const CUtensorMap& tv, const PrefillParams& p, int max_len,
-                        cudaStream_t st) {
+                        int sms, cudaStream_t st) {
   auto kern = prefill_tc_kernel<BLK>;
   static std::atomic<uint64_t> attr_done{0};
   cudaError_t e = ensure_smem_limit(kern, (int)kSmem, attr_done);
   if (e != cudaSuccess) return e;
   const int P = kM / p.g;
-  const dim3 grid((max_len + P - 1) / P, p.Hkv, p.B);
+  const long long items = (long long)((max_len + P - 1) / P) * p.Hkv * p.B;
+  const dim3 grid((unsigned)std::min<long long>(items, std::max(sms, 1)));
   e = launch_pdl(kern, grid, dim3(kThreads), kSmem, st, tk, tv, p);
   if (e != cudaSuccess) return e;
   const dim3 tgrid((max_len + kTgPos - 1) / kTgPos, p.Hkv, p.B);
@@ -634,9 +754,9 @@ bool prefill_tc_supported(int D, int BLK, int g) {
 }
 
 cudaError_t launch_prefill_tc(const CUtensorMap& tk, const CUtensorMap& tv, const PrefillParams& p, int D, int BLK,
-                              int max_len, cudaStream_t s) {
+                              int max_len, int sms, cudaStream_t s) {
   if (!prefill_tc_supported(D, BLK, p.g)) return cudaErrorInvalidValue;
-  return BLK == 64 ? launch_tc_t<64>(tk, tv, p, max_len, s) : launch_tc_t<128>(tk, tv, p, max_len, s);
+  return BLK == 64 ? launch_tc_t<64>(tk, tv, p, max_len, sms, s) : launch_tc_t<128>(tk, tv, p, max_len, sms, s);
 }
 
 }  // namespace seer

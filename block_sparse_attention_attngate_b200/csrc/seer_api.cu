@@ -418,7 +418,7 @@ seer_status seer_prefill_gt(const seer_dims_t* dims, const void* q, int32_t max_
   p.err = err_word;
   // the tcgen05 / TMEM kernel where it takes the shape, the warp-level mma kernel otherwise
   cudaError_t e = seer::prefill_tc_supported(dims->head_dim, dims->block_size, p.g)
-                      ? seer::launch_prefill_tc(tk, tv, p, dims->head_dim, dims->block_size, max_len,
+                      ? seer::launch_prefill_tc(tk, tv, p, dims->head_dim, dims->block_size, max_len, df->sms,
                                                 static_cast<cudaStream_t>(stream))
                       : seer::launch_prefill_gt(tk, tv, p, dims->head_dim, dims->block_size, max_len,
                                                 static_cast<cudaStream_t>(stream));

@@ -116,8 +116,9 @@ cudaError_t launch_prefill_gt(const CUtensorMap& tk, const CUtensorMap& tv, cons
                               int max_len, cudaStream_t s);
 // The same forward on tcgen05 / TMEM (prefill_tc.cu): head_dim 128, groups of 1, 2, 4 or 8.
 bool prefill_tc_supported(int D, int BLK, int g);
+// One persistent CTA per SM (sms = the device's SM count), items of 128 rows heaviest first.
 cudaError_t launch_prefill_tc(const CUtensorMap& tk, const CUtensorMap& tv, const PrefillParams& p, int D, int BLK,
-                              int max_len, cudaStream_t s);
+                              int max_len, int sms, cudaStream_t s);
 
 // ---------------------------------------------------------------- gate score
 struct GateParams {
