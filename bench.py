@@ -292,8 +292,11 @@ def _up(bits, dev):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
 
 
-def time_decode_alone(S, steps_, q_list, seql, stream, iters=60, warm=5):
-    """Mean device time of the sparse decode alone (eager launches rotating over the replicas)."""
+def time_decode_alone(S, steps_, q_list, seql, stream, per_graph=30, replays=4, warm=2):
+    """Mean device time of the sparse decode alone: a CUDA graph of `per_graph` consecutive launches
+    rotating over the replicas (no host work between launches: eager calls through the binding
+    cost about as much host time as a high-sparsity launch takes on the GPU), replayed `replays`
+    times after `warm` untimed replays."""
     import torch
     R = len(steps_)
 
@@ -302,17 +305,26 @@ def time_decode_alone(S, steps_, q_list, seql, stream, iters=60, warm=5):
         S.sparse_decode(st.shape, q_list[i % R], st.k, st.v, st.block_idx, st.block_cnt, seql, st.out, st.workspace,
                         st.num_split, st.lse, st.err, stream=stream)
     with torch.cuda.stream(stream):
-        for i in range(warm):
+        for i in range(R):
             one(i)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(per_graph):
+            one(i)
+    with torch.cuda.stream(stream):
+        for _ in range(warm):
+            g.replay()
     stream.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         e0.record(stream)
-        for i in range(iters):
-            one(i)
+        for _ in range(replays):
+            g.replay()
         e1.record(stream)
     e1.synchronize()
-    return e0.elapsed_time(e1) / iters * 1e3
+    del g
+    return e0.elapsed_time(e1) / (replays * per_graph) * 1e3
 
 
 def time_step_graph(steps_, q_list, seql, stream, per_graph=30, replays=8, warm=2):
@@ -787,9 +799,24 @@ def run_seer(args):
     clocks = clk.summary()
     ms_step = ranks_max(ms_step)
 
-    # ---------------- per-part device times (eager launches, same replica rotation)
+    # ---------------- per-part device times (same replica rotation).  The decode and the plan are timed
+    # from a CUDA graph of 30 consecutive launches (device time alone); the unfused helper kernels from
+    # eager calls, which the binding's host cost bounds.
     def part(fn):
         return ranks_max(timed(fn, args.steps)) * 1e3
+
+    def graph_part(fn, per_graph=30, replays=4):
+        with torch.cuda.stream(stream):
+            for i in range(R):
+                fn(i)
+        stream.synchronize()
+        g_ = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_, stream=stream):
+            for i in range(per_graph):
+                fn(i)
+        us_ = ranks_max(timed(lambda i: g_.replay(), replays)) * 1e3 / per_graph
+        del g_
+        return us_
 
     def run_decode(i):
         st = reps[i % R]["step"]
@@ -815,8 +842,8 @@ def run_seer(args):
                       cfg.budget, 0.0, k_nope=st.k_nope, valid_blocks=st.valid_blocks, w_k=w_k, logits=st.logits,
                       stream=stream)
 
-    decode_us = part(run_decode)
-    plan_us = part(run_plan)
+    decode_us = graph_part(run_decode)
+    plan_us = graph_part(run_plan)
     # the whole step from a graph of consecutive steps (no host work between launches): the default
     # two-launch form (plan, decode), and the whole step as one launch (seer_decode_step)
     two_launch_us = ranks_max(time_step_graph([rp["step"] for rp in reps], [rp["q"] for rp in reps], seqlens,
