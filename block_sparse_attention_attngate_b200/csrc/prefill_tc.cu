@@ -25,21 +25,22 @@
 //              P.V has read them) by TMA (128-byte swizzle, boxes of 64
 //              channels x b keys)
 //   warp 1     allocates TMEM; one lane issues the MMAs: S_u = Q K_u^T into
-//              TMEM S[u % 2] (M = 128 rows, N = 128 keys, K = d; both operands
-//              in shared memory) two tiles ahead -- S_{u+2} as soon as the
-//              softmax has read S_u, before P_u exists -- and O += P_u V_u into
-//              TMEM O (N = d, K = 128 keys; P read from TMEM P[u % 2], V from
-//              shared memory), each group closed by a commit to an mbarrier
+//              TMEM buffer u % 3 (M = 128 rows, N = 128 keys, K = d; both
+//              operands in shared memory) three tiles ahead -- S_{u+3} as soon
+//              as the P.V of tile u has read that buffer -- and O += P_u V_u
+//              into TMEM O (N = d, K = 128 keys; P read from TMEM, V from shared
+//              memory), each group closed by a commit to an mbarrier
 //   warps 2 .. 1 + 4 kNP: kNP threads per row (the row's TMEM lane; one
 //              thread per 128 / kNP keys of the tile, the kNP exchanging their
 //              maxima through shared memory): S by tcgen05.ld, causal mask, the
 //              row maximum of each block (stored for the targets),
-//              P = exp2(s - m_ref) as bf16 pairs into TMEM P[u % 2] by
-//              tcgen05.st (once the P.V of tile u - 2 has read that buffer, so
-//              tile u's exponentials overlap the P.V of tile u - 1),
+//              P = exp2(s - m_ref) as bf16 pairs by tcgen05.st over the first
+//              64 columns of S_u's own buffer (both parts have read it: the
+//              pair barrier), so tile u's exponentials overlap the P.V of
+//              tile u - 1 and no P buffer is waited for,
 //              V rows past the sequence zeroed (the cache may hold NaN there),
 //              at the end O / l, the LSE and the row's log2 normaliser m + log2 l
-// TMEM columns: S[0] 0-127, S[1] 128-255, O 256-383, P[0] 384-447, P[1] 448-511.
+// TMEM columns: S/P buffers 0-127, 128-255, 256-383; O 384-511.
 // A second kernel (prefill_targets_kernel, launched behind it) forms the targets from the stored
 // block maxima and normalisers: bandwidth-bound work that would otherwise hold each CTA's tensor
 // cores idle at its end.
@@ -69,7 +70,8 @@ constexpr int kNP = 2;                  // softmax threads per row (each a 128 /
 constexpr int kSW = 4 * kNP;            // softmax warps (kNP per TMEM lane quarter)
 constexpr int kVWarp = 2 + kSW;         // the V producer (after the softmax warps)
 constexpr int kThreads = (kSW + 3) * 32;
-constexpr uint32_t kTmemCols = 512;     // S[0] 0..127, S[1] 128..255, O 256..383, P[0] 384..447, P[1] 448..511
+constexpr int kSB = 3;                  // S / P buffers in TMEM (S_u and then P_u in buffer u % 3)
+constexpr uint32_t kTmemCols = 512;     // buffers 0..127, 128..255, 256..383 (P in a buffer's first 64), O 384..511
 constexpr float kLazy = 8.f;            // m_ref moves when a tile maximum exceeds it by more than this
 constexpr size_t kSmem = 1024 + kTileB /* Q */ + (size_t)(kKStages + kVStages) * kTileB /* K, V */ +
                          256 /* barriers */ + 2 * kNP * kM * 4 /* the parts' tile maxima, two tiles */ +
@@ -220,11 +222,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* k_empty = k_full + kKStages;
   uint64_t* v_full = k_empty + kKStages;
   uint64_t* v_empty = v_full + kVStages;
-  uint64_t* s_full = v_empty + kVStages;   // [2]
-  uint64_t* s_free = s_full + 2;           // [2]
-  uint64_t* p_full = s_free + 2;     // [2] P[k] written (tile u, k = u % 2)
-  uint64_t* p_free = p_full + 2;     // [2] one completion per P.V of P[k]
-  uint64_t* o_fin = p_free + 2;      // an item's last P.V done (one completion per item)
+  uint64_t* s_full = v_empty + kVStages;   // [kSB] S_u in buffer u % kSB
+  uint64_t* p_full = s_full + kSB;   // [kSB] P_u written over S_u
+  uint64_t* p_free = p_full + kSB;   // [kSB] one completion per P.V (the buffer may take S_{u+kSB})
+  uint64_t* o_fin = p_free + kSB;    // an item's last P.V done (one completion per item)
   uint64_t* o_drain = o_fin + 1;     // an item's O read out of TMEM (one completion per item)
   uint64_t* q_ready = o_drain + 1;   // an item's Q tile in shared memory (one completion per item)
   uint64_t* drain = q_ready + 1;
@@ -251,15 +252,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
-    for (int k = 0; k < 2; ++k) {
+    for (int k = 0; k < kSB; ++k) {
       mbar_init(&s_full[k], 1);
-      mbar_init(&s_free[k], kSW);
-    }
-    for (int k = 0; k < 4; ++k) mbar_init(&pbar[k], kNP);
-    for (int k = 0; k < 2; ++k) {
       mbar_init(&p_full[k], kSW);
       mbar_init(&p_free[k], 1);
     }
+    for (int k = 0; k < 4; ++k) mbar_init(&pbar[k], kNP);
     mbar_init(o_fin, 1);
     mbar_init(o_drain, kSW);
     mbar_init(q_ready, kSW);
@@ -278,9 +276,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   // TMEM columns: S[k] at 128 k, O at 256, P[k] at 384 + 64 k (computed, not indexed: a runtime index into
   // a local array would put it in local memory)
-  const uint32_t tO = tmem + 256;
-  auto tS = [tmem](uint32_t k) { return tmem + 128u * k; };
-  auto tP = [tmem](uint32_t k) { return tmem + 384u + 64u * k; };
+  const uint32_t tO = tmem + 384;
+  auto tS = [tmem](uint32_t k) { return tmem + 128u * k; };   // buffer k: S, then P in its first 64 columns
+  auto tP = [tmem](uint32_t k) { return tmem + 128u * k; };
   pdl_wait();
   pdl_trigger();
   if (blockIdx.x == 0 && tid == 0)
@@ -338,8 +336,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // O += P_m V_m (m counts tiles over every item); the item's first P.V overwrites O, once the
       // previous item's O has been read out
       auto issue_pv = [&](uint32_t m, bool first) {
-        const uint32_t sv = m % kVStages, pb = m & 1;
-        ok = ok && mbar_wait(&p_full[pb], (m >> 1) & 1) && mbar_wait(&v_full[sv], (m / kVStages) & 1);
+        const uint32_t sv = m % kVStages, pb = m % kSB;
+        ok = ok && mbar_wait(&p_full[pb], (m / kSB) & 1) && mbar_wait(&v_full[sv], (m / kVStages) & 1);
         if (first && items > 0) ok = ok && mbar_wait(o_drain, (items - 1) & 1);
         if (!ok) return;
         tc_fence_after();
@@ -350,11 +348,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(&v_empty[sv]);
         umma_commit(&p_free[pb]);
       };
-      // S_u = Q K_u^T into S[u % 2], once K_u has landed and the softmax has read S_{u-2}
+      // S_u = Q K_u^T into buffer u % kSB, once K_u has landed and P_{u-kSB} (in that buffer) has
+      // been consumed by its P.V
       auto issue_s = [&](uint32_t u) {
-        const uint32_t sk = u % kKStages, k2 = u & 1;
+        const uint32_t sk = u % kKStages, k2 = u % kSB;
         ok = ok && mbar_wait(&k_full[sk], (u / kKStages) & 1);
-        ok = ok && (u < 2 || mbar_wait(&s_free[k2], ((u >> 1) - 1) & 1));
+        ok = ok && (u < (uint32_t)kSB || mbar_wait(&p_free[k2], ((u / kSB) - 1) & 1));
         if (!ok) return;
         tc_fence_after();
         const uint32_t kb = smem_u32(kring + (size_t)sk * kTileB);
@@ -365,20 +364,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(&k_empty[sk]);
         umma_commit(&s_full[k2]);
       };
-      // Issue order within an item: S_0, S_1, then for each tile n: S_{n+2} (as soon as the softmax
-      // has read S_n, before P_n exists) and P_n V_n.  S thus runs two tiles ahead and never queues
-      // behind a P.V that waits for the softmax.
+      // Issue order within an item: S_0 .. S_{kSB-1}, then for each tile n: P_n V_n and S_{n+kSB}
+      // (into P_n's buffer once that P.V has read it).  S thus runs kSB tiles ahead of the softmax.
       for (int r = 0; r < rounds && ok; ++r) {
         const int it = tc_item_index(r);
         if (it >= n_items) continue;
         const TcItem w = tc_item(p, P, npt, it);
         if (w.nt == 0) continue;
         ok = mbar_wait(q_ready, items & 1);
-        issue_s(u0);
-        if (w.nt > 1) issue_s(u0 + 1);
+        for (int n = 0; n < w.nt && n < kSB; ++n) issue_s(u0 + n);
         for (int n = 0; n < w.nt && ok; ++n) {
-          if (n + 2 < w.nt) issue_s(u0 + n + 2);
           issue_pv(u0 + n, n == 0);
+          if (n + kSB < w.nt) issue_s(u0 + n + kSB);
         }
         if (ok) umma_commit(o_fin);
         u0 += w.nt;
@@ -442,17 +439,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* rws = p.rmax + ((size_t)w.b * p.Hq + h) * p.NB * p.T;
       float m_ref = -INFINITY, l = 0.f;
       for (int n = 0; n < w.nt && ok; ++n) {
-        const uint32_t u = u0 + n, k2 = u & 1, sv = u % kVStages;
-        ok = __all_sync(0xffffffffu, mbar_wait(&s_full[k2], (u >> 1) & 1));
+        const uint32_t u = u0 + n, k2 = u % kSB, sv = u % kVStages;
+        ok = __all_sync(0xffffffffu, mbar_wait(&s_full[k2], (u / kSB) & 1));
         if (!ok) break;
         tc_fence_after();
         float x[HK];
 #pragma unroll
         for (int c0 = 0; c0 < HK; c0 += 32) tmem_ld32(tS(k2) + lane_base + part * HK + c0, x + c0);
         tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_free[k2]);   // S[k2] may be overwritten (tile u + 2)
         // causal mask (key kt visible to row i iff kt <= min(i, L - 1)) where the tile needs one; the
         // maximum of this part (raw scores: the scale is positive)
         const int k0 = n * kKT + part * HK;     // first key of this part
@@ -472,14 +466,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         hm *= sl2;   // log2 domain
         // the parts' maxima (double-buffered by tile parity: every part has read tile u - 2's values
         // before it arrived at tile u - 1's barrier)
-        xch[(k2 * kNP + part) * kM + row] = hm;
+        // (the pair barrier also orders this thread's completed S reads before the partner's P writes
+        // over the same buffer)
+        xch[((u & 1) * kNP + part) * kM + row] = hm;
+        tc_fence_before();
         if (!warps_sync(&pbar[quarter], pph)) {
           ok = false;
           break;
         }
+        tc_fence_after();
         float pm[kNP];
 #pragma unroll
-        for (int q = 0; q < kNP; ++q) pm[q] = xch[(k2 * kNP + q) * kM + row];
+        for (int q = 0; q < kNP; ++q) pm[q] = xch[((u & 1) * kNP + q) * kM + row];
         float mx = pm[0];
 #pragma unroll
         for (int q = 1; q < kNP; ++q) mx = fmaxf(mx, pm[q]);
@@ -506,17 +504,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           move = true;
         }
         l *= alpha;
-        // P[u % 2] is free once the P.V of tile u - 2 has read it (that buffer's (u / 2)-th completion;
-        // the next one needs P of tile u, not yet written, so a parity wait is exact).  A rescale of O
-        // waits for the P.V of tile u - 1 as well (O then holds the item's earlier tiles and nothing
-        // adds to it).
-        const uint32_t pb = u & 1;
-        if (u > 1) {
-          ok = __all_sync(0xffffffffu, mbar_wait(&p_free[pb], ((u >> 1) - 1) & 1));
-          if (!ok) break;
-        }
+        // P_u goes over S_u in the same buffer (read by both parts: the pair barrier above).  A rescale
+        // of O waits for the P.V of tile u - 1 (O then holds the item's earlier tiles and nothing
+        // adds to it; that buffer's next completion needs P_{u-1+kSB}, not yet written, so a parity
+        // wait is exact).
+        const uint32_t pb = k2;
         if (__any_sync(0xffffffffu, move)) {
-          ok = __all_sync(0xffffffffu, mbar_wait(&p_free[pb ^ 1], ((u - 1) >> 1) & 1));
+          ok = __all_sync(0xffffffffu, mbar_wait(&p_free[(u - 1) % kSB], ((u - 1) / kSB) & 1));
           if (!ok) break;
           tc_fence_after();
 #pragma unroll 1
@@ -629,24 +623,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 // One CTA per (32 positions, kv head, sequence), 8 warps; lane t is position i0 + t while the
 // scores are formed (the row maxima are position-contiguous per (head, block): 128-byte loads),
 // and the block index while the rows are written (block-contiguous per position: 128-byte
-// stores).  Score of block n for position i: max over the group's heads j of exp2(r_j - c_j)
+// stores).  Score of block n for position i: max over the group's G heads j of exp2(r_j - c_j)
 // (c = m + log2 l, the row's final log2 normaliser), for the blocks holding a key at or before i,
-// normalised to sum to 1; 0 for the other blocks.  Blocks are taken kTgChunk at a time through
-// shared memory; with more blocks than one chunk the sum is a first pass of its own and each
-// chunk's scores are formed again (from L2: the CTA's maxima are a few hundred KB at most).
+// normalised to sum to 1; 0 for the other blocks.  A thread keeps kTgU blocks x G heads (up to
+// 32) of loads in flight (the maxima come from DRAM: the workspace is larger than L2).  Blocks are taken
+// kTgChunk at a time through shared memory; with more blocks than one chunk the sum is a first
+// pass of its own and each chunk's scores are formed again (from L2: the CTA's maxima are a few
+// hundred KB at most).
 constexpr int kTgPos = 32;
 constexpr int kTgWarps = 8;
 constexpr int kTgChunk = 256;
 
-template <int BLK>
-__global__ void __launch_bounds__(kTgWarps * 32)
+template <int BLK, int G>
+__global__ void __launch_bounds__(kTgWarps * 32, 2)
     prefill_targets_kernel(const __grid_constant__ PrefillParams p) {
+  constexpr int kTgU = G >= 8 ? 4 : 8;   // blocks per batch of loads (kTgU x G loads in flight per thread)
   __shared__ float vals[kTgChunk][kTgPos + 1];
   __shared__ float psum[kTgWarps][kTgPos];
   __shared__ float inv_s[kTgPos];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.z, hk = blockIdx.y, i0 = blockIdx.x * kTgPos;
-  const int g = p.g;
   pdl_wait();   // the forward's row maxima and normalisers are complete
   pdl_trigger();
   const int L = min(max(p.seqlens[b], 0), min(p.T, p.kcap));
@@ -655,35 +651,36 @@ __global__ void __launch_bounds__(kTgWarps * 32)
   const bool live = i < L;
   const int nb_i = live ? i / BLK + 1 : 0;                 // blocks with a key visible to position i
   const int nb_max = (min(i0 + kTgPos, L) - 1) / BLK + 1;  // the largest nb_i of the CTA
-  const float* r_b = p.rmax + ((size_t)b * p.Hq + (size_t)hk * g) * p.NB * p.T;
-  float c[kMaxGroup];
+  const float* r_b = p.rmax + ((size_t)b * p.Hq + (size_t)hk * G) * p.NB * p.T + i;
+  const size_t hstride = (size_t)p.NB * p.T;
+  float c[G];
 #pragma unroll
-  for (int j = 0; j < kMaxGroup; ++j)
-    c[j] = (j < g && live) ? __ldg(p.rnorm + ((size_t)b * p.Hq + (size_t)hk * g + j) * p.T + i) : 0.f;
-  // scores of blocks n0 + 8u (u = 0..3), every load issued before any use
-  auto score4 = [&](int n0, float (&v)[4]) {
-    float r[4][kMaxGroup];
+  for (int j = 0; j < G; ++j) c[j] = live ? __ldg(p.rnorm + ((size_t)b * p.Hq + (size_t)hk * G + j) * p.T + i) : 0.f;
+  // scores of blocks n0 + kTgWarps * u (u < kTgU), every load issued before any use
+  auto scores = [&](int n0, float (&v)[kTgU]) {
+    float r[kTgU][G];
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
+    for (int u = 0; u < kTgU; ++u) {
+      const int n = n0 + kTgWarps * u;
 #pragma unroll
-      for (int j = 0; j < kMaxGroup; ++j)
-        r[u][j] = (j < g && n0 + kTgWarps * u < nb_i) ? __ldcg(r_b + ((size_t)j * p.NB + n0 + kTgWarps * u) * p.T + i)
-                                                       : -INFINITY;
+      for (int j = 0; j < G; ++j) r[u][j] = n < nb_i ? __ldcg(r_b + j * hstride + (size_t)n * p.T) : -INFINITY;
+    }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kTgU; ++u) {
       v[u] = 0.f;
+      if (n0 + kTgWarps * u < nb_i) {
 #pragma unroll
-      for (int j = 0; j < kMaxGroup; ++j)
-        if (j < g && n0 + kTgWarps * u < nb_i) v[u] = fmaxf(v[u], exp2f(r[u][j] - c[j]));
+        for (int j = 0; j < G; ++j) v[u] = fmaxf(v[u], exp2f(r[u][j] - c[j]));
+      }
     }
   };
   // chunk [n_lo, n_hi): scores into vals (and into the sum when `add`)
   auto fill = [&](int n_lo, int n_hi, bool add, float& part) {
-    for (int n0 = n_lo + warp; n0 < n_hi; n0 += 4 * kTgWarps) {
-      float v[4];
-      score4(n0, v);
+    for (int n0 = n_lo + warp; n0 < n_hi; n0 += kTgU * kTgWarps) {
+      float v[kTgU];
+      scores(n0, v);
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < kTgU; ++u) {
         const int n = n0 + kTgWarps * u;
         if (n < n_hi) {
           vals[n - n_lo][lane] = v[u];
@@ -697,19 +694,20 @@ __global__ void __launch_bounds__(kTgWarps * 32)
   if (one) {
     fill(0, nb_max, true, part);
   } else {
-    for (int n0 = warp; n0 < nb_max; n0 += 4 * kTgWarps) {
-      float v[4];
-      score4(n0, v);
-      part += (v[0] + v[1]) + (v[2] + v[3]);   // blocks past nb_i score 0
+    for (int n0 = warp; n0 < nb_max; n0 += kTgU * kTgWarps) {
+      float v[kTgU];
+      scores(n0, v);
+#pragma unroll
+      for (int u = 0; u < kTgU; ++u) part += v[u];   // blocks past nb_i score 0
     }
   }
   psum[warp][lane] = part;
   __syncthreads();
   if (warp == 0) {
-    float s = 0.f;
+    float sum = 0.f;
 #pragma unroll
-    for (int w = 0; w < kTgWarps; ++w) s += psum[w][lane];
-    inv_s[lane] = s > 0.f ? 1.f / s : 0.f;
+    for (int w = 0; w < kTgWarps; ++w) sum += psum[w][lane];
+    inv_s[lane] = sum > 0.f ? 1.f / sum : 0.f;
   }
   __syncthreads();
   float* gt_b = p.gt + ((size_t)b * p.Hkv + hk) * p.T * p.NB;
@@ -732,6 +730,18 @@ __global__ void __launch_bounds__(kTgWarps * 32)
 }
 
 template <int BLK>
+cudaError_t launch_targets(const PrefillParams& p, int max_len, cudaStream_t st) {
+  const dim3 tgrid((max_len + kTgPos - 1) / kTgPos, p.Hkv, p.B);
+  const dim3 blk(kTgWarps * 32);
+  switch (p.g) {
+    case 1: return launch_pdl(prefill_targets_kernel<BLK, 1>, tgrid, blk, 0, st, p);
+    case 2: return launch_pdl(prefill_targets_kernel<BLK, 2>, tgrid, blk, 0, st, p);
+    case 4: return launch_pdl(prefill_targets_kernel<BLK, 4>, tgrid, blk, 0, st, p);
+    default: return launch_pdl(prefill_targets_kernel<BLK, 8>, tgrid, blk, 0, st, p);
+  }
+}
+
+template <int BLK>
 cudaError_t launch_tc_t(const CUtensorMap& tk, const CUtensorMap& tv, const PrefillParams& p, int max_len,
                         int sms, cudaStream_t st) {
   auto kern = prefill_tc_kernel<BLK>;
@@ -743,8 +753,7 @@ cudaError_t launch_tc_t(const CUtensorMap& tk, const CUtensorMap& tv, const Pref
   const dim3 grid((unsigned)std::min<long long>(items, std::max(sms, 1)));
   e = launch_pdl(kern, grid, dim3(kThreads), kSmem, st, tk, tv, p);
   if (e != cudaSuccess) return e;
-  const dim3 tgrid((max_len + kTgPos - 1) / kTgPos, p.Hkv, p.B);
-  return launch_pdl(prefill_targets_kernel<BLK>, tgrid, dim3(kTgWarps * 32), 0, st, p);
+  return launch_targets<BLK>(p, max_len, st);
 }
 
 }  // namespace
