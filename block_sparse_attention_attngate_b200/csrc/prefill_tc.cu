@@ -635,7 +635,7 @@ constexpr int kTgWarps = 8;
 constexpr int kTgChunk = 256;
 
 template <int BLK, int G>
-__global__ void __launch_bounds__(kTgWarps * 32, 2)
+__global__ void __launch_bounds__(kTgWarps * 32, 3)
     prefill_targets_kernel(const __grid_constant__ PrefillParams p) {
   constexpr int kTgU = G >= 8 ? 4 : 8;   // blocks per batch of loads (kTgU x G loads in flight per thread)
   __shared__ float vals[kTgChunk][kTgPos + 1];
@@ -656,22 +656,24 @@ __global__ void __launch_bounds__(kTgWarps * 32, 2)
   float c[G];
 #pragma unroll
   for (int j = 0; j < G; ++j) c[j] = live ? __ldg(p.rnorm + ((size_t)b * p.Hq + (size_t)hk * G + j) * p.T + i) : 0.f;
-  // scores of blocks n0 + kTgWarps * u (u < kTgU), every load issued before any use
+  // scores of blocks n0 + kTgWarps * u (u < kTgU), every load issued before any use (one 64-bit
+  // offset per block; the heads' offsets are fixed multiples of the head stride)
   auto scores = [&](int n0, float (&v)[kTgU]) {
     float r[kTgU][G];
 #pragma unroll
     for (int u = 0; u < kTgU; ++u) {
       const int n = n0 + kTgWarps * u;
+      const bool in = n < nb_i;
+      const float* rn = r_b + (size_t)n * p.T;
 #pragma unroll
-      for (int j = 0; j < G; ++j) r[u][j] = n < nb_i ? __ldcg(r_b + j * hstride + (size_t)n * p.T) : -INFINITY;
+      for (int j = 0; j < G; ++j) r[u][j] = in ? __ldcg(rn + j * hstride) : -INFINITY;
     }
 #pragma unroll
     for (int u = 0; u < kTgU; ++u) {
-      v[u] = 0.f;
-      if (n0 + kTgWarps * u < nb_i) {
+      float m = 0.f;
 #pragma unroll
-        for (int j = 0; j < G; ++j) v[u] = fmaxf(v[u], exp2f(r[u][j] - c[j]));
-      }
+      for (int j = 0; j < G; ++j) m = fmaxf(m, ex2(r[u][j] - c[j]));   // masked blocks: ex2(-inf) = 0
+      v[u] = m;
     }
   };
   // chunk [n_lo, n_hi): scores into vals (and into the sum when `add`)
