@@ -75,9 +75,25 @@ def _check_case(d, blk, g, Hkv, nan_tail, lengths=None):
 
 
 @pytest.mark.parametrize("d,blk,g,Hkv", [(128, 64, 4, 2), (128, 128, 2, 2), (64, 64, 8, 1), (64, 128, 1, 3),
-                                         (128, 64, 5, 1)])
+                                         (128, 64, 5, 1), (128, 64, 1, 3), (128, 64, 8, 1), (128, 128, 8, 1),
+                                         (128, 128, 1, 2)])
 def test_prefill_gt_vs_oracle(d, blk, g, Hkv):
+    """head_dim 128 with g in {1, 2, 4, 8} runs the tcgen05 forward (every group size, both block
+    sizes); head_dim 64 and g = 5 the warp-level mma one."""
     _check_case(d, blk, g, Hkv, nan_tail=False)
+
+
+@pytest.mark.parametrize("d,blk,g,Hkv", [(128, 64, 4, 2), (128, 128, 8, 1), (64, 64, 2, 2)])
+def test_prefill_gt_nan_past_the_length(d, blk, g, Hkv):
+    """q, K and V hold NaN at every position past each sequence's length: nothing of it may reach
+    the outputs, the LSEs or the targets (rows, keys and V rows past L are masked or zeroed)."""
+    _check_case(d, blk, g, Hkv, nan_tail=True)
+
+
+def test_prefill_gt_empty_and_one_token():
+    """Sequences of 0 and 1 tokens beside a longer one (tcgen05 path): the empty one writes nothing;
+    a one-token row attends to itself only (its target is the single block, 1.0)."""
+    _check_case(128, 64, 4, 1, nan_tail=True, lengths=[0, 1, 200])
 
 
 def test_prefill_rescales_when_later_keys_dominate():
